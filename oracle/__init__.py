@@ -1,0 +1,234 @@
+"""fp8bq oracle: numpy/ctypes front end of the plain CPU library in fp8bq_oracle.c.
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import this package.  It
+imports nothing from the CUDA path and the CUDA path imports nothing from it.
+
+Method source: "NVIDIA NeMo RL Achieves 48% Speedup With End-to-End FP8
+Precision Training", section "Technical breakthrough" (block-wise E4M3, 128x128
+weight tiles, 1x128 activation tiles), section "Real-world performance gains"
+(per-step scale recalibration) and section "Why this matters for AI economics"
+(power-of-2 scales).  Each wrapper below names the C function it calls; the C
+file states every reading taken where the pages are silent.
+
+Arrays: bf16 data travels as ``np.uint16`` bit patterns, codes as ``np.uint8``,
+scales as ``np.float32``, GEMM results as ``np.float64``.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+SCALE_FP32 = 0
+SCALE_POW2 = 1
+
+_lib = None
+
+
+def lib():
+    """Load (building first if needed) liboracle.so."""
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        L.o_e4m3_decode.restype = ctypes.c_double
+        L.o_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.o_e4m3_encode.restype = ctypes.c_uint8
+        L.o_e4m3_encode.argtypes = [ctypes.c_float]
+        L.o_e4m3_encode_nearest.restype = ctypes.c_uint8
+        L.o_e4m3_encode_nearest.argtypes = [ctypes.c_float]
+        L.o_sweep_encoders.restype = ctypes.c_uint64
+        L.o_sweep_encoders.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint32)]
+        L.o_encode_patterns.restype = None
+        L.o_encode_patterns.argtypes = [ctypes.c_uint64, ctypes.c_uint64, P]
+        L.o_encode_array.restype = None
+        L.o_encode_array.argtypes = [P, I64, P]
+        L.o_bf16_to_f32.restype = ctypes.c_float
+        L.o_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        L.o_scale.restype = ctypes.c_float
+        L.o_scale.argtypes = [ctypes.c_float, ctypes.c_int]
+        L.o_quant_act.restype = None
+        L.o_quant_act.argtypes = [P, I64, I64, I64, P, I64, P, I64, ctypes.c_int]
+        L.o_quant_weight.restype = None
+        L.o_quant_weight.argtypes = [P, I64, I64, I64, P, I64, P, ctypes.c_int]
+        L.o_dequant_act.restype = None
+        L.o_dequant_act.argtypes = [P, I64, I64, I64, P, I64, P]
+        L.o_dequant_weight.restype = None
+        L.o_dequant_weight.argtypes = [P, I64, I64, I64, P, P]
+        for name in ("o_gemm_rows", "o_gemm_blockint_rows"):
+            f = getattr(L, name)
+            f.restype = None
+            f.argtypes = [P, I64, P, I64, P, I64, P, I64, I64, I64, P, I64, P]
+        L.o_grouped_gemm_rows.restype = None
+        L.o_grouped_gemm_rows.argtypes = [P, I64, P, I64, P, P, P, I64, I64, I64, P, I64, P]
+        L.o_f64_to_bf16.restype = ctypes.c_uint16
+        L.o_f64_to_bf16.argtypes = [ctypes.c_double]
+        L.o_f64_to_bf16_array.restype = None
+        L.o_f64_to_bf16_array.argtypes = [P, I64, P]
+        L.o_num_threads.restype = ctypes.c_int
+        L.o_num_threads.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    a = np.asarray(a)
+    if a.dtype != dtype:
+        raise TypeError("expected %s, got %s" % (np.dtype(dtype), a.dtype))
+    return np.ascontiguousarray(a)
+
+
+def num_threads():
+    return lib().o_num_threads()
+
+
+# --- E4M3 --------------------------------------------------------------------
+
+def e4m3_decode(code):
+    return lib().o_e4m3_decode(int(code))
+
+
+def e4m3_decode_table():
+    """float64[256]: the exact value of every code (NaN for 0x7F / 0xFF)."""
+    return np.array([e4m3_decode(c) for c in range(256)], dtype=np.float64)
+
+
+def e4m3_encode(v):
+    """Encoder A (round to nearest even, saturate at 448) of one float."""
+    return lib().o_e4m3_encode(float(np.float32(v)))
+
+
+def e4m3_encode_nearest(v):
+    """Encoder B (nearest value by brute force, ties to even code)."""
+    return lib().o_e4m3_encode_nearest(float(np.float32(v)))
+
+
+def e4m3_encode_array(v):
+    v = _c(np.asarray(v, dtype=np.float32), np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().o_encode_array(_p(v), v.size, _p(out))
+    return out
+
+
+def encode_patterns(start, count):
+    """Encoder A over the fp32 bit patterns [start, start + count)."""
+    out = np.empty(count, dtype=np.uint8)
+    lib().o_encode_patterns(start, count, _p(out))
+    return out
+
+
+def sweep_encoders(start, count):
+    """(mismatches, first mismatching pattern) of encoder A vs B over a pattern range."""
+    first = ctypes.c_uint32(0)
+    bad = lib().o_sweep_encoders(start, count, ctypes.byref(first))
+    return int(bad), int(first.value)
+
+
+# --- scales and quantizers ----------------------------------------------------
+
+def scale(amax, mode):
+    return lib().o_scale(float(np.float32(amax)), int(mode))
+
+
+def bf16_to_f32(bits):
+    """Exact widening of bf16 bit patterns (uint16) to float32."""
+    bits = np.asarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def quant_act(x_bits, mode, ldsa=None):
+    """1x128 activation quantization of bf16 bits [M, K] -> (codes [M, K], sa [KB, ldsa])."""
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    KB = (K + 127) // 128
+    ldsa = M if ldsa is None else ldsa
+    q = np.empty((M, K), dtype=np.uint8)
+    sa = np.zeros((KB, ldsa), dtype=np.float32)
+    lib().o_quant_act(_p(x), M, K, K, _p(q), K, _p(sa), ldsa, int(mode))
+    return q, sa
+
+
+def quant_weight(w_bits, mode):
+    """128x128 weight quantization of bf16 bits [N, K] -> (codes [N, K], sw [NB, KB])."""
+    w = _c(w_bits, np.uint16)
+    N, K = w.shape
+    NB, KB = (N + 127) // 128, (K + 127) // 128
+    q = np.empty((N, K), dtype=np.uint8)
+    sw = np.empty((NB, KB), dtype=np.float32)
+    lib().o_quant_weight(_p(w), N, K, K, _p(q), K, _p(sw), int(mode))
+    return q, sw
+
+
+def dequant_act(q, sa):
+    q = _c(q, np.uint8)
+    sa = _c(sa, np.float32)
+    M, K = q.shape
+    out = np.empty((M, K), dtype=np.float64)
+    lib().o_dequant_act(_p(q), M, K, K, _p(sa), sa.shape[1], _p(out))
+    return out
+
+
+def dequant_weight(q, sw):
+    q = _c(q, np.uint8)
+    sw = _c(sw, np.float32)
+    N, K = q.shape
+    out = np.empty((N, K), dtype=np.float64)
+    lib().o_dequant_weight(_p(q), N, K, K, _p(sw), _p(out))
+    return out
+
+
+def gemm(qa, sa, qw, sw, rows=None, blockint=False):
+    """Y64 = deq(qa) . deq(qw)^T in double (rows: optional subset of output rows)."""
+    qa = _c(qa, np.uint8)
+    sa = _c(sa, np.float32)
+    qw = _c(qw, np.uint8)
+    sw = _c(sw, np.float32)
+    M, K = qa.shape
+    N = qw.shape[0]
+    if rows is None:
+        r = None
+        R = M
+    else:
+        r = _c(np.asarray(rows, dtype=np.int64), np.int64)
+        R = r.size
+    y = np.empty((R, N), dtype=np.float64)
+    f = lib().o_gemm_blockint_rows if blockint else lib().o_gemm_rows
+    f(_p(qa), K, _p(sa), sa.shape[1], _p(qw), K, _p(sw), M, N, K,
+      None if r is None else _p(r), R, _p(y))
+    return y
+
+
+def grouped_gemm(qa, sa, qw, sw, offsets, rows=None):
+    """Per-expert Y64 for row-sorted activations; qw [E, N, K], sw [E, NB, KB]."""
+    qa = _c(qa, np.uint8)
+    sa = _c(sa, np.float32)
+    qw = _c(qw, np.uint8)
+    sw = _c(sw, np.float32)
+    off = _c(np.asarray(offsets, dtype=np.int64), np.int64)
+    E, N, K = qw.shape
+    if rows is None:
+        r = None
+        R = int(off[-1])
+    else:
+        r = _c(np.asarray(rows, dtype=np.int64), np.int64)
+        R = r.size
+    y = np.empty((R, N), dtype=np.float64)
+    lib().o_grouped_gemm_rows(_p(qa), K, _p(sa), sa.shape[1], _p(qw), _p(sw), _p(off), E, N, K,
+                              None if r is None else _p(r), R, _p(y))
+    return y
+
+
+def f64_to_bf16(v):
+    """Round doubles to bf16 (nearest even), returned as uint16 bit patterns."""
+    v = _c(np.asarray(v, dtype=np.float64), np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    lib().o_f64_to_bf16_array(_p(v), v.size, _p(out))
+    return out
