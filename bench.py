@@ -1,0 +1,428 @@
+"""Benchmark of the block-wise FP8 linear layer hot path on B200.
+
+One step = one pass of the whole hot path over one Llama-3.1-8B-shaped layer
+at M = 8192 prefill tokens (4 x 2048), FP32 block scales:
+  - per-step recalibration of the layer's four weight tensors
+    (QKV 6144x4096, O 4096x4096, gate+up 28672x4096, down 4096x14336) into
+    E4M3 codes + 128x128 scales, one launch;
+  - for each of the four linears: 1x128 quantization of its bf16 input and the
+    block-scaled FP8 GEMM (FP32 promotion, bf16 out).
+Metric: FP8 GEMM throughput of the step in TFLOP/s (GEMM FLOPs of the four
+linears / step time, so the quantization and recalibration time counts
+against it).  Per-row figures (quantize / recalibrate GB/s, each GEMM's
+TFLOP/s) are reported under "rows".
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun (N > 1) every rank runs the same single-GPU workload on its own
+GPU (replicas: the path has no exchange step); value = all ranks' FLOPs / the
+slowest rank's time.
+
+--impl reference times the CPU oracle (oracle/) on the host cores on a bounded
+sample of the same workload (the slow reference program; parity and the
+roofline fraction are the headline, not this ratio).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import fp8bq_workloads as wl  # noqa: E402
+
+METRIC = "block-scaled FP8 GEMM TFLOP/s (% of dense FP8 peak); quantize/recal GB/s (% HBM)"
+WORKLOAD = "llama3.1-8b-shaped prefill layer: 4 linears (qkv, o, gate_up, down) at M=8192 tokens, fp32 block scales"
+NAMES = list(wl.LLAMA8B_SHAPES)
+M_TOKENS = wl.PREFILL_TOKENS
+LAUNCHES_PER_STEP = 1 + 2 * len(NAMES)        # recalibrate + (quant_act + gemm) per linear
+
+
+def gemm_flops_step():
+    return sum(2.0 * M_TOKENS * N * K for N, K in wl.LLAMA8B_SHAPES.values())
+
+
+def quant_act_bytes(M, K):
+    """bf16 in + E4M3 out + one fp32 scale per 128 elements."""
+    return M * K * 2 + M * K + M * ((K + 127) // 128) * 4
+
+
+def recal_bytes(N, K):
+    return N * K * 2 + N * K + ((N + 127) // 128) * ((K + 127) // 128) * 4
+
+
+def gemm_bytes(M, N, K):
+    return M * K + N * K + M * N * 2 + M * (K // 128) * 4 + ((N + 127) // 128) * (K // 128) * 4
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "device.cuh"):
+        h.update(open(os.path.join(ROOT, "fp8_block_scaled_fp8bq_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu summary, if the kernel is unchanged."""
+    p = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_sha") != kernel_source_sha():
+        return None
+    return d.get("dram_bytes_per_launch_step_avg")
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clocks_setting"}
+
+    def __init__(self, device_index, period_s=0.02):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                self.reasons |= self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if self.nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- our arm
+class LayerStep:
+    """Device buffers and the launch sequence of one step."""
+
+    def __init__(self, fq, device, seed=0, mode=0):
+        self.fq = fq
+        self.mode = mode
+        self.x, self.w, self.q_w, self.s_w, self.q_a, self.s_a, self.y = {}, {}, {}, {}, {}, {}, {}
+        layer = wl.llama_layer(seed=seed, M=M_TOKENS, device=device)
+        for name, (N, K) in wl.LLAMA8B_SHAPES.items():
+            x, w = layer[name]
+            self.x[name], self.w[name] = x, w
+            self.q_w[name] = torch.empty((N, K), dtype=torch.uint8, device=device)
+            self.s_w[name] = torch.empty((fq.ceil_div(N, 128), fq.ceil_div(K, 128)), dtype=torch.float32,
+                                         device=device)
+            self.q_a[name] = torch.empty((M_TOKENS, K), dtype=torch.uint8, device=device)
+            self.s_a[name] = torch.empty(fq.act_scale_shape(M_TOKENS, K), dtype=torch.float32, device=device)
+            self.y[name] = torch.empty((M_TOKENS, N), dtype=torch.bfloat16, device=device)
+        self.recal_list = [(self.w[n], self.q_w[n], self.s_w[n]) for n in NAMES]
+
+    def run(self, events=None):
+        """One step.  events: optional dict name -> list of (start, end) CUDA events to record."""
+        fq = self.fq
+
+        def ev(key):
+            if events is None:
+                return None
+            e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            events.setdefault(key, []).append(e)
+            return e
+
+        e = ev("recalibrate")
+        if e:
+            e[0].record()
+        fq.recalibrate(self.recal_list, self.mode)
+        if e:
+            e[1].record()
+        for name in NAMES:
+            e = ev("quant_act:" + name)
+            if e:
+                e[0].record()
+            fq.quant_act(self.x[name], self.mode, q=self.q_a[name], sa=self.s_a[name])
+            if e:
+                e[1].record()
+            e = ev("gemm:" + name)
+            if e:
+                e[0].record()
+            fq.gemm(self.q_a[name], self.s_a[name], self.q_w[name], self.s_w[name], self.mode, out=self.y[name])
+            if e:
+                e[1].record()
+
+
+def timed_steps(step, K, W, rank_sync):
+    """Run W warm-up steps, then K timed steps; returns (seconds, events)."""
+    for _ in range(W):
+        step.run()
+    torch.cuda.synchronize()
+    rank_sync()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    events = {}
+    start.record()
+    for _ in range(K):
+        step.run(events)
+    end.record()
+    torch.cuda.synchronize()
+    rank_sync()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / 1e3, events
+
+
+def e2e_steps(fq, step, K, rank_sync):
+    """The same step with inputs copied from pinned host memory and outputs copied back, every step."""
+    host_x = {n: step.x[n].cpu().pin_memory() for n in NAMES}
+    host_w = {n: step.w[n].cpu().pin_memory() for n in NAMES}
+    host_y = {n: torch.empty(step.y[n].shape, dtype=torch.bfloat16).pin_memory() for n in NAMES}
+    h2d = sum(t.numel() * t.element_size() for t in list(host_x.values()) + list(host_w.values()))
+    d2h = sum(t.numel() * t.element_size() for t in host_y.values())
+
+    def one():
+        for n in NAMES:
+            step.x[n].copy_(host_x[n], non_blocking=True)
+            step.w[n].copy_(host_w[n], non_blocking=True)
+        step.run()
+        for n in NAMES:
+            host_y[n].copy_(step.y[n], non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    rank_sync()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(K):
+        one()
+    t1.record()
+    torch.cuda.synchronize()
+    rank_sync()
+    return t0.elapsed_time(t1) / 1e3, h2d, d2h
+
+
+def cpu_baseline_oracle(budget_s=15.0):
+    """The oracle on a bounded sample of the step, on the host cores.
+
+    Sample: quantization of R rows of each linear's input, the oracle GEMM of
+    those rows against the full weight, and the 128x128 quantization of the
+    full weight; the time of a full step is extrapolated (rows scale
+    linearly) and the metric is GEMM FLOPs / extrapolated step time.
+    """
+    import oracle
+    R = max(1, oracle.num_threads())
+    t_weight = 0.0
+    t_rows = 0.0
+    for i, (name, (N, K)) in enumerate(wl.LLAMA8B_SHAPES.items()):
+        x = wl.activations(R, K, seed=100 + i)
+        w = wl.weights(N, K, seed=200 + i)
+        xb = x.view(torch.int16).numpy().view(np.uint16)
+        wb = w.view(torch.int16).numpy().view(np.uint16)
+        t0 = time.perf_counter()
+        qw, sw = oracle.quant_weight(wb, 0)
+        t1 = time.perf_counter()
+        qa, sa = oracle.quant_act(xb, 0)
+        oracle.gemm(qa, sa, qw, sw)
+        t2 = time.perf_counter()
+        t_weight += t1 - t0
+        t_rows += t2 - t1
+    step_s = t_weight + t_rows * (M_TOKENS / R)
+    return {"value": gemm_flops_step() / step_s / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "%d rows of each of the 4 linears (act quant + FP64 GEMM) plus the full 128x128 weight "
+                      "quantization; step time extrapolated to M=%d rows" % (R, M_TOKENS),
+            "sample_seconds": round(t_weight + t_rows, 2)}
+
+
+def ours(args):
+    import torch.distributed as dist
+    import fp8_block_scaled_fp8bq_b200 as fq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    fq.lib()
+
+    def rank_sync():
+        if world > 1:
+            dist.barrier()
+
+    step = LayerStep(fq, device)
+    with ClockSampler(local) as clk:
+        secs, events = timed_steps(step, args.steps, args.warmup, rank_sync)
+    if world > 1:
+        t = torch.tensor([secs], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        secs = float(t.item())
+    K = args.steps
+    flops = gemm_flops_step()
+    value = world * flops * K / secs / 1e12
+
+    # per-row figures from the per-launch events
+    def avg_ms(key):
+        return sum(a.elapsed_time(b) for a, b in events[key]) / len(events[key])
+
+    peaks = load_peaks()
+    sustained = secs > 1.0
+    bf16_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    fp8_peak = 2.0 * bf16_peak
+    rows = {}
+    gemm_ms_total = 0.0
+    for name, (N, K_) in wl.LLAMA8B_SHAPES.items():
+        ms = avg_ms("gemm:" + name)
+        gemm_ms_total += ms
+        tf = 2.0 * M_TOKENS * N * K_ / (ms / 1e3) / 1e12
+        rows["gemm:" + name] = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac_fp8_peak": round(tf / fp8_peak, 3)}
+        qms = avg_ms("quant_act:" + name)
+        gbs = quant_act_bytes(M_TOKENS, K_) / (qms / 1e3) / 1e9
+        rows["quant_act:" + name] = {"ms": round(qms, 4), "gbs": round(gbs, 1),
+                                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+    rms = avg_ms("recalibrate")
+    rb = sum(recal_bytes(N, K_) for N, K_ in wl.LLAMA8B_SHAPES.values())
+    rows["recalibrate:layer"] = {"ms": round(rms, 4), "gbs": round(rb / (rms / 1e3) / 1e9, 1),
+                                 "frac_hbm": round(rb / (rms / 1e3) / 1e9 / peaks["hbm_gbs"], 3)}
+    achieved = flops / (gemm_ms_total / 1e3) / 1e12
+    traffic = committed_traffic()
+    roofline = {"bound": "tensor", "kernel": "gemm_promote_kernel (4 launches per step, averaged)",
+                "achieved": round(achieved, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / fp8_peak, 4), "traffic": traffic,
+                "peak_note": "%s bf16 %s x 2 (nominal fp8:bf16 ratio)" % (
+                    "of measured" if peaks["source"] == "measured" else "of fallback",
+                    "sustained" if sustained else "burst")}
+
+    # end to end: host buffers, copies inside the timed region
+    Ke = max(1, min(K, 10))
+    e2e_s, h2d, d2h = e2e_steps(fq, step, Ke, rank_sync)
+    if world > 1:
+        t = torch.tensor([e2e_s], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    e2e = {"value": round(world * flops * Ke / e2e_s / 1e12, 2), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": Ke}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(secs / K * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 x e4m3 -> f32 accumulate, bf16 out",
+            "data": "synthetic (seeded; Llama-3.1-8B shapes, no model weights)",
+            "config": {"workload": WORKLOAD, "tokens": M_TOKENS,
+                       "shapes_NK": {n: list(s) for n, s in wl.LLAMA8B_SHAPES.items()}, "scale_mode": "fp32",
+                       "l2": "inputs larger than L2 (about 2 GB touched per step vs 126 MB L2); no flush",
+                       "parallelism": "replicas" if world > 1 else "single gpu"},
+            "roofline": roofline, "rows": rows, "e2e": e2e,
+            "gpu_launches": LAUNCHES_PER_STEP * K, "clocks": clk.summary(),
+        }
+        if world == 1:
+            line["cpu_baseline"] = cpu_baseline_oracle()
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def reference(args):
+    """The oracle as it stands, on the host cores, K steps of a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    R = max(1, min(32, oracle.num_threads()))
+    data = []
+    for i, (name, (N, K)) in enumerate(wl.LLAMA8B_SHAPES.items()):
+        x = wl.activations(R, K, seed=100 + i).view(torch.int16).numpy().view(np.uint16)
+        # the weight sample: 128-row block rows of W (all of K), enough for every thread
+        nrows = min(N, 128 * max(1, min(8, R // 2)))
+        w = wl.weights(nrows, K, seed=200 + i).view(torch.int16).numpy().view(np.uint16)
+        data.append((x, w, N, K, nrows))
+
+    def one_step():
+        flops = 0.0
+        for x, w, N, K, nrows in data:
+            qw, sw = oracle.quant_weight(w, 0)
+            qa, sa = oracle.quant_act(x, 0)
+            oracle.gemm(qa, sa, qw, sw)
+            flops += 2.0 * x.shape[0] * nrows * K
+        return flops
+
+    for _ in range(args.warmup):
+        one_step()
+    t0 = time.perf_counter()
+    flops = 0.0
+    for _ in range(args.steps):
+        flops += one_step()
+    secs = time.perf_counter() - t0
+    value = flops / secs / 1e12
+    sample = ("per step: %d rows of each linear's input (1x128 quant) times a %d-row block of its weight "
+              "(128x128 quant + FP64 GEMM)" % (R, data[0][4]))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "tokens": M_TOKENS},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        reference(args)
+    else:
+        ours(args)
+
+
+if __name__ == "__main__":
+    main()

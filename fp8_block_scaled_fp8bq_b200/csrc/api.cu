@@ -1,0 +1,208 @@
+// C ABI of libfp8bq: argument validation, status codes, device error word,
+// TMA descriptor encoding.  Every entry point checks its arguments before it
+// launches anything, and never throws.
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "device.cuh"
+#include "internal.h"
+
+namespace fp8bq {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices] = {0};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+thread_local char g_last_cuda_error[256] = {0};
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) return 0;
+  return d;
+}
+
+}  // namespace
+
+int num_sms() {
+  int d = current_device();
+  if (d < 0 || d >= kMaxDevices) d = 0;
+  if (g_sms[d] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0) n = 148;
+    g_sms[d] = n;
+  }
+  return g_sms[d];
+}
+
+fp8bq_status cuda_fail(cudaError_t e, const char *what) {
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", what, cudaGetErrorString(e));
+  return FP8BQ_ERR_CUDA;
+}
+
+fp8bq_status check_launch(const char *what) {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FP8BQ_OK : cuda_fail(e, what);
+}
+
+bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
+                  uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  std::call_once(g_encode_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  if (g_encode == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = g_encode(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace fp8bq
+
+using namespace fp8bq;
+
+namespace {
+
+bool bad_mode(int mode) { return mode != FP8BQ_SCALE_FP32 && mode != FP8BQ_SCALE_POW2; }
+
+constexpr int64_t kMaxDim = (int64_t)1 << 31;
+
+fp8bq_status check_gemm_operands(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                                 int64_t ldw, const float *sw, const void *y, int64_t ldy, int64_t M, int64_t N,
+                                 int64_t K, int mode) {
+  if (M < 0 || N < 0 || K < 0 || bad_mode(mode)) return FP8BQ_ERR_INVALID_ARG;
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return FP8BQ_OK;
+  if (y == nullptr || ldy < N || !aligned(y, 16) || ldy % 8 != 0) return FP8BQ_ERR_INVALID_ARG;
+  if (K == 0) return FP8BQ_OK;
+  if (K % 128 != 0) return FP8BQ_ERR_UNSUPPORTED;
+  if (!qa || !sa || !qw || !sw) return FP8BQ_ERR_INVALID_ARG;
+  if (lda < K || ldw < K || ldsa < M) return FP8BQ_ERR_INVALID_ARG;
+  if (!aligned(qa, 16) || !aligned(qw, 16) || lda % 16 != 0 || ldw % 16 != 0) return FP8BQ_ERR_INVALID_ARG;
+  if (!aligned(sa, 16) || !aligned(sw, 4) || ldsa % 4 != 0) return FP8BQ_ERR_INVALID_ARG;
+  return FP8BQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp8bq_version(void) { return 100; }
+
+const char *fp8bq_status_string(fp8bq_status s) {
+  switch (s) {
+    case FP8BQ_OK: return "FP8BQ_OK";
+    case FP8BQ_ERR_INVALID_ARG: return "FP8BQ_ERR_INVALID_ARG";
+    case FP8BQ_ERR_UNSUPPORTED: return "FP8BQ_ERR_UNSUPPORTED";
+    case FP8BQ_ERR_CUDA: return "FP8BQ_ERR_CUDA";
+    case FP8BQ_ERR_WORKSPACE: return "FP8BQ_ERR_WORKSPACE";
+    case FP8BQ_ERR_TIMEOUT: return "FP8BQ_ERR_TIMEOUT";
+  }
+  return "FP8BQ_ERR_UNKNOWN";
+}
+
+const char *fp8bq_last_cuda_error(void) { return g_last_cuda_error; }
+
+fp8bq_status fp8bq_get_device_error(uint64_t *code) {
+  unsigned long long v = 0, w = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  cudaError_t (*takers[])(unsigned long long *) = {take_device_error_gemm};
+  for (auto take : takers) {
+    e = take(&w);
+    if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+    if (v == 0) v = w;
+  }
+  if (code) *code = v;
+  return v ? FP8BQ_ERR_TIMEOUT : FP8BQ_OK;
+}
+
+fp8bq_status fp8bq_e4m3_encode(const float *x, int64_t n, uint8_t *q, void *stream) {
+  if (n < 0) return FP8BQ_ERR_INVALID_ARG;
+  if (n == 0) return FP8BQ_OK;
+  if (!x || !q || !aligned(x, 16) || !aligned(q, 4)) return FP8BQ_ERR_INVALID_ARG;
+  return launch_encode(x, n, q, static_cast<cudaStream_t>(stream));
+}
+
+fp8bq_status fp8bq_quant_act(const void *x, int64_t M, int64_t K, int64_t ldx, uint8_t *q, int64_t ldq, float *sa,
+                             int64_t ldsa, int mode, void *stream) {
+  if (M < 0 || K < 0 || bad_mode(mode)) return FP8BQ_ERR_INVALID_ARG;
+  if (M == 0 || K == 0) return FP8BQ_OK;
+  if (!x || !q || !sa) return FP8BQ_ERR_INVALID_ARG;
+  if (ldx < K || ldq < K || ldsa < M) return FP8BQ_ERR_INVALID_ARG;
+  if (!aligned(x, 2) || !aligned(sa, 4)) return FP8BQ_ERR_INVALID_ARG;
+  return launch_quant_act(x, M, K, ldx, q, ldq, sa, ldsa, mode, static_cast<cudaStream_t>(stream));
+}
+
+static fp8bq_status check_weight_desc(const fp8bq_weight_desc &d) {
+  if (d.N < 0 || d.K < 0) return FP8BQ_ERR_INVALID_ARG;
+  if (d.N == 0 || d.K == 0) return FP8BQ_OK;
+  if (!d.w || !d.q || !d.s) return FP8BQ_ERR_INVALID_ARG;
+  if (d.ldw < d.K || d.ldq < d.K) return FP8BQ_ERR_INVALID_ARG;
+  if (!aligned(d.w, 2) || !aligned(d.s, 4)) return FP8BQ_ERR_INVALID_ARG;
+  return FP8BQ_OK;
+}
+
+fp8bq_status fp8bq_quant_weight(const void *w, int64_t N, int64_t K, int64_t ldw, uint8_t *q, int64_t ldq, float *sw,
+                                int mode, void *stream) {
+  if (bad_mode(mode)) return FP8BQ_ERR_INVALID_ARG;
+  fp8bq_weight_desc d;
+  d.w = w;
+  d.q = q;
+  d.s = sw;
+  d.N = N;
+  d.K = K;
+  d.ldw = ldw;
+  d.ldq = ldq;
+  fp8bq_status st = check_weight_desc(d);
+  if (st != FP8BQ_OK || N == 0 || K == 0) return st;
+  return launch_recalibrate(&d, 1, mode, static_cast<cudaStream_t>(stream));
+}
+
+fp8bq_status fp8bq_recalibrate(const fp8bq_weight_desc *descs, int n, int mode, void *stream) {
+  if (n < 0 || bad_mode(mode)) return FP8BQ_ERR_INVALID_ARG;
+  if (n == 0) return FP8BQ_OK;
+  if (!descs) return FP8BQ_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    fp8bq_status st = check_weight_desc(descs[i]);
+    if (st != FP8BQ_OK) return st;
+  }
+  return launch_recalibrate(descs, n, mode, static_cast<cudaStream_t>(stream));
+}
+
+fp8bq_status fp8bq_gemm_ex(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                           int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                           int mode, int variant, void *stream) {
+  if (variant < FP8BQ_GEMM_AUTO || variant > FP8BQ_GEMM_NATIVE_POW2) return FP8BQ_ERR_INVALID_ARG;
+  if (variant == FP8BQ_GEMM_NATIVE_POW2 && mode != FP8BQ_SCALE_POW2) return FP8BQ_ERR_INVALID_ARG;
+  fp8bq_status st = check_gemm_operands(qa, lda, sa, ldsa, qw, ldw, sw, y, ldy, M, N, K, mode);
+  if (st != FP8BQ_OK || M == 0 || N == 0) return st;
+  return launch_gemm(qa, lda, sa, ldsa, qw, ldw, sw, y, ldy, M, N, K, mode, variant,
+                     static_cast<cudaStream_t>(stream));
+}
+
+fp8bq_status fp8bq_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw, int64_t ldw,
+                        const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K, int mode,
+                        void *stream) {
+  return fp8bq_gemm_ex(qa, lda, sa, ldsa, qw, ldw, sw, y, ldy, M, N, K, mode, FP8BQ_GEMM_AUTO, stream);
+}
+
+}  // extern "C"

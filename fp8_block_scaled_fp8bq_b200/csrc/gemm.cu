@@ -1,0 +1,402 @@
+// Block-scaled FP8 GEMM for sm_100a: Y[M,N] (bf16) = X[M,K] . W[N,K]^T with
+// E4M3 operands, 1x128 activation scales and 128x128 weight scales.
+//
+// Method: "NVIDIA NeMo RL Achieves 48% Speedup With End-to-End FP8 Precision
+// Training", section "Technical breakthrough": the linear layers run in FP8 on
+// block-wise quantized E4M3 operands (activations 1x128, weights 128x128).
+//
+// Promotion design (FP32 scales).  A scale varies with the row m (activation)
+// and with the 128-column block of n (weight) and with the K-block, so it
+// cannot be folded into the MMA.  Each 128-deep K-block's product
+//   P_kb[m][n] = sum_{k in kb} qa[m][k] * qw[n][k]      (E4M3 x E4M3, exact in FP32)
+// is produced by the tensor cores into TMEM, and the epilogue warps add
+//   acc[m][n] += P_kb[m][n] * (sa[kb][m] * sw[n/128][kb])
+// into FP32 registers.  The result is rounded to bf16 once.
+//
+// Structure (one persistent CTA per SM, 384 threads = 3 warpgroups):
+//   warp 0      TMA producer: A (128x128 B) and B (256x128 B) tiles of each
+//               K-block into a 4-stage shared-memory ring (128-byte swizzle).
+//   warp 1      TMEM owner and MMA issuer: 4 x tcgen05.mma kind::f8f6f4
+//               (128x256x32) per K-block into one of two 256-column TMEM
+//               buffers; tcgen05.commit frees the smem stage and hands the
+//               buffer to the epilogue.
+//   warps 2-3   idle (warpgroup 0 gives its registers to the epilogue with
+//               setmaxnreg).
+//   warps 4-11  promotion + epilogue (warpgroups 1 and 2): warp w reads TMEM
+//               lanes 32*(w%4)..+31 (its 32 rows) and columns
+//               [128*h, 128*h+128) with h = (w-4)/4, i.e. exactly one 128-wide
+//               weight block, so each thread needs one scale product per
+//               K-block and holds 128 FP32 accumulators.  After the last
+//               K-block the accumulators go to shared memory as bf16 and out
+//               with TMA stores.
+// The MMA of K-block kb+1 overlaps the promotion of kb (two TMEM buffers), and
+// the stores of one tile overlap the MMAs of the next.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "device.cuh"
+#include "internal.h"
+
+namespace fp8bq {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 128;
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK;
+constexpr int kBBytes = BN * BK;
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kEpiWarps = 8;
+constexpr int kEpiBufBytes = 32 * 128;  // 32 rows x 64 bf16
+constexpr int kThreads = 128 + kEpiWarps * 32;
+// Register split (setmaxnreg): the launch gives every thread kLaunchRegs; the
+// producer/MMA warpgroup drops to kLowRegs and the two epilogue warpgroups
+// rise to kHighRegs.  128 * kLowRegs + 256 * kHighRegs must not exceed
+// 384 * kLaunchRegs (the build checks ptxas's count against kLaunchRegs).
+constexpr int kLaunchRegs = 168;
+constexpr int kLowRegs = 56;
+constexpr int kHighRegs = 224;
+static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split");
+constexpr int kTmemCols = 2 * BN;
+constexpr int kGroupM = 16;
+constexpr int kBarBytes = 256;
+constexpr int kSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiBufBytes + kBarBytes + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+struct GemmArgs {
+  const float *sa;
+  const float *sw;
+  int64_t ldsa;
+  int32_t M, N, KB, NB;
+  int32_t num_m, num_n;
+};
+
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int &mb, int &nb) {
+  const int per_group = kGroupM * num_n;
+  const int g = t / per_group;
+  const int first_m = g * kGroupM;
+  const int gm = min(num_m - first_m, kGroupM);
+  const int r = t - g * per_group;
+  mb = first_m + r % gm;
+  nb = r / gm;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Shared-memory carve-up and pipeline state common to the three roles.
+struct Smem {
+  uint8_t *a;        // kStages x [128 rows x 128 B], 128-byte swizzled
+  uint8_t *b;        // kStages x [256 rows x 128 B], 128-byte swizzled
+  uint8_t *epi;      // kEpiWarps x [32 rows x 128 B] bf16 staging
+  uint64_t *full;    // [kStages] TMA bytes landed
+  uint64_t *empty;   // [kStages] MMAs done reading the stage
+  uint64_t *tfull;   // [2] K-block partial ready in TMEM buffer
+  uint64_t *tempty;  // [2] TMEM buffer read by all epilogue warps
+  uint64_t *drain;   // MMA drain on the error path
+  uint32_t *tmem_slot;
+  volatile int *abort_flag;
+};
+
+__device__ __forceinline__ Smem carve(uint8_t *raw) {
+  Smem s;
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  s.a = base;
+  s.b = base + kStages * kABytes;
+  s.epi = s.b + kStages * kBBytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(s.epi + kEpiWarps * kEpiBufBytes);
+  s.full = bars;
+  s.empty = bars + kStages;
+  s.tfull = bars + 2 * kStages;
+  s.tempty = s.tfull + 2;
+  s.drain = s.tempty + 2;
+  s.tmem_slot = reinterpret_cast<uint32_t *>(s.drain + 1);
+  s.abort_flag = reinterpret_cast<volatile int *>(s.tmem_slot + 1);
+  return s;
+}
+
+// TMA producer (one thread): stream the A and B tiles of every K-block of this
+// CTA's tiles through the stage ring.
+__device__ __forceinline__ void run_producer(const Smem &S, const CUtensorMap *tmA, const CUtensorMap *tmB,
+                                             const GemmArgs &args) {
+  const int total = args.num_m * args.num_n;
+  int stage = 0;
+  uint32_t phase = 0, armed = 0, armed_parity = 0;
+  bool ok = true;
+  for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    int mb, nb;
+    tile_coords(t, args.num_m, args.num_n, mb, nb);
+    for (int kb = 0; kb < args.KB; ++kb) {
+      if (!mbar_wait(&S.empty[stage], phase ^ 1, S.abort_flag, kSiteProducerEmpty)) {
+        ok = false;
+        break;
+      }
+      mbar_arrive_expect_tx(&S.full[stage], kStageBytes);
+      tma_load_2d(S.a + stage * kABytes, tmA, &S.full[stage], kb * BK, mb * BM);
+      tma_load_2d(S.b + stage * kBBytes, tmB, &S.full[stage], kb * BK, nb * BN);
+      armed |= 1u << stage;
+      armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+      if (++stage == kStages) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+  }
+  if (!ok) {  // every load issued must land before the CTA may exit
+    for (int s = 0; s < kStages; ++s)
+      if (armed >> s & 1u) mbar_wait(&S.full[s], (armed_parity >> s) & 1u, nullptr, kSiteDrain);
+  }
+}
+
+// MMA issuer (one thread): per K-block, four 128x256x32 E4M3 MMAs into a fresh
+// TMEM buffer (the first one overwrites, the rest accumulate).
+__device__ __forceinline__ void run_mma(const Smem &S, uint32_t tmem_base, const GemmArgs &args) {
+  const int total = args.num_m * args.num_n;
+  const uint32_t idesc = idesc_f8f6f4_e4m3_f32(BM, BN);
+  int stage = 0, buf = 0;
+  uint32_t phase = 0, bphase = 0;
+  bool ok = true, issued = false;
+  for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    for (int kb = 0; kb < args.KB; ++kb) {
+      if (!mbar_wait(&S.tempty[buf], bphase ^ 1, S.abort_flag, kSiteMmaTmemEmpty) ||
+          !mbar_wait(&S.full[stage], phase, S.abort_flag, kSiteMmaFull)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d = tmem_base + (uint32_t)(buf * BN);
+      const uint32_t a0 = smem_addr(S.a + stage * kABytes);
+      const uint32_t b0 = smem_addr(S.b + stage * kBBytes);
+#pragma unroll
+      for (int k = 0; k < BK / 32; ++k)
+        mma_f8f6f4(d, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k), idesc, k > 0 ? 1u : 0u);
+      mma_commit(&S.empty[stage]);
+      mma_commit(&S.tfull[buf]);
+      issued = true;
+      if (++stage == kStages) {
+        stage = 0;
+        phase ^= 1;
+      }
+      if (++buf == 2) {
+        buf = 0;
+        bphase ^= 1;
+      }
+    }
+  }
+  if (!ok && issued) {  // TMEM must be quiescent before it is freed
+    mma_commit(S.drain);
+    mbar_wait(S.drain, 0, nullptr, kSiteDrain);
+  }
+}
+
+// Promotion + epilogue (one warp of the two epilogue warpgroups).
+__device__ __forceinline__ void run_epilogue(const Smem &S, uint32_t tmem_base, const CUtensorMap *tmY,
+                                             const GemmArgs &args, int warp, int lane) {
+  const int total = args.num_m * args.num_n;
+  const int KB = args.KB;
+  const int ew = warp - 4;
+  const int quarter = warp & 3;  // TMEM lanes this warp may access
+  const int half = ew >> 2;      // 128-column half of the tile = one weight block
+  const int row = quarter * 32 + lane;
+  uint8_t *ebuf = S.epi + ew * kEpiBufBytes;
+  int buf = 0;
+  uint32_t bphase = 0;
+  for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    int mb, nb;
+    tile_coords(t, args.num_m, args.num_n, mb, nb);
+    const int m = mb * BM + row;
+    const int wn = nb * 2 + half;
+    const bool live = m < args.M && wn < args.NB;
+    const float *sa_p = args.sa + m;
+    const float *sw_p = args.sw + (int64_t)wn * KB;
+    float acc[128];
+#pragma unroll
+    for (int j = 0; j < 128; ++j) acc[j] = 0.f;
+    // scale products for K-blocks kb and kb+1 (loaded two K-blocks ahead)
+    float sc0 = live ? __ldg(sa_p) * __ldg(sw_p) : 0.f;
+    float sc1 = (live && KB > 1) ? __ldg(sa_p + args.ldsa) * __ldg(sw_p + 1) : 0.f;
+    bool ok = true;
+    for (int kb = 0; kb < KB; ++kb) {
+      const float sc = sc0;
+      sc0 = sc1;
+      sc1 = (live && kb + 2 < KB) ? __ldg(sa_p + (int64_t)(kb + 2) * args.ldsa) * __ldg(sw_p + kb + 2) : 0.f;
+      const bool got = mbar_wait(&S.tfull[buf], bphase, S.abort_flag, kSiteEpiTmemFull);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN + half * 128);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + 32 * c, r);
+        tmem_ld_wait();
+        if (c == 3) {  // the buffer has been read: hand it back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.tempty[buf]);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[32 * c + j] = fmaf(__uint_as_float(r[j]), sc, acc[32 * c + j]);
+      }
+      if (++buf == 2) {
+        buf = 0;
+        bphase ^= 1;
+      }
+    }
+    if (!ok) break;
+    // bf16 out: two 64-column chunks through this warp's 4 KB staging buffer,
+    // written in the 128-byte swizzled order the TMA store expects.
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      if (lane == 0) bulk_wait_group_read0();
+      __syncwarp();
+      uint8_t *rowp = ebuf + lane * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float *a = &acc[c * 64 + j * 8];
+        uint4 pk;
+        pk.x = pack_bf16x2(a[0], a[1]);
+        pk.y = pack_bf16x2(a[2], a[3]);
+        pk.z = pack_bf16x2(a[4], a[5]);
+        pk.w = pack_bf16x2(a[6], a[7]);
+        *reinterpret_cast<uint4 *>(rowp + ((j ^ (lane & 7)) << 4)) = pk;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const int x = nb * BN + half * 128 + c * 64;
+        const int y = mb * BM + quarter * 32;
+        if (x < args.N && y < args.M) {
+          tma_store_2d(tmY, ebuf, x, y);
+          bulk_commit_group();
+        }
+      }
+    }
+  }
+  if (lane == 0) bulk_wait_group0();
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_promote_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmY, const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  const Smem S = carve(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.tfull[b], 1);
+      mbar_init(&S.tempty[b], kEpiWarps);
+    }
+    mbar_init(S.drain, 1);
+    *S.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmY);
+  }
+  if (warp == 1) {
+    tmem_alloc(S.tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *S.tmem_slot;
+
+  // Each role's setmaxnreg sits inside the role's own branch, so the code of
+  // the role is compiled under that role's register budget.
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
+    if (warp == 0 && lane == 0) run_producer(S, &tmA, &tmB, args);
+    else if (warp == 1 && lane == 0) run_mma(S, tmem_base, args);
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
+    run_epilogue(S, tmem_base, &tmY, args, warp, lane);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// Per-device one-time setup: opt in to the large shared-memory carve-up and
+// confirm that the kernel was built with the register count the setmaxnreg
+// split assumes (a smaller count would make setmaxnreg.inc wait forever).
+int g_ready[64] = {0};  // 0 unknown, 1 ready, -1 refused
+
+fp8bq_status prepare_kernel() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (g_ready[dev] == 1) return FP8BQ_OK;
+  if (g_ready[dev] == -1) return FP8BQ_ERR_UNSUPPORTED;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, gemm_promote_kernel);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(gemm)");
+  if (fa.numRegs != kLaunchRegs) {
+    g_ready[dev] = -1;
+    return FP8BQ_ERR_UNSUPPORTED;
+  }
+  e = cudaFuncSetAttribute(gemm_promote_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
+  g_ready[dev] = 1;
+  return FP8BQ_OK;
+}
+
+}  // namespace
+
+cudaError_t take_device_error_gemm(unsigned long long *v) { return take_tu_device_error(v); }
+
+fp8bq_status launch_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                         int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K, int mode,
+                         int variant, cudaStream_t stream) {
+  (void)mode;
+  (void)variant;
+  if (M == 0 || N == 0) return FP8BQ_OK;
+  if (K == 0) {
+    cudaError_t e = cudaMemset2DAsync(y, (size_t)ldy * 2, 0, (size_t)N * 2, (size_t)M, stream);
+    return e == cudaSuccess ? FP8BQ_OK : cuda_fail(e, "memset(y)");
+  }
+  CUtensorMap tA, tB, tY;
+  if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qa, (uint64_t)K, (uint64_t)M, (uint64_t)lda, BK, BM,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, (uint64_t)K, (uint64_t)N, (uint64_t)ldw, BK, BN,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M, (uint64_t)ldy * 2, 64, 32,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return FP8BQ_ERR_INVALID_ARG;
+  fp8bq_status st = prepare_kernel();
+  if (st != FP8BQ_OK) return st;
+  GemmArgs a;
+  a.sa = sa;
+  a.sw = sw;
+  a.ldsa = ldsa;
+  a.M = (int32_t)M;
+  a.N = (int32_t)N;
+  a.KB = (int32_t)(K / BK);
+  a.NB = (int32_t)((N + 127) / 128);
+  a.num_m = (int32_t)((M + BM - 1) / BM);
+  a.num_n = (int32_t)((N + BN - 1) / BN);
+  const int64_t tiles = (int64_t)a.num_m * a.num_n;
+  const int grid = (int)std::min<int64_t>(tiles, num_sms());
+  gemm_promote_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tA, tB, tY, a);
+  return check_launch("gemm");
+}
+
+}  // namespace fp8bq

@@ -1,0 +1,38 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fp8bq.h"
+
+namespace fp8bq {
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+// Record the failing CUDA call for diagnostics and map it to FP8BQ_ERR_CUDA.
+fp8bq_status cuda_fail(cudaError_t e, const char *what);
+
+// Check the last launch.
+fp8bq_status check_launch(const char *what);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+// Returns false if the driver rejects the map.
+bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
+                  uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
+
+// Per translation unit: read and clear its device error word.
+cudaError_t take_device_error_gemm(unsigned long long *v);
+
+// Launchers (arguments already validated).
+fp8bq_status launch_encode(const float *x, int64_t n, uint8_t *q, cudaStream_t stream);
+fp8bq_status launch_quant_act(const void *x, int64_t M, int64_t K, int64_t ldx, uint8_t *q, int64_t ldq, float *sa,
+                              int64_t ldsa, int mode, cudaStream_t stream);
+fp8bq_status launch_recalibrate(const fp8bq_weight_desc *descs, int n, int mode, cudaStream_t stream);
+fp8bq_status launch_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                         int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K, int mode,
+                         int variant, cudaStream_t stream);
+
+}  // namespace fp8bq

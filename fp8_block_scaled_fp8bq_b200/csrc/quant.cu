@@ -1,0 +1,368 @@
+// E4M3 quantization kernels: 1x128 activation tiles, 128x128 weight tiles and
+// the multi-tensor per-step recalibration.
+//
+// Method: "NVIDIA NeMo RL Achieves 48% Speedup With End-to-End FP8 Precision
+// Training", section "Technical breakthrough" (block-wise E4M3; weights
+// 128x128, activations 1x128) and section "Real-world performance gains"
+// (scales recalibrated after every training step); power-of-2 scales from
+// section "Why this matters for AI economics".
+//
+// These kernels are HBM-bound (2 bytes read, 1 byte written per element):
+// 16-byte vector loads of bf16, an integer max over |x| bit patterns (for
+// non-negative bf16 the bit order is the value order, so the amax is exact),
+// one IEEE division per element (FP32 scales) or a multiply by the exact
+// reciprocal power of two (POW2 scales), and the hardware E4M3 conversion with
+// round-to-nearest-even and saturation (cvt.rn.satfinite.e4m3x2.f32).
+#include <cuda_fp8.h>
+
+#include <algorithm>
+
+#include "device.cuh"
+#include "internal.h"
+
+namespace fp8bq {
+namespace {
+
+// ---------------------------------------------------------------------------
+// Scales
+// ---------------------------------------------------------------------------
+// Smallest e with amax <= 448 * 2^e, clamped to [-127, 127].  With
+// amax = f * 2^E, f in [1, 2): 448 * 2^e = 1.75 * 2^(e+8), so e = E - 8 when
+// f <= 1.75 and e = E - 7 otherwise.  amax > 0.
+__device__ __forceinline__ int pow2_exponent(float amax) {
+  uint32_t b = __float_as_uint(amax);
+  int ef = (int)(b >> 23);
+  uint32_t frac = b & 0x7FFFFFu;
+  int E;
+  if (ef == 0) {                        // denormal: normalize the fraction
+    int p = 31 - __clz((int)frac);      // leading one, 0..22
+    E = p - 149;
+    frac = (frac << (23 - p)) & 0x7FFFFFu;
+  } else {
+    E = ef - 127;
+  }
+  int e = (frac <= 0x600000u) ? E - 8 : E - 7;
+  return max(-127, min(127, e));
+}
+
+// 2^e for e in [-127, 127], exactly (2^-127 is a binary32 denormal).
+__device__ __forceinline__ float exp2_exact(int e) {
+  return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+template <int MODE>
+__device__ __forceinline__ void tile_scale(float amax, float &s, float &inv) {
+  if (!(amax > 0.f)) {
+    s = 1.f;
+    inv = 1.f;
+  } else if (MODE == FP8BQ_SCALE_FP32) {
+    s = __fdiv_rn(amax, 448.f);
+    inv = 0.f;  // unused: the FP32 path divides
+  } else {
+    int e = pow2_exponent(amax);
+    s = exp2_exact(e);
+    inv = exp2_exact(-e);
+  }
+}
+
+// The binary32 quotient x / s, correctly rounded.  For a power-of-two scale the
+// product with the exact reciprocal is the same single rounding.
+template <int MODE>
+__device__ __forceinline__ float quotient(float x, float s, float inv) {
+  if (MODE == FP8BQ_SCALE_FP32) return __fdiv_rn(x, s);
+  return x * inv;
+}
+
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+}
+
+// 8 bf16 (one 16-byte vector) -> 8 E4M3 codes (8 bytes).
+template <int MODE>
+__device__ __forceinline__ uint2 encode8(uint4 v, float s, float inv) {
+  uint2 r;
+  r.x = e4m3x2(quotient<MODE>(bf16_lo(v.x), s, inv), quotient<MODE>(bf16_hi(v.x), s, inv)) |
+        (e4m3x2(quotient<MODE>(bf16_lo(v.y), s, inv), quotient<MODE>(bf16_hi(v.y), s, inv)) << 16);
+  r.y = e4m3x2(quotient<MODE>(bf16_lo(v.z), s, inv), quotient<MODE>(bf16_hi(v.z), s, inv)) |
+        (e4m3x2(quotient<MODE>(bf16_lo(v.w), s, inv), quotient<MODE>(bf16_hi(v.w), s, inv)) << 16);
+  return r;
+}
+
+// max |x| of 8 bf16 as a bf16 bit pattern (exact for finite values).
+__device__ __forceinline__ uint32_t absmax_bits8(uint4 v) {
+  uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu), __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+__device__ __forceinline__ float bits_to_amax(uint32_t b16) { return __uint_as_float(b16 << 16); }
+
+// ---------------------------------------------------------------------------
+// Activation quantization, 1x128 tiles
+// ---------------------------------------------------------------------------
+// Block = 8 warps; a half-warp owns one 1x128 tile (16 lanes x 8 elements);
+// each half-warp handles U rows of one K-block, all loads issued first.
+// Block covers rows [blockIdx.x * 16U, +16U) of K-block blockIdx.y.
+template <int MODE, int U>
+__global__ void __launch_bounds__(256) quant_act_vec_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
+                                                            int64_t ldx, uint8_t *__restrict__ q, int64_t ldq,
+                                                            float *__restrict__ sa, int64_t ldsa) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hl = lane & 15, half = lane >> 4;
+  const int64_t kb = blockIdx.y;
+  const int64_t k = kb * 128 + hl * 8;
+  const bool kin = k < K;  // K % 8 == 0 here: a vector is wholly in or out
+  const int64_t rbase = (int64_t)blockIdx.x * (16 * U) + warp * (2 * U) + half;
+
+  uint4 v[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int64_t r = rbase + 2 * u;
+    v[u] = (kin && r < M) ? ld_nc_v4(x + r * ldx + k) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int64_t r = rbase + 2 * u;
+    uint32_t m = absmax_bits8(v[u]);
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 8));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    float s, inv;
+    tile_scale<MODE>(bits_to_amax(m), s, inv);
+    if (r < M) {
+      if (kin) *reinterpret_cast<uint2 *>(q + r * ldq + k) = encode8<MODE>(v[u], s, inv);
+      if (hl == 0) sa[kb * ldsa + r] = s;
+    }
+  }
+}
+
+// Any alignment: one half-warp per tile, element j of lane hl is k0 + hl + 16 j.
+template <int MODE>
+__global__ void __launch_bounds__(256) quant_act_scalar_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
+                                                               int64_t ldx, uint8_t *__restrict__ q, int64_t ldq,
+                                                               float *__restrict__ sa, int64_t ldsa) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hl = lane & 15, half = lane >> 4;
+  const int64_t kb = blockIdx.y;
+  const int64_t r = (int64_t)blockIdx.x * 16 + warp * 2 + half;
+  uint16_t e[8];
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int64_t k = kb * 128 + hl + 16 * j;
+    e[j] = (r < M && k < K) ? x[r * ldx + k] : (uint16_t)0;
+    m = max(m, (uint32_t)(e[j] & 0x7FFFu));
+  }
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 8));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  float s, inv;
+  tile_scale<MODE>(bits_to_amax(m), s, inv);
+  if (r >= M) return;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int64_t k = kb * 128 + hl + 16 * j;
+    if (k < K) {
+      const float f = __uint_as_float((uint32_t)e[j] << 16);
+      q[r * ldq + k] = (uint8_t)(e4m3x2(quotient<MODE>(f, s, inv), 0.f) & 0xFFu);
+    }
+  }
+  if (hl == 0) sa[kb * ldsa + r] = s;
+}
+
+// ---------------------------------------------------------------------------
+// Weight quantization / recalibration, 128x128 tiles
+// ---------------------------------------------------------------------------
+constexpr int kMaxDescs = 128;
+
+struct TileTensor {
+  const uint16_t *w;
+  uint8_t *q;
+  float *s;
+  int64_t N, K, ldw, ldq;
+  int64_t tile_begin;  // global id of this tensor's first tile
+  int32_t KB;          // tiles along K
+  int32_t vec;         // 16-byte vector path allowed
+};
+
+struct RecalParams {
+  int32_t n;
+  int64_t total;  // tiles over all tensors
+  TileTensor t[kMaxDescs];
+};
+
+// One 128x128 tile, 256 threads: thread t holds rows (t>>4) + 16 i, i = 0..7, of
+// the 16-byte column chunk (t & 15).  The tile stays in registers between the
+// amax and the encode, so it is read from HBM once.
+template <int MODE>
+__device__ __forceinline__ void quant_tile_vec(const TileTensor &T, int64_t nb, int64_t kb, uint32_t *red) {
+  const int t = threadIdx.x;
+  const int c = t & 15, r0 = t >> 4;
+  const int64_t k = kb * 128 + c * 8;
+  const bool kin = k < T.K;
+  uint4 v[8];
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t n = nb * 128 + r0 + 16 * i;
+    v[i] = (kin && n < T.N) ? ld_nc_v4(T.w + n * T.ldw + k) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = max(m, absmax_bits8(v[i]));
+  m = __reduce_max_sync(0xffffffffu, m);
+  if ((t & 31) == 0) red[t >> 5] = m;
+  __syncthreads();
+  m = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) m = max(m, red[w]);
+  float s, inv;
+  tile_scale<MODE>(bits_to_amax(m), s, inv);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t n = nb * 128 + r0 + 16 * i;
+    if (kin && n < T.N) *reinterpret_cast<uint2 *>(T.q + n * T.ldq + k) = encode8<MODE>(v[i], s, inv);
+  }
+  if (t == 0) T.s[nb * T.KB + kb] = s;
+  __syncthreads();  // red[] is reused by the next tile
+}
+
+// Any alignment: two passes over the (cached) tile with scalar accesses.
+template <int MODE>
+__device__ __forceinline__ void quant_tile_scalar(const TileTensor &T, int64_t nb, int64_t kb, uint32_t *red) {
+  const int t = threadIdx.x;
+  uint32_t m = 0;
+  for (int idx = t; idx < 128 * 128; idx += 256) {
+    const int64_t n = nb * 128 + (idx >> 7), k = kb * 128 + (idx & 127);
+    if (n < T.N && k < T.K) m = max(m, (uint32_t)(T.w[n * T.ldw + k] & 0x7FFFu));
+  }
+  m = __reduce_max_sync(0xffffffffu, m);
+  if ((t & 31) == 0) red[t >> 5] = m;
+  __syncthreads();
+  m = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) m = max(m, red[w]);
+  float s, inv;
+  tile_scale<MODE>(bits_to_amax(m), s, inv);
+  for (int idx = t; idx < 128 * 128; idx += 256) {
+    const int64_t n = nb * 128 + (idx >> 7), k = kb * 128 + (idx & 127);
+    if (n < T.N && k < T.K) {
+      const float f = __uint_as_float((uint32_t)T.w[n * T.ldw + k] << 16);
+      T.q[n * T.ldq + k] = (uint8_t)(e4m3x2(quotient<MODE>(f, s, inv), 0.f) & 0xFFu);
+    }
+  }
+  if (t == 0) T.s[nb * T.KB + kb] = s;
+  __syncthreads();
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(256) recalibrate_kernel(const __grid_constant__ RecalParams p) {
+  __shared__ uint32_t red[8];
+  for (int64_t tile = blockIdx.x; tile < p.total; tile += gridDim.x) {
+    int lo = 0, hi = p.n - 1;  // last tensor whose first tile is <= tile
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.t[mid].tile_begin <= tile) lo = mid;
+      else hi = mid - 1;
+    }
+    const TileTensor &T = p.t[lo];
+    const int64_t local = tile - T.tile_begin;
+    const int64_t nb = local / T.KB, kb = local - nb * T.KB;
+    if (T.vec) quant_tile_vec<MODE>(T, nb, kb, red);
+    else quant_tile_scalar<MODE>(T, nb, kb, red);
+  }
+}
+
+__global__ void __launch_bounds__(256) encode_kernel(const float *__restrict__ x, int64_t n, uint8_t *__restrict__ q) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x * 4;
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4; i < n; i += stride) {
+    if (i + 4 <= n) {
+      const float4 v = *reinterpret_cast<const float4 *>(x + i);
+      *reinterpret_cast<uint32_t *>(q + i) = e4m3x2(v.x, v.y) | (e4m3x2(v.z, v.w) << 16);
+    } else {
+      for (int64_t j = i; j < n; ++j) q[j] = (uint8_t)(e4m3x2(x[j], 0.f) & 0xFFu);
+    }
+  }
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int g_recal_blocks_per_sm[2] = {0, 0};
+
+}  // namespace
+
+fp8bq_status launch_encode(const float *x, int64_t n, uint8_t *q, cudaStream_t stream) {
+  if (n == 0) return FP8BQ_OK;
+  const int64_t blocks = std::min<int64_t>((n + 1023) / 1024, (int64_t)num_sms() * 16);
+  encode_kernel<<<(unsigned)blocks, 256, 0, stream>>>(x, n, q);
+  return check_launch("e4m3_encode");
+}
+
+fp8bq_status launch_quant_act(const void *x, int64_t M, int64_t K, int64_t ldx, uint8_t *q, int64_t ldq, float *sa,
+                              int64_t ldsa, int mode, cudaStream_t stream) {
+  const int64_t KB = (K + 127) / 128;
+  if (M == 0 || K == 0) return FP8BQ_OK;
+  if (KB > 65535) return FP8BQ_ERR_UNSUPPORTED;
+  const uint16_t *xs = static_cast<const uint16_t *>(x);
+  const bool vec = aligned(x, 16) && ldx % 8 == 0 && K % 8 == 0 && aligned(q, 8) && ldq % 8 == 0;
+  if (vec) {
+    constexpr int U = 4;
+    dim3 grid((unsigned)((M + 16 * U - 1) / (16 * U)), (unsigned)KB);
+    if (mode == FP8BQ_SCALE_FP32)
+      quant_act_vec_kernel<FP8BQ_SCALE_FP32, U><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, ldq, sa, ldsa);
+    else
+      quant_act_vec_kernel<FP8BQ_SCALE_POW2, U><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, ldq, sa, ldsa);
+  } else {
+    dim3 grid((unsigned)((M + 15) / 16), (unsigned)KB);
+    if (mode == FP8BQ_SCALE_FP32)
+      quant_act_scalar_kernel<FP8BQ_SCALE_FP32><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, ldq, sa, ldsa);
+    else
+      quant_act_scalar_kernel<FP8BQ_SCALE_POW2><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, ldq, sa, ldsa);
+  }
+  return check_launch("quant_act");
+}
+
+fp8bq_status launch_recalibrate(const fp8bq_weight_desc *descs, int n, int mode, cudaStream_t stream) {
+  const int mi = mode == FP8BQ_SCALE_FP32 ? 0 : 1;
+  if (g_recal_blocks_per_sm[mi] == 0) {
+    int b = 0;
+    cudaError_t e = mode == FP8BQ_SCALE_FP32
+                        ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, recalibrate_kernel<FP8BQ_SCALE_FP32>, 256, 0)
+                        : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, recalibrate_kernel<FP8BQ_SCALE_POW2>, 256, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "occupancy(recalibrate)");
+    g_recal_blocks_per_sm[mi] = std::max(1, b);
+  }
+  const int64_t resident = (int64_t)num_sms() * g_recal_blocks_per_sm[mi];
+  for (int base = 0; base < n; base += kMaxDescs) {
+    RecalParams p;
+    p.n = 0;
+    p.total = 0;
+    for (int i = base; i < n && i < base + kMaxDescs; ++i) {
+      const fp8bq_weight_desc &d = descs[i];
+      if (d.N == 0 || d.K == 0) continue;
+      TileTensor &t = p.t[p.n++];
+      t.w = static_cast<const uint16_t *>(d.w);
+      t.q = d.q;
+      t.s = d.s;
+      t.N = d.N;
+      t.K = d.K;
+      t.ldw = d.ldw;
+      t.ldq = d.ldq;
+      t.KB = (int32_t)((d.K + 127) / 128);
+      t.tile_begin = p.total;
+      t.vec = aligned(d.w, 16) && d.ldw % 8 == 0 && d.K % 8 == 0 && aligned(d.q, 8) && d.ldq % 8 == 0;
+      p.total += ((d.N + 127) / 128) * (int64_t)t.KB;
+    }
+    if (p.total == 0) continue;
+    const unsigned grid = (unsigned)std::min<int64_t>(p.total, resident);
+    if (mode == FP8BQ_SCALE_FP32)
+      recalibrate_kernel<FP8BQ_SCALE_FP32><<<grid, 256, 0, stream>>>(p);
+    else
+      recalibrate_kernel<FP8BQ_SCALE_POW2><<<grid, 256, 0, stream>>>(p);
+    fp8bq_status st = check_launch("recalibrate");
+    if (st != FP8BQ_OK) return st;
+  }
+  return FP8BQ_OK;
+}
+
+}  // namespace fp8bq

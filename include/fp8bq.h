@@ -1,0 +1,235 @@
+/*
+ * fp8bq: block-wise FP8 (E4M3) linear layer for NVIDIA B200 (sm_100a).
+ *
+ * Method source: the article "NVIDIA NeMo RL Achieves 48% Speedup With
+ * End-to-End FP8 Precision Training" (three translations of one page):
+ *   section "Technical breakthrough"          block-wise quantized FP8 in E4M3,
+ *                                             128x128 tiles for weights, 1x128
+ *                                             tiles for activations, linear
+ *                                             layers computed in FP8;
+ *   section "Real-world performance gains"    scales recalibrated after every
+ *                                             training step; the recipe also
+ *                                             runs on a mixture-of-experts model;
+ *   section "Why this matters for AI economics"  power-of-2 scaling factors
+ *                                             as an option.
+ *
+ * Definitions used by every entry point (the pages fix only the format and the
+ * tile shapes; these are the plainest readings and the library's contract):
+ *   E4M3          OCP 8-bit float, 1-4-3 bits, bias 7, max 448, no infinity.
+ *   tile amax     max |x| over the tile's in-bounds elements (exact).
+ *   scale         FP8BQ_SCALE_FP32: s = amax / 448 (one IEEE binary32 division);
+ *                 FP8BQ_SCALE_POW2: s = 2^e, e the smallest integer with
+ *                 amax <= 448 * 2^e, clamped to [-127, 127];
+ *                 an all-zero tile has s = 1.
+ *   code          q = E4M3(x / s): the binary32 quotient (correctly rounded),
+ *                 then round-to-nearest-even onto E4M3 with saturation at
+ *                 +-448; zero results keep the sign of x.
+ *   GEMM          Y[m][n] = sum_kb sa[kb][m] * sw[n/128][kb] * P_kb[m][n], where
+ *                 P_kb is the exact E4M3 x E4M3 dot product over K-block kb,
+ *                 accumulated in FP32 and written as BF16 (round to nearest
+ *                 even).  Y = X W^T: both operands are K-contiguous.
+ *
+ * Conventions
+ *   - Every pointer argument is DEVICE memory owned by the caller, except the
+ *     descriptor array of fp8bq_recalibrate (host memory, read during the call).
+ *     The library allocates no device memory.
+ *   - Every call is asynchronous and ordered on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  No call synchronizes the host, except
+ *     fp8bq_get_device_error.  Calls are safe from several host threads.
+ *   - Leading dimensions (ld*) count elements, not bytes.
+ *   - Status: FP8BQ_OK means the work was launched.  Arguments are checked
+ *     before anything is launched; a failed check launches nothing.
+ *   - A kernel that waits on an on-chip barrier for longer than about a second
+ *     gives up, records an error word on the device and returns; the next
+ *     fp8bq_get_device_error reports FP8BQ_ERR_TIMEOUT.  No kernel traps.
+ *   - Non-finite inputs are outside the contract: they never hang or trap a
+ *     kernel, but their codes and outputs are unspecified.
+ *   - Sizes of 0 (M, N, K, E or rows) are successful no-ops, except that a GEMM
+ *     with K == 0 writes zeros.
+ */
+#ifndef FP8BQ_H
+#define FP8BQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FP8BQ_API __attribute__((visibility("default")))
+#else
+#define FP8BQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP8BQ_OK = 0,
+    FP8BQ_ERR_INVALID_ARG = 1,   /* null pointer with a nonzero size, negative size,
+                                    ld smaller than the row, misaligned pointer/ld */
+    FP8BQ_ERR_UNSUPPORTED = 2,   /* valid but not supported (e.g. GEMM K % 128 != 0) */
+    FP8BQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    FP8BQ_ERR_WORKSPACE = 4,     /* workspace missing or too small */
+    FP8BQ_ERR_TIMEOUT = 5        /* a kernel gave up waiting on an on-chip barrier */
+} fp8bq_status;
+
+typedef enum {
+    FP8BQ_SCALE_FP32 = 0,        /* s = amax / 448 */
+    FP8BQ_SCALE_POW2 = 1         /* s = 2^ceil(log2(amax / 448)), exact integer rule */
+} fp8bq_scale_mode;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+FP8BQ_API int fp8bq_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+FP8BQ_API const char *fp8bq_status_string(fp8bq_status status);
+
+/*
+ * Text of the last failing CUDA call made by this host thread inside the
+ * library ("" if none); valid until the thread's next failing call.
+ */
+FP8BQ_API const char *fp8bq_last_cuda_error(void);
+
+/*
+ * Reads and clears the device error word of the current device (this call
+ * synchronizes the device).  *code receives the raw word (0 = none; otherwise
+ * (where << 16) | block, for diagnostics).  Returns FP8BQ_ERR_TIMEOUT if a
+ * kernel gave up waiting since the last call, FP8BQ_OK otherwise.
+ */
+FP8BQ_API fp8bq_status fp8bq_get_device_error(uint64_t *code);
+
+/*
+ * Element-wise E4M3 encoding of fp32 values that are already scaled:
+ * q[i] = E4M3(x[i]) with round-to-nearest-even and saturation at +-448 (the
+ * conversion every quantizer here ends with).  x: fp32 [n]; q: uint8 [n].
+ */
+FP8BQ_API fp8bq_status fp8bq_e4m3_encode(const float *x, int64_t n, uint8_t *q, void *stream);
+
+/*
+ * Activation quantization over 1x128 tiles ("Technical breakthrough": 1x128
+ * activation granularity).
+ *   x     bf16 [M][ldx], row-major.
+ *   q     uint8 E4M3 codes [M][ldq], row-major.
+ *   sa    fp32 scales, K-block-major: the scale of tile (m, kb) is
+ *         sa[kb * ldsa + m], kb = 0 .. ceil(K/128)-1; ldsa >= M.
+ *         (One K-block's row scales are contiguous, which is the order in which
+ *         the GEMM consumes them.)
+ *   The last tile of a row may hold fewer than 128 elements.
+ * Requirements: ldx >= K, ldq >= K, ldsa >= M.  Any alignment is accepted;
+ * 16-byte-aligned x with ldx % 8 == 0 and K % 8 == 0, and 8-byte-aligned q with
+ * ldq % 8 == 0, take the vectorized path.
+ */
+FP8BQ_API fp8bq_status fp8bq_quant_act(const void *x, int64_t M, int64_t K, int64_t ldx,
+                             uint8_t *q, int64_t ldq, float *sa, int64_t ldsa,
+                             int mode, void *stream);
+
+/*
+ * Weight quantization over 128x128 tiles ("Technical breakthrough": 128x128
+ * weight granularity).
+ *   w     bf16 [N][ldw], row-major (out features x in features).
+ *   q     uint8 E4M3 codes [N][ldq].
+ *   sw    fp32 scales [ceil(N/128)][ceil(K/128)], row-major, dense.
+ * Edge tiles are clipped to the tensor.  Requirements: ldw >= K, ldq >= K.
+ */
+FP8BQ_API fp8bq_status fp8bq_quant_weight(const void *w, int64_t N, int64_t K, int64_t ldw,
+                                uint8_t *q, int64_t ldq, float *sw,
+                                int mode, void *stream);
+
+/* One weight tensor of a recalibration: fields as in fp8bq_quant_weight. */
+typedef struct {
+    const void *w;       /* bf16 [N][ldw] (device) */
+    uint8_t *q;          /* E4M3 codes [N][ldq] (device) */
+    float *s;            /* fp32 scales [ceil(N/128)][ceil(K/128)] (device) */
+    int64_t N, K, ldw, ldq;
+} fp8bq_weight_desc;
+
+/*
+ * Per-step recalibration ("Real-world performance gains": the policy weights
+ * change every step, so their scales are recomputed after each step): requantize
+ * every 128x128 tile of n weight tensors, in as few launches as possible
+ * (one launch per 128 tensors).  `descs` is a HOST array read before the call
+ * returns (the caller may free it on return).  Results equal calling
+ * fp8bq_quant_weight on each tensor.  Tensors must not overlap.
+ */
+FP8BQ_API fp8bq_status fp8bq_recalibrate(const fp8bq_weight_desc *descs, int n, int mode, void *stream);
+
+/*
+ * Block-scaled FP8 GEMM, Y = X W^T ("Technical breakthrough": linear layers in
+ * FP8 on the tensor cores).
+ *   qa    E4M3 [M][lda]      activation codes (from fp8bq_quant_act)
+ *   sa    fp32 [K/128][ldsa] activation scales (layout of fp8bq_quant_act)
+ *   qw    E4M3 [N][ldw]      weight codes (from fp8bq_quant_weight)
+ *   sw    fp32 [ceil(N/128)][K/128] weight scales
+ *   y     bf16 [M][ldy]      output
+ * Each 128-deep K-block's FP32 partial product is multiplied by
+ * sa[kb][m] * sw[n/128][kb] and added into an FP32 accumulator; the result is
+ * rounded to bf16.  `mode` states how the scales were made; FP8BQ_SCALE_POW2
+ * lets the library use the tensor cores' native block-scaled MMA (scales are
+ * exact powers of two, so only the summation order differs).
+ * Requirements: K % 128 == 0; M, N, K < 2^31; qa, qw 16-byte aligned with
+ * lda, ldw >= K and multiples of 16; y 16-byte aligned with ldy >= N a
+ * multiple of 8; sa 16-byte aligned with ldsa >= M a multiple of 4; sw
+ * 4-byte aligned.  Violations return FP8BQ_ERR_INVALID_ARG (layout) or
+ * FP8BQ_ERR_UNSUPPORTED (K % 128, sizes).
+ */
+FP8BQ_API fp8bq_status fp8bq_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa,
+                        const uint8_t *qw, int64_t ldw, const float *sw,
+                        void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                        int mode, void *stream);
+
+/* Variant selector for fp8bq_gemm_ex (testing and benchmarking). */
+typedef enum {
+    FP8BQ_GEMM_AUTO = 0,          /* what fp8bq_gemm does */
+    FP8BQ_GEMM_PROMOTE = 1,       /* FP32 promotion of every K-block partial */
+    FP8BQ_GEMM_NATIVE_POW2 = 2    /* native block-scaled MMA (POW2 scales only) */
+} fp8bq_gemm_variant;
+
+FP8BQ_API fp8bq_status fp8bq_gemm_ex(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa,
+                           const uint8_t *qw, int64_t ldw, const float *sw,
+                           void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                           int mode, int variant, void *stream);
+
+/*
+ * Decode-shaped (small-M, memory-bound) linear with on-the-fly activation
+ * quantization: q(x) over 1x128 tiles, then the block-scaled GEMM against the
+ * pre-quantized weight (generation side of the recipe, "Technical
+ * breakthrough": FP8 in both generation and training).
+ *   x     bf16 [M][ldx]; qw, sw as in fp8bq_gemm; y bf16 [M][ldy].
+ *   ws    device workspace of at least fp8bq_gemm_decode_workspace_size(M, N, K)
+ *         bytes, 256-byte aligned; its contents need not be initialized and are
+ *         overwritten.  Calls that share a workspace must be stream-ordered.
+ * Requirements: as fp8bq_gemm, and M <= 256.  Output equals fp8bq_quant_act
+ * followed by fp8bq_gemm up to FP32 summation order.
+ */
+FP8BQ_API size_t fp8bq_gemm_decode_workspace_size(int64_t M, int64_t N, int64_t K);
+
+FP8BQ_API fp8bq_status fp8bq_gemm_decode(const void *x, int64_t ldx,
+                               const uint8_t *qw, int64_t ldw, const float *sw,
+                               void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                               int mode, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Grouped (mixture-of-experts) GEMM ("Real-world performance gains": the
+ * recipe on a mixture-of-experts model): rows [offsets[e], offsets[e+1]) of the
+ * expert-sorted activations are multiplied by expert e's weight.
+ *   qa, sa   as fp8bq_gemm over total_rows rows (sa: [K/128][ldsa])
+ *   qw       E4M3 [E][N][K], dense          sw  fp32 [E][ceil(N/128)][K/128]
+ *   offsets  int32 [E+1] on the device, nondecreasing, offsets[0] = 0,
+ *            offsets[E] = total_rows.  Read on the device (no host sync): a
+ *            device-side scheduler maps output tiles to (expert, row block,
+ *            column block).
+ *   y        bf16 [total_rows][ldy]
+ * Requirements: as fp8bq_gemm; 1 <= E <= 1024.  Offsets that break the rules
+ * above give unspecified output rows but no out-of-bounds access.
+ */
+FP8BQ_API fp8bq_status fp8bq_grouped_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa,
+                                const uint8_t *qw, const float *sw,
+                                const int32_t *offsets, int E, int64_t total_rows,
+                                int64_t N, int64_t K, void *y, int64_t ldy,
+                                int mode, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8BQ_H */

@@ -1,0 +1,99 @@
+"""The C-ABI library builds, loads without a GPU, exports every entry point that
+include/fp8bq.h declares, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import fp8_block_scaled_fp8bq_b200 as fq
+from fp8_block_scaled_fp8bq_b200 import build as fbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8bq.h")
+
+INVALID, UNSUPPORTED = 1, 2
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FP8BQ_API\s+[\w\s\*]+?\b(fp8bq_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    fbuild.build()
+    return fq.lib()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("fp8bq_quant_act", "fp8bq_quant_weight", "fp8bq_recalibrate", "fp8bq_gemm",
+              "fp8bq_grouped_gemm", "fp8bq_gemm_decode"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", fq.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r" T (fp8bq_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    # and nothing else from the library's internals leaks out
+    extra = [n for n in exported if n not in declared_functions()]
+    assert not extra, extra
+    assert set(fq.SIGNATURES) == set(declared_functions())
+
+
+def test_header_compiles_as_c():
+    src = '#include "fp8bq.h"\nint main(void){return FP8BQ_OK;}\n'
+    r = subprocess.run(["gcc", "-x", "c", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        "-fsyntax-only", "-"], input=src, text=True, capture_output=True)
+    assert r.returncode == 0, r.stderr
+
+
+def test_status_strings(L):
+    assert L.fp8bq_status_string(0) == b"FP8BQ_OK"
+    assert L.fp8bq_status_string(5) == b"FP8BQ_ERR_TIMEOUT"
+    assert L.fp8bq_version() >= 100
+
+
+FAKE = ctypes.c_void_p(0x10000)      # a 64 KiB-aligned address: never dereferenced
+
+
+def test_quant_act_validation(L):
+    f = L.fp8bq_quant_act
+    assert f(FAKE, -1, 128, 128, FAKE, 128, FAKE, 4, 0, None) == INVALID
+    assert f(FAKE, 4, 128, 64, FAKE, 128, FAKE, 4, 0, None) == INVALID     # ldx < K
+    assert f(FAKE, 4, 128, 128, FAKE, 128, FAKE, 3, 0, None) == INVALID    # ldsa < M
+    assert f(None, 4, 128, 128, FAKE, 128, FAKE, 4, 0, None) == INVALID
+    assert f(FAKE, 4, 128, 128, FAKE, 128, FAKE, 4, 7, None) == INVALID    # bad mode
+    assert f(None, 0, 128, 128, None, 128, None, 4, 0, None) == 0          # empty: no-op
+
+
+def test_gemm_validation(L):
+    g = L.fp8bq_gemm
+
+    def call(M=256, N=256, K=256, lda=256, ldw=256, ldy=256, ldsa=256, qa=FAKE, y=FAKE, mode=0):
+        return g(qa, lda, FAKE, ldsa, FAKE, ldw, FAKE, y, ldy, M, N, K, mode, None)
+    assert call(K=200, lda=256, ldw=256) == UNSUPPORTED                   # K % 128
+    assert call(lda=128) == INVALID                                       # lda < K
+    assert call(ldy=255) == INVALID                                       # ldy < N
+    assert call(ldy=260) == INVALID                                       # ldy % 8
+    assert call(ldsa=255) == INVALID                                      # ldsa < M
+    assert call(ldsa=258) == INVALID                                      # ldsa % 4
+    assert call(qa=ctypes.c_void_p(0x10008)) == INVALID                   # 16-byte alignment
+    assert call(M=-1) == INVALID
+    assert call(M=0) == 0 and call(N=0) == 0                              # empty: no-op
+    assert call(mode=2) == INVALID
+    assert L.fp8bq_gemm_ex(FAKE, 256, FAKE, 256, FAKE, 256, FAKE, FAKE, 256, 256, 256, 256, 0, 2, None) == INVALID
+
+
+def test_recalibrate_validation(L):
+    arr = (fq.WeightDesc * 2)()
+    arr[0] = fq.WeightDesc(0x10000, 0x20000, 0x30000, 128, 128, 128, 128)
+    arr[1] = fq.WeightDesc(0x10000, 0x20000, 0x30000, 128, 128, 64, 128)   # ldw < K
+    assert L.fp8bq_recalibrate(arr, 2, 1, None) == INVALID
+    assert L.fp8bq_recalibrate(arr, -1, 1, None) == INVALID
+    assert L.fp8bq_recalibrate(arr, 0, 1, None) == 0

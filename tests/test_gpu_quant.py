@@ -1,0 +1,172 @@
+"""GPU parity of the quantizers against the CPU oracle: codes and scales bit-exact.
+
+Covers the element encoder over all 2^32 float32 patterns, the division over a
+sweep of (tile amax, element) pairs, the single-linear and Llama-8B-shaped
+activations at full size, ragged and unaligned shapes (vector and scalar
+paths), weight tiles of every Llama-8B projection, and the multi-tensor
+recalibration.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fp8_block_scaled_fp8bq_b200 as fq
+import fp8bq_workloads as wl
+import oracle
+from helpers import bf16_bits, f32, need_gpu, u8
+
+pytestmark = pytest.mark.gpu
+MODES = [fq.SCALE_FP32, fq.SCALE_POW2]
+
+
+@pytest.fixture(autouse=True)
+def _gpu_and_clean_error_word():
+    need_gpu()
+    yield
+    st, word = fq.device_error()
+    assert st == 0 and word == 0, "device error word 0x%x" % word
+
+
+def check_act(x, mode, q=None, sa=None, ldsa=None):
+    """Quantize x on the GPU and compare codes and scales with the oracle."""
+    M, K = x.shape
+    q, sa = fq.quant_act(x, mode, q=q, sa=sa)
+    torch.cuda.synchronize()
+    oq, osa = oracle.quant_act(bf16_bits(x), mode, ldsa=sa.shape[1])
+    gq = u8(q)[:, :K] if q.dim() == 2 else u8(q)
+    assert np.array_equal(gq, oq), "codes differ at %s" % (np.argwhere(gq != oq)[:5],)
+    g = f32(sa)[:, :M]
+    assert np.array_equal(g.view(np.uint32), osa[:, :M].view(np.uint32)), "scales differ"
+
+
+def test_e4m3_encoder_all_fp32_patterns():
+    step = 1 << 26
+    for start in range(-(1 << 31), 1 << 31, step):
+        x = torch.arange(start, start + step, dtype=torch.int32, device="cuda").view(torch.float32)
+        q = u8(fq.e4m3_encode(x))
+        first = start & 0xFFFFFFFF
+        ref = oracle.encode_patterns(first, step)
+        pats = np.arange(first, first + step, dtype=np.uint32)
+        nan = ((pats & 0x7F800000) == 0x7F800000) & ((pats & 0x7FFFFF) != 0)  # outside the contract
+        ok = (q == ref) | nan
+        assert ok.all(), "first mismatch at pattern 0x%08x" % int(pats[np.argmin(ok)])
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_division_sweep_over_tile_amax(mode):
+    """Rows whose amax is a chosen bf16 value and whose other elements run over
+    every bf16 pattern below it: the quotient x/s for many (amax, x) pairs."""
+    rng = np.random.default_rng(7)
+    amax_bits = np.unique(np.concatenate([
+        np.arange(1, 0x7F80, 97, dtype=np.uint16), np.array([1, 2, 0x7F, 0x80, 0x3F80, 0x43E0, 0x7F7F], np.uint16),
+        rng.integers(0x0080, 0x7F80, 200).astype(np.uint16)]))
+    allx = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    allx = allx[(allx & 0x7FFF) < 0x7F80]                 # finite patterns only
+    K = 128
+    rows = []
+    for a in amax_bits:
+        ok = allx[(allx & 0x7FFF) <= a]
+        for i in range(0, ok.size, K - 1):
+            chunk = ok[i:i + K - 1]
+            row = np.zeros(K, dtype=np.uint16)
+            row[0] = a
+            row[1:1 + chunk.size] = chunk
+            rows.append(row)
+    xb = np.stack(rows)
+    x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
+    check_act(x, mode)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_single_linear_activation(mode):
+    x, _ = wl.single_linear(seed=0)
+    check_act(x.cuda(), mode)
+
+
+@pytest.mark.parametrize("K", [4096, 14336])
+def test_llama_prefill_activation_full(K):
+    x = wl.activations(wl.PREFILL_TOKENS, K, seed=K, device="cuda")
+    check_act(x, fq.SCALE_FP32)
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("M,K", [(1, 128), (3, 8), (129, 136), (37, 300), (5, 1), (64, 4096), (17, 1000)])
+def test_activation_ragged_shapes(mode, M, K):
+    x = wl.activations(M, K, seed=M * 1000 + K, n_out=min(4, K))
+    check_act(x.cuda(), mode)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_activation_unaligned_views(mode):
+    base = wl.activations(70, 520, seed=3, n_out=5).cuda()
+    x = base[:, 3:259]                                    # ldx = 520, pointer off by 6 bytes
+    q = torch.zeros((70, 300), dtype=torch.uint8, device="cuda")[:, 1:257]
+    check_act(x, mode, q=q)
+
+
+def test_activation_special_values():
+    x = torch.zeros((4, 256), dtype=torch.bfloat16)
+    x[1, 3] = -0.0
+    x[2, :128] = torch.linspace(-448, 448, 128)
+    x[2, 5] = -1e-30                                      # negative underflow keeps its sign
+    x[3, 130] = 3.0e38                                    # huge amax
+    x[3, 131] = 1e-38
+    for mode in MODES:
+        check_act(x.cuda(), mode)
+
+
+def check_weight(w, mode):
+    q, sw = fq.quant_weight(w, mode)
+    torch.cuda.synchronize()
+    oq, osw = oracle.quant_weight(bf16_bits(w), mode)
+    assert np.array_equal(u8(q), oq)
+    assert np.array_equal(f32(sw).view(np.uint32), osw.view(np.uint32))
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("name", list(wl.LLAMA8B_SHAPES))
+def test_weight_llama_shapes(mode, name):
+    N, K = wl.LLAMA8B_SHAPES[name]
+    check_weight(wl.weights(N, K, seed=N + K, device="cuda"), mode)
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("N,K", [(1, 1), (200, 300), (128, 128), (129, 257), (300, 1000)])
+def test_weight_ragged(mode, N, K):
+    check_weight(wl.weights(N, K, seed=N * 7 + K).cuda(), mode)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_recalibrate_layer_equals_oracle(mode):
+    tensors = []
+    for name, (N, K) in wl.LLAMA8B_SHAPES.items():
+        w = wl.weights(N, K, seed=wl.layer_weight_seed(0, name), device="cuda")
+        w = wl.weight_step(w, seed=wl.layer_weight_seed(0, name) + 1)
+        q = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+        s = torch.empty((fq.ceil_div(N, 128), fq.ceil_div(K, 128)), dtype=torch.float32, device="cuda")
+        tensors.append((w, q, s))
+    odd = wl.weights(200, 300, seed=5).cuda()              # a ragged tensor in the same launch
+    tensors.append((odd, torch.empty((200, 300), dtype=torch.uint8, device="cuda"),
+                    torch.empty((2, 3), dtype=torch.float32, device="cuda")))
+    fq.recalibrate(tensors, mode)
+    torch.cuda.synchronize()
+    for w, q, s in tensors:
+        oq, osw = oracle.quant_weight(bf16_bits(w), mode)
+        assert np.array_equal(u8(q), oq)
+        assert np.array_equal(f32(s).view(np.uint32), osw.view(np.uint32))
+
+
+def test_recalibrate_many_tensors_crosses_launch_chunks():
+    tensors = []
+    for i in range(300):                                  # > 128 descriptors: several launches
+        N, K = 64 + (i % 5) * 40, 128 + (i % 3) * 72
+        w = wl.weights(N, K, seed=i).cuda()
+        tensors.append((w, torch.empty((N, K), dtype=torch.uint8, device="cuda"),
+                        torch.empty((fq.ceil_div(N, 128), fq.ceil_div(K, 128)), dtype=torch.float32,
+                                    device="cuda")))
+    fq.recalibrate(tensors, fq.SCALE_POW2)
+    torch.cuda.synchronize()
+    for w, q, s in tensors[::7]:
+        oq, osw = oracle.quant_weight(bf16_bits(w), fq.SCALE_POW2)
+        assert np.array_equal(u8(q), oq)
+        assert np.array_equal(f32(s), osw)
