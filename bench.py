@@ -409,8 +409,114 @@ def reference(args):
     print(json.dumps(line), flush=True)
 
 
+CASES = (["gemm:" + n for n in NAMES] + ["decode:" + n for n in NAMES] +
+         ["quant_act:4096", "quant_act:14336", "recalibrate:layer", "quant_weight:gate_up", "moe:up", "moe:down"])
+
+
+def decode_bytes(M, N, K):
+    """Weight codes + weight scales + bf16 activations in + bf16 out."""
+    return N * K + ((N + 127) // 128) * (K // 128) * 4 + M * K * 2 + M * N * 2
+
+
+def moe_bytes(R, E, N, K):
+    """Expert weights + activation codes/scales + bf16 out (each read once)."""
+    return E * N * K + E * (N // 128) * (K // 128) * 4 + R * K + R * (K // 128) * 4 + R * N * 2
+
+
+def run_case(args):
+    """One kernel on one shape, for profiling (ncu) and per-kernel timing: --warmup
+    untimed launches, then --steps timed launches; prints a JSON line with the
+    average launch time.  Not the benchmark line."""
+    import fp8_block_scaled_fp8bq_b200 as fq
+    fq.lib()
+    M = args.tokens
+    kind, what = args.case.split(":")
+    dev = torch.device("cuda", 0)
+    mode = fq.SCALE_POW2 if args.pow2 else fq.SCALE_FP32
+    if kind == "gemm":
+        N, K = wl.LLAMA8B_SHAPES[what]
+        x = wl.activations(M, K, seed=1, device=dev)
+        w = wl.weights(N, K, seed=2, device=dev)
+        qa, sa = fq.quant_act(x, mode)
+        qw, sw = fq.quant_weight(w, mode)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.gemm(qa, sa, qw, sw, mode, out=y)  # noqa: E731
+        work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
+    elif kind == "decode":
+        N, K = wl.LLAMA8B_SHAPES[what]
+        x = wl.activations(M, K, seed=1, device=dev)
+        w = wl.weights(N, K, seed=2, device=dev)
+        qw, sw = fq.quant_weight(w, mode)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(256, fq.gemm_decode_workspace_size(M, N, K)), dtype=torch.uint8, device=dev)
+        fn = lambda: fq.gemm_decode(x, qw, sw, mode, out=y, ws=ws)  # noqa: E731
+        work, unit = decode_bytes(M, N, K) / 1e9, "GB/s"
+    elif kind == "moe":
+        moe = wl.moe_layer(seed=0, device=dev)
+        x, w = moe["x_" + what], moe["w_" + what]
+        E, N, K = w.shape
+        R = x.shape[0]
+        qa, sa = fq.quant_act(x, mode)
+        qw, sw = fq.quant_weight(w.reshape(E * N, K), mode)
+        qw, sw = qw.view(E, N, K), sw.view(E, N // 128, K // 128)
+        off = moe["offsets"].to(torch.int32).to(dev)
+        y = torch.empty((R, N), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.grouped_gemm(qa, sa, qw, sw, off, mode, out=y)  # noqa: E731
+        work, unit = moe_bytes(R, E, N, K) / 1e9, "GB/s"
+        print(json.dumps({"case": args.case, "flops": 2.0 * R * N * K}))
+    elif kind == "quant_act":
+        K = int(what)
+        x = wl.activations(M, K, seed=1, device=dev)
+        q = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        sa = torch.empty(fq.act_scale_shape(M, K), dtype=torch.float32, device=dev)
+        fn = lambda: fq.quant_act(x, mode, q=q, sa=sa)  # noqa: E731
+        work, unit = quant_act_bytes(M, K) / 1e9, "GB/s"
+    elif kind == "quant_weight":
+        N, K = wl.LLAMA8B_SHAPES[what]
+        w = wl.weights(N, K, seed=2, device=dev)
+        q = torch.empty((N, K), dtype=torch.uint8, device=dev)
+        sw = torch.empty((fq.ceil_div(N, 128), fq.ceil_div(K, 128)), dtype=torch.float32, device=dev)
+        fn = lambda: fq.quant_weight(w, mode, q=q, sw=sw)  # noqa: E731
+        work, unit = recal_bytes(N, K) / 1e9, "GB/s"
+    else:
+        step = LayerStep(fq, dev, mode=mode)
+        fn = lambda: fq.recalibrate(step.recal_list, mode)  # noqa: E731
+        work, unit = sum(recal_bytes(N, K) for N, K in wl.LLAMA8B_SHAPES.values()) / 1e9, "GB/s"
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if args.graph:
+        # launch-bound cases: capture the launches in a CUDA graph so the host
+        # does not pace the GPU; one replay runs --steps calls
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(args.steps):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        t0.record()
+        g.replay()
+        t1.record()
+    else:
+        t0.record()
+        for _ in range(args.steps):
+            fn()
+        t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / args.steps
+    print(json.dumps({"case": args.case, "tokens": M, "pow2": bool(args.pow2), "graph": bool(args.graph),
+                      "launches": args.steps,
+                      "ms_per_launch": round(ms, 5), "rate": round(work / (ms / 1e3), 1), "unit": unit}))
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--case", choices=CASES, default=None,
+                    help="time one kernel on one shape instead of the benchmark step (for profiling)")
+    ap.add_argument("--tokens", type=int, default=M_TOKENS, help="M for --case")
+    ap.add_argument("--pow2", action="store_true", help="power-of-2 scales for --case")
+    ap.add_argument("--graph", action="store_true", help="--case: time a CUDA graph of --steps calls")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
@@ -418,7 +524,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    if args.impl == "reference":
+    if args.case:
+        run_case(args)
+    elif args.impl == "reference":
         reference(args)
     else:
         ours(args)

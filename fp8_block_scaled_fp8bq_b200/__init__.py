@@ -176,7 +176,7 @@ def gemm_decode(x, qw, sw, mode=SCALE_FP32, out=None, ws=None, stream=None):
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     need = gemm_decode_workspace_size(M, N, K)
     if ws is None:
-        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
     _check(lib().fp8bq_gemm_decode(_ptr(x), _ld(x), _ptr(qw), _ld(qw), _ptr(sw), _ptr(out), _ld(out), M, N, K,
                                    mode, _ptr(ws), ws.numel(), _stream(stream)), "fp8bq_gemm_decode")
     return out

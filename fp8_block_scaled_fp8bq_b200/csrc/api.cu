@@ -75,6 +75,21 @@ bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                  uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
+                  CUtensorMapSwizzle swizzle) {
+  CUtensorMap probe;
+  if (!make_tmap_2d(&probe, dtype, base, d0, d1, stride1_bytes, box0, box1, swizzle)) return false;  // loads g_encode
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = g_encode(map, dtype, 3, const_cast<void *>(base), dims, strides, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace fp8bq
 
 using namespace fp8bq;
@@ -125,7 +140,7 @@ fp8bq_status fp8bq_get_device_error(uint64_t *code) {
   unsigned long long v = 0, w = 0;
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-  cudaError_t (*takers[])(unsigned long long *) = {take_device_error_gemm};
+  cudaError_t (*takers[])(unsigned long long *) = {take_device_error_gemm, take_device_error_decode, take_device_error_native};
   for (auto take : takers) {
     e = take(&w);
     if (e != cudaSuccess) return cuda_fail(e, "read device error word");
@@ -197,6 +212,40 @@ fp8bq_status fp8bq_gemm_ex(const uint8_t *qa, int64_t lda, const float *sa, int6
   if (st != FP8BQ_OK || M == 0 || N == 0) return st;
   return launch_gemm(qa, lda, sa, ldsa, qw, ldw, sw, y, ldy, M, N, K, mode, variant,
                      static_cast<cudaStream_t>(stream));
+}
+
+size_t fp8bq_gemm_decode_workspace_size(int64_t M, int64_t N, int64_t K) { return decode_workspace_size(M, N, K); }
+
+fp8bq_status fp8bq_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, int64_t ldw, const float *sw, void *y,
+                               int64_t ldy, int64_t M, int64_t N, int64_t K, int mode, void *ws, size_t ws_bytes,
+                               void *stream) {
+  if (M < 0 || N < 0 || K < 0 || bad_mode(mode)) return FP8BQ_ERR_INVALID_ARG;
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return FP8BQ_OK;
+  if (y == nullptr || ldy < N || !aligned(y, 16) || ldy % 8 != 0) return FP8BQ_ERR_INVALID_ARG;
+  if (K == 0) {
+    cudaError_t e = cudaMemset2DAsync(y, (size_t)ldy * 2, 0, (size_t)N * 2, (size_t)M, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FP8BQ_OK : cuda_fail(e, "memset(y)");
+  }
+  if (K % 128 != 0 || M > 256) return FP8BQ_ERR_UNSUPPORTED;
+  if (!x || !qw || !sw || ldx < K || ldw < K) return FP8BQ_ERR_INVALID_ARG;
+  if (!aligned(x, 2) || !aligned(qw, 16) || ldw % 16 != 0 || !aligned(sw, 4)) return FP8BQ_ERR_INVALID_ARG;
+  return launch_gemm_decode(x, ldx, qw, ldw, sw, y, ldy, M, N, K, mode, ws, ws_bytes,
+                            static_cast<cudaStream_t>(stream));
+}
+
+fp8bq_status fp8bq_grouped_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                                const float *sw, const int32_t *offsets, int E, int64_t total_rows, int64_t N,
+                                int64_t K, void *y, int64_t ldy, int mode, void *stream) {
+  if (E < 1 || E > kMaxExperts || total_rows < 0) return E > kMaxExperts ? FP8BQ_ERR_UNSUPPORTED : FP8BQ_ERR_INVALID_ARG;
+  if (!offsets || !aligned(offsets, 4)) return FP8BQ_ERR_INVALID_ARG;
+  if (N % 8 != 0) return FP8BQ_ERR_UNSUPPORTED;
+  if ((int64_t)E * N >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
+  // the expert weights are dense [E][N][K]: lda-like checks apply with ldw = K
+  fp8bq_status st = check_gemm_operands(qa, lda, sa, ldsa, qw, K, sw, y, ldy, total_rows, N, K, mode);
+  if (st != FP8BQ_OK || total_rows == 0 || N == 0) return st;
+  return launch_grouped_gemm(qa, lda, sa, ldsa, qw, sw, offsets, E, total_rows, N, K, y, ldy,
+                             static_cast<cudaStream_t>(stream));
 }
 
 fp8bq_status fp8bq_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw, int64_t ldw,

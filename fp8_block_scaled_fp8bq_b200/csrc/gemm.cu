@@ -1,9 +1,13 @@
 // Block-scaled FP8 GEMM for sm_100a: Y[M,N] (bf16) = X[M,K] . W[N,K]^T with
-// E4M3 operands, 1x128 activation scales and 128x128 weight scales.
+// E4M3 operands, 1x128 activation scales and 128x128 weight scales; and its
+// grouped (mixture-of-experts) form, where rows [offsets[e], offsets[e+1]) of
+// the expert-sorted activations multiply expert e's weight.
 //
 // Method: "NVIDIA NeMo RL Achieves 48% Speedup With End-to-End FP8 Precision
 // Training", section "Technical breakthrough": the linear layers run in FP8 on
-// block-wise quantized E4M3 operands (activations 1x128, weights 128x128).
+// block-wise quantized E4M3 operands (activations 1x128, weights 128x128);
+// section "Real-world performance gains": the recipe also runs on a
+// mixture-of-experts model.
 //
 // Promotion design (FP32 scales).  A scale varies with the row m (activation)
 // and with the 128-column block of n (weight) and with the K-block, so it
@@ -20,18 +24,27 @@
 //               (128x256x32) per K-block into one of two 256-column TMEM
 //               buffers; tcgen05.commit frees the smem stage and hands the
 //               buffer to the epilogue.
-//   warps 2-3   idle (warpgroup 0 gives its registers to the epilogue with
-//               setmaxnreg).
+//   warps 2-3   idle after the prologue (warpgroup 0 gives its registers to
+//               the epilogue with setmaxnreg).
 //   warps 4-11  promotion + epilogue (warpgroups 1 and 2): warp w reads TMEM
 //               lanes 32*(w%4)..+31 (its 32 rows) and columns
 //               [128*h, 128*h+128) with h = (w-4)/4, i.e. exactly one 128-wide
 //               weight block, so each thread needs one scale product per
-//               K-block and holds 128 FP32 accumulators.  After the last
-//               K-block the accumulators go to shared memory as bf16 and out
-//               with TMA stores.
+//               K-block and holds 128 FP32 accumulators (packed fma pairs).
+//               After the last K-block the accumulators leave as bf16: TMA
+//               stores (dense) or row-masked coalesced stores (grouped, where
+//               a 128-row tile can run past its expert's last row).
 // The MMA of K-block kb+1 overlaps the promotion of kb (two TMEM buffers), and
 // the stores of one tile overlap the MMAs of the next.
+//
+// Grouped scheduling is on the device: every CTA reads offsets[0..E], builds
+// the prefix of tile counts per expert in shared memory, and maps each tile
+// id to (expert, 128-row block, 256-column block) by binary search, so no
+// host synchronization is needed.  Tiles of one expert are consecutive (row
+// blocks fastest), so concurrently running CTAs share that expert's weight
+// tiles in L2.
 #include <cuda_bf16.h>
+#include <string.h>
 
 #include <algorithm>
 
@@ -47,12 +60,12 @@ constexpr int kABytes = BM * BK;
 constexpr int kBBytes = BN * BK;
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kEpiWarps = 8;
-constexpr int kEpiBufBytes = 32 * 128;  // 32 rows x 64 bf16
 constexpr int kThreads = 128 + kEpiWarps * 32;
 // Register split (setmaxnreg): the launch gives every thread kLaunchRegs; the
 // producer/MMA warpgroup drops to kLowRegs and the two epilogue warpgroups
 // rise to kHighRegs.  128 * kLowRegs + 256 * kHighRegs must not exceed
-// 384 * kLaunchRegs (the build checks ptxas's count against kLaunchRegs).
+// 384 * kLaunchRegs (the build checks ptxas's count against kLaunchRegs, and
+// the launcher checks it again at run time).
 constexpr int kLaunchRegs = 168;
 constexpr int kLowRegs = 56;
 constexpr int kHighRegs = 224;
@@ -60,25 +73,73 @@ static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "regis
 constexpr int kTmemCols = 2 * BN;
 constexpr int kGroupM = 16;
 constexpr int kBarBytes = 256;
-constexpr int kSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiBufBytes + kBarBytes + 1024;
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+// Per-warp bf16 staging: dense = 32 rows x 64 columns in the TMA 128-byte
+// swizzle; grouped = 32 rows x 32 columns (64-byte rows, 16-byte chunks XOR
+// ((row >> 1) & 3), conflict-free for both the row writes and the copy-out).
+template <bool G>
+struct Cfg {
+  static constexpr int kEpiBufBytes = G ? 32 * 64 : 32 * 128;
+  static constexpr int kSchedBytes = G ? 2 * (kMaxExperts + 1) * 4 : 0;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiBufBytes + kBarBytes + kSchedBytes + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 
 struct GemmArgs {
   const float *sa;
   const float *sw;
   int64_t ldsa;
-  int32_t M, N, KB, NB;
-  int32_t num_m, num_n;
+  int32_t M, N, KB, NB;     // grouped: M = total rows
+  int32_t num_m, num_n;     // dense tile grid; grouped: num_n only
+  // grouped only
+  const int32_t *offsets;   // [E+1], device
+  int32_t E;
+  uint16_t *y;              // output base for the masked stores (bf16 bits)
+  int64_t ldy;
 };
 
-__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int &mb, int &nb) {
-  const int per_group = kGroupM * num_n;
+// A tile: rows [row0, row_end) of the activations (row_end clips the last
+// tile of a matrix or of an expert), 256-column block nb, expert e.
+struct Tile {
+  int e, row0, row_end, nb;
+};
+
+__device__ __forceinline__ Tile dense_tile(int t, const GemmArgs &a) {
+  const int per_group = kGroupM * a.num_n;
   const int g = t / per_group;
   const int first_m = g * kGroupM;
-  const int gm = min(num_m - first_m, kGroupM);
+  const int gm = min(a.num_m - first_m, kGroupM);
   const int r = t - g * per_group;
-  mb = first_m + r % gm;
-  nb = r / gm;
+  Tile tl;
+  tl.e = 0;
+  tl.row0 = (first_m + r % gm) * BM;
+  tl.row_end = a.M;
+  tl.nb = r / gm;
+  return tl;
+}
+
+// prefix[e] = tiles of experts before e (prefix[E] = total); offs = clamped offsets.
+__device__ __forceinline__ Tile grouped_tile(int t, const GemmArgs &a, const int *prefix, const int *offs) {
+  int lo = 0, hi = a.E - 1;  // last expert whose first tile is <= t (empty experts are skipped)
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  const int local = t - prefix[lo];
+  const int mt_e = (offs[lo + 1] - offs[lo] + BM - 1) / BM;
+  Tile tl;
+  tl.e = lo;
+  tl.nb = local / mt_e;
+  tl.row0 = offs[lo] + (local - tl.nb * mt_e) * BM;
+  tl.row_end = offs[lo + 1];
+  return tl;
+}
+
+template <bool G>
+__device__ __forceinline__ Tile tile_at(int t, const GemmArgs &a, const int *prefix, const int *offs) {
+  if constexpr (G) return grouped_tile(t, a, prefix, offs);
+  else return dense_tile(t, a);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -90,7 +151,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 struct Smem {
   uint8_t *a;        // kStages x [128 rows x 128 B], 128-byte swizzled
   uint8_t *b;        // kStages x [256 rows x 128 B], 128-byte swizzled
-  uint8_t *epi;      // kEpiWarps x [32 rows x 128 B] bf16 staging
+  uint8_t *epi;      // kEpiWarps x bf16 staging
   uint64_t *full;    // [kStages] TMA bytes landed
   uint64_t *empty;   // [kStages] MMAs done reading the stage
   uint64_t *tfull;   // [2] K-block partial ready in TMEM buffer
@@ -98,15 +159,18 @@ struct Smem {
   uint64_t *drain;   // MMA drain on the error path
   uint32_t *tmem_slot;
   volatile int *abort_flag;
+  int *prefix;       // grouped: [E+1] tile prefix
+  int *offs;         // grouped: [E+1] clamped offsets
 };
 
+template <bool G>
 __device__ __forceinline__ Smem carve(uint8_t *raw) {
   Smem s;
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   s.a = base;
   s.b = base + kStages * kABytes;
   s.epi = s.b + kStages * kBBytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(s.epi + kEpiWarps * kEpiBufBytes);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(s.epi + kEpiWarps * Cfg<G>::kEpiBufBytes);
   s.full = bars;
   s.empty = bars + kStages;
   s.tfull = bars + 2 * kStages;
@@ -114,28 +178,78 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
   s.drain = s.tempty + 2;
   s.tmem_slot = reinterpret_cast<uint32_t *>(s.drain + 1);
   s.abort_flag = reinterpret_cast<volatile int *>(s.tmem_slot + 1);
+  s.prefix = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(bars) + kBarBytes);
+  s.offs = s.prefix + (kMaxExperts + 1);
   return s;
+}
+
+// Grouped prologue (one warp): clamp the offsets into [0, M] and make them
+// nondecreasing (so offsets that break the contract cannot cause an
+// out-of-bounds access), then the exclusive prefix of tiles per expert.
+__device__ __forceinline__ void build_schedule(const Smem &S, const GemmArgs &a, int lane) {
+  const int n = a.E + 1;
+  const int per = (n + 31) / 32;
+  const int i0 = min(lane * per, n), i1 = min(i0 + per, n);
+  int run = 0;
+  for (int i = i0; i < i1; ++i) {
+    int v = __ldg(a.offsets + i);
+    v = max(0, min(v, a.M));
+    run = max(run, v);
+    S.offs[i] = run;
+  }
+  // max-scan of the chunk maxima across lanes
+  int incl = run;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl = max(incl, o);
+  }
+  int before = __shfl_up_sync(0xffffffffu, incl, 1);
+  if (lane == 0) before = 0;
+  for (int i = i0; i < i1; ++i) S.offs[i] = max(S.offs[i], before);
+  __syncwarp();
+  // tiles per expert and their exclusive prefix
+  int sum = 0;
+  for (int i = i0; i < i1 && i < a.E; ++i) sum += ((S.offs[i + 1] - S.offs[i] + BM - 1) / BM) * a.num_n;
+  int excl = sum;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, excl, d);
+    if (lane >= d) excl += o;
+  }
+  excl -= sum;
+  for (int i = i0; i < i1; ++i) {
+    S.prefix[i] = excl;
+    if (i < a.E) excl += ((S.offs[i + 1] - S.offs[i] + BM - 1) / BM) * a.num_n;
+  }
+}
+
+template <bool G>
+__device__ __forceinline__ int total_tiles(const Smem &S, const GemmArgs &a) {
+  if constexpr (G) return S.prefix[a.E];
+  else return a.num_m * a.num_n;
 }
 
 // TMA producer (one thread): stream the A and B tiles of every K-block of this
 // CTA's tiles through the stage ring.
+template <bool G>
 __device__ __forceinline__ void run_producer(const Smem &S, const CUtensorMap *tmA, const CUtensorMap *tmB,
                                              const GemmArgs &args) {
-  const int total = args.num_m * args.num_n;
+  const int total = total_tiles<G>(S, args);
   int stage = 0;
   uint32_t phase = 0, armed = 0, armed_parity = 0;
   bool ok = true;
   for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-    int mb, nb;
-    tile_coords(t, args.num_m, args.num_n, mb, nb);
+    const Tile tl = tile_at<G>(t, args, S.prefix, S.offs);
     for (int kb = 0; kb < args.KB; ++kb) {
       if (!mbar_wait(&S.empty[stage], phase ^ 1, S.abort_flag, kSiteProducerEmpty)) {
         ok = false;
         break;
       }
       mbar_arrive_expect_tx(&S.full[stage], kStageBytes);
-      tma_load_2d(S.a + stage * kABytes, tmA, &S.full[stage], kb * BK, mb * BM);
-      tma_load_2d(S.b + stage * kBBytes, tmB, &S.full[stage], kb * BK, nb * BN);
+      tma_load_2d(S.a + stage * kABytes, tmA, &S.full[stage], kb * BK, tl.row0);
+      if constexpr (G) tma_load_3d(S.b + stage * kBBytes, tmB, &S.full[stage], kb * BK, tl.nb * BN, tl.e);
+      else tma_load_2d(S.b + stage * kBBytes, tmB, &S.full[stage], kb * BK, tl.nb * BN);
       armed |= 1u << stage;
       armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
       if (++stage == kStages) {
@@ -152,8 +266,9 @@ __device__ __forceinline__ void run_producer(const Smem &S, const CUtensorMap *t
 
 // MMA issuer (one thread): per K-block, four 128x256x32 E4M3 MMAs into a fresh
 // TMEM buffer (the first one overwrites, the rest accumulate).
+template <bool G>
 __device__ __forceinline__ void run_mma(const Smem &S, uint32_t tmem_base, const GemmArgs &args) {
-  const int total = args.num_m * args.num_n;
+  const int total = total_tiles<G>(S, args);
   const uint32_t idesc = idesc_f8f6f4_e4m3_f32(BM, BN);
   int stage = 0, buf = 0;
   uint32_t phase = 0, bphase = 0;
@@ -192,36 +307,51 @@ __device__ __forceinline__ void run_mma(const Smem &S, uint32_t tmem_base, const
 }
 
 // Promotion + epilogue (one warp of the two epilogue warpgroups).
+template <bool G>
 __device__ __forceinline__ void run_epilogue(const Smem &S, uint32_t tmem_base, const CUtensorMap *tmY,
                                              const GemmArgs &args, int warp, int lane) {
-  const int total = args.num_m * args.num_n;
+  const int total = total_tiles<G>(S, args);
   const int KB = args.KB;
   const int ew = warp - 4;
   const int quarter = warp & 3;  // TMEM lanes this warp may access
   const int half = ew >> 2;      // 128-column half of the tile = one weight block
   const int row = quarter * 32 + lane;
-  uint8_t *ebuf = S.epi + ew * kEpiBufBytes;
+  uint8_t *ebuf = S.epi + ew * Cfg<G>::kEpiBufBytes;
   int buf = 0;
   uint32_t bphase = 0;
   for (int t = blockIdx.x; t < total; t += gridDim.x) {
-    int mb, nb;
-    tile_coords(t, args.num_m, args.num_n, mb, nb);
-    const int m = mb * BM + row;
-    const int wn = nb * 2 + half;
-    const bool live = m < args.M && wn < args.NB;
+    const Tile tl = tile_at<G>(t, args, S.prefix, S.offs);
+    const int m = tl.row0 + row;
+    const int wn = tl.nb * 2 + half;
+    const bool live = m < tl.row_end && wn < args.NB;
     const float *sa_p = args.sa + m;
-    const float *sw_p = args.sw + (int64_t)wn * KB;
-    float acc[128];
+    const float *sw_p = args.sw + ((int64_t)tl.e * args.NB + wn) * KB;
+    // 128 FP32 accumulators as 64 pairs: the promotion is a packed fma (two
+    // lanes of FP32 per instruction).
+    float2 acc[64];
 #pragma unroll
-    for (int j = 0; j < 128; ++j) acc[j] = 0.f;
-    // scale products for K-blocks kb and kb+1 (loaded two K-blocks ahead)
-    float sc0 = live ? __ldg(sa_p) * __ldg(sw_p) : 0.f;
-    float sc1 = (live && KB > 1) ? __ldg(sa_p + args.ldsa) * __ldg(sw_p + 1) : 0.f;
+    for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.f, 0.f);
+    // Scale factors are loaded two K-blocks before use so their latency is
+    // hidden: (a0, w0) belong to kb, (a1, w1) to kb+1.
+    float a0 = 0.f, w0 = 0.f, a1 = 0.f, w1 = 0.f;
+    if (live) {
+      a0 = __ldg(sa_p);
+      w0 = __ldg(sw_p);
+      if (KB > 1) {
+        a1 = __ldg(sa_p + args.ldsa);
+        w1 = __ldg(sw_p + 1);
+      }
+    }
     bool ok = true;
     for (int kb = 0; kb < KB; ++kb) {
-      const float sc = sc0;
-      sc0 = sc1;
-      sc1 = (live && kb + 2 < KB) ? __ldg(sa_p + (int64_t)(kb + 2) * args.ldsa) * __ldg(sw_p + kb + 2) : 0.f;
+      const float sc = a0 * w0;
+      a0 = a1;
+      w0 = w1;
+      if (live && kb + 2 < KB) {
+        a1 = __ldg(sa_p + (int64_t)(kb + 2) * args.ldsa);
+        w1 = __ldg(sw_p + kb + 2);
+      }
+      const float2 sc2 = make_float2(sc, sc);
       const bool got = mbar_wait(&S.tfull[buf], bphase, S.abort_flag, kSiteEpiTmemFull);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
@@ -230,17 +360,20 @@ __device__ __forceinline__ void run_epilogue(const Smem &S, uint32_t tmem_base, 
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN + half * 128);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + 32 * c, r);
+      for (int c = 0; c < 2; ++c) {  // two 64-column halves, two loads in flight each
+        uint32_t r[64];
+        tmem_ld_32x32b_x32(taddr + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld_32x32b_x32(taddr + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         tmem_ld_wait();
-        if (c == 3) {  // the buffer has been read: hand it back to the MMA warp
+        if (c == 1) {  // the buffer has been read: hand it back to the MMA warp
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.tempty[buf]);
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc[32 * c + j] = fmaf(__uint_as_float(r[j]), sc, acc[32 * c + j]);
+        for (int j = 0; j < 32; ++j)
+          acc[32 * c + j] =
+              __ffma2_rn(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])), sc2, acc[32 * c + j]);
       }
       if (++buf == 2) {
         buf = 0;
@@ -248,44 +381,82 @@ __device__ __forceinline__ void run_epilogue(const Smem &S, uint32_t tmem_base, 
       }
     }
     if (!ok) break;
-    // bf16 out: two 64-column chunks through this warp's 4 KB staging buffer,
-    // written in the 128-byte swizzled order the TMA store expects.
+
+    if constexpr (!G) {
+      // bf16 out: two 64-column chunks through this warp's 4 KB staging buffer,
+      // written in the 128-byte swizzled order the TMA store expects.
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      if (lane == 0) bulk_wait_group_read0();
-      __syncwarp();
-      uint8_t *rowp = ebuf + lane * 128;
+      for (int c = 0; c < 2; ++c) {
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+        uint8_t *rowp = ebuf + lane * 128;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float *a = &acc[c * 64 + j * 8];
-        uint4 pk;
-        pk.x = pack_bf16x2(a[0], a[1]);
-        pk.y = pack_bf16x2(a[2], a[3]);
-        pk.z = pack_bf16x2(a[4], a[5]);
-        pk.w = pack_bf16x2(a[6], a[7]);
-        *reinterpret_cast<uint4 *>(rowp + ((j ^ (lane & 7)) << 4)) = pk;
+        for (int j = 0; j < 8; ++j) {
+          const float2 *a = &acc[c * 32 + j * 4];
+          uint4 pk;
+          pk.x = pack_bf16x2(a[0].x, a[0].y);
+          pk.y = pack_bf16x2(a[1].x, a[1].y);
+          pk.z = pack_bf16x2(a[2].x, a[2].y);
+          pk.w = pack_bf16x2(a[3].x, a[3].y);
+          *reinterpret_cast<uint4 *>(rowp + ((j ^ (lane & 7)) << 4)) = pk;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int x = tl.nb * BN + half * 128 + c * 64;
+          const int y = tl.row0 + quarter * 32;
+          if (x < args.N && y < args.M) {
+            tma_store_2d(tmY, ebuf, x, y);
+            bulk_commit_group();
+          }
+        }
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        const int x = nb * BN + half * 128 + c * 64;
-        const int y = mb * BM + quarter * 32;
-        if (x < args.N && y < args.M) {
-          tma_store_2d(tmY, ebuf, x, y);
-          bulk_commit_group();
+    } else {
+      // bf16 out, rows masked to the expert: four 32-column chunks; each lane
+      // writes its row into the staging buffer, then the warp copies 8 rows x
+      // 64 bytes per instruction to global memory.
+      const int rbase = tl.row0 + quarter * 32;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        __syncwarp();
+        uint8_t *rowp = ebuf + lane * 64;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 *a = &acc[c * 16 + j * 4];
+          uint4 pk;
+          pk.x = pack_bf16x2(a[0].x, a[0].y);
+          pk.y = pack_bf16x2(a[1].x, a[1].y);
+          pk.z = pack_bf16x2(a[2].x, a[2].y);
+          pk.w = pack_bf16x2(a[3].x, a[3].y);
+          *reinterpret_cast<uint4 *>(rowp + ((j ^ ((lane >> 1) & 3)) << 4)) = pk;
+        }
+        __syncwarp();
+        const int n0 = tl.nb * BN + half * 128 + c * 32;
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          const int r = it * 8 + (lane >> 2);
+          const int p = lane & 3;
+          const uint4 v = *reinterpret_cast<const uint4 *>(ebuf + r * 64 + ((p ^ ((r >> 1) & 3)) << 4));
+          const int gr = rbase + r;
+          const int gc = n0 + p * 8;
+          if (gr < tl.row_end && gc < args.N)
+            *reinterpret_cast<uint4 *>(args.y + (int64_t)gr * args.ldy + gc) = v;
         }
       }
     }
   }
-  if (lane == 0) bulk_wait_group0();
+  if constexpr (!G) {
+    if (lane == 0) bulk_wait_group0();
+  }
   __syncwarp();
 }
 
+template <bool G>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_promote_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmY, const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
-  const Smem S = carve(smem_raw);
+  const Smem S = carve<G>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -304,7 +475,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
-    prefetch_tensormap(&tmY);
+    if constexpr (!G) prefetch_tensormap(&tmY);
+  }
+  if constexpr (G) {
+    if (warp == 2) build_schedule(S, args, lane);
   }
   if (warp == 1) {
     tmem_alloc(S.tmem_slot, kTmemCols);
@@ -319,11 +493,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the role is compiled under that role's register budget.
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
-    if (warp == 0 && lane == 0) run_producer(S, &tmA, &tmB, args);
-    else if (warp == 1 && lane == 0) run_mma(S, tmem_base, args);
+    if (warp == 0 && lane == 0) run_producer<G>(S, &tmA, &tmB, args);
+    else if (warp == 1 && lane == 0) run_mma<G>(S, tmem_base, args);
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
-    run_epilogue(S, tmem_base, &tmY, args, warp, lane);
+    run_epilogue<G>(S, tmem_base, &tmY, args, warp, lane);
   }
 
   tc_fence_before();
@@ -337,25 +511,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Per-device one-time setup: opt in to the large shared-memory carve-up and
 // confirm that the kernel was built with the register count the setmaxnreg
 // split assumes (a smaller count would make setmaxnreg.inc wait forever).
-int g_ready[64] = {0};  // 0 unknown, 1 ready, -1 refused
+int g_ready[2][64] = {{0}};  // 0 unknown, 1 ready, -1 refused
 
+template <bool G>
 fp8bq_status prepare_kernel() {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= 64) dev = 0;
-  if (g_ready[dev] == 1) return FP8BQ_OK;
-  if (g_ready[dev] == -1) return FP8BQ_ERR_UNSUPPORTED;
+  int &ready = g_ready[G ? 1 : 0][dev];
+  if (ready == 1) return FP8BQ_OK;
+  if (ready == -1) return FP8BQ_ERR_UNSUPPORTED;
   cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, gemm_promote_kernel);
+  e = cudaFuncGetAttributes(&fa, gemm_promote_kernel<G>);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(gemm)");
   if (fa.numRegs != kLaunchRegs) {
-    g_ready[dev] = -1;
+    ready = -1;
     return FP8BQ_ERR_UNSUPPORTED;
   }
-  e = cudaFuncSetAttribute(gemm_promote_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  e = cudaFuncSetAttribute(gemm_promote_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<G>::kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
-  g_ready[dev] = 1;
+  ready = 1;
   return FP8BQ_OK;
 }
 
@@ -367,12 +543,13 @@ fp8bq_status launch_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_
                          int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K, int mode,
                          int variant, cudaStream_t stream) {
   (void)mode;
-  (void)variant;
   if (M == 0 || N == 0) return FP8BQ_OK;
   if (K == 0) {
     cudaError_t e = cudaMemset2DAsync(y, (size_t)ldy * 2, 0, (size_t)N * 2, (size_t)M, stream);
     return e == cudaSuccess ? FP8BQ_OK : cuda_fail(e, "memset(y)");
   }
+  if (variant == FP8BQ_GEMM_NATIVE_POW2)
+    return launch_gemm_native(qa, lda, sa, ldsa, qw, ldw, sw, y, ldy, M, N, K, stream);
   CUtensorMap tA, tB, tY;
   if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qa, (uint64_t)K, (uint64_t)M, (uint64_t)lda, BK, BM,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -381,9 +558,9 @@ fp8bq_status launch_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_
       !make_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M, (uint64_t)ldy * 2, 64, 32,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return FP8BQ_ERR_INVALID_ARG;
-  fp8bq_status st = prepare_kernel();
+  fp8bq_status st = prepare_kernel<false>();
   if (st != FP8BQ_OK) return st;
-  GemmArgs a;
+  GemmArgs a = {};
   a.sa = sa;
   a.sw = sw;
   a.ldsa = ldsa;
@@ -395,8 +572,43 @@ fp8bq_status launch_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_
   a.num_n = (int32_t)((N + BN - 1) / BN);
   const int64_t tiles = (int64_t)a.num_m * a.num_n;
   const int grid = (int)std::min<int64_t>(tiles, num_sms());
-  gemm_promote_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tA, tB, tY, a);
+  gemm_promote_kernel<false><<<grid, kThreads, Cfg<false>::kSmemBytes, stream>>>(tA, tB, tY, a);
   return check_launch("gemm");
+}
+
+fp8bq_status launch_grouped_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                                 const float *sw, const int32_t *offsets, int E, int64_t rows, int64_t N, int64_t K,
+                                 void *y, int64_t ldy, cudaStream_t stream) {
+  if (rows == 0 || N == 0) return FP8BQ_OK;
+  if (K == 0) {
+    cudaError_t e = cudaMemset2DAsync(y, (size_t)ldy * 2, 0, (size_t)N * 2, (size_t)rows, stream);
+    return e == cudaSuccess ? FP8BQ_OK : cuda_fail(e, "memset(y)");
+  }
+  CUtensorMap tA, tB, tY;
+  memset(&tY, 0, sizeof(tY));
+  if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qa, (uint64_t)K, (uint64_t)rows, (uint64_t)lda, BK, BM,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_3d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, (uint64_t)K, (uint64_t)N, (uint64_t)E, (uint64_t)K,
+                    (uint64_t)N * (uint64_t)K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return FP8BQ_ERR_INVALID_ARG;
+  fp8bq_status st = prepare_kernel<true>();
+  if (st != FP8BQ_OK) return st;
+  GemmArgs a = {};
+  a.sa = sa;
+  a.sw = sw;
+  a.ldsa = ldsa;
+  a.M = (int32_t)rows;
+  a.N = (int32_t)N;
+  a.KB = (int32_t)(K / BK);
+  a.NB = (int32_t)((N + 127) / 128);
+  a.num_m = 0;
+  a.num_n = (int32_t)((N + BN - 1) / BN);
+  a.offsets = offsets;
+  a.E = E;
+  a.y = static_cast<uint16_t *>(y);
+  a.ldy = ldy;
+  gemm_promote_kernel<true><<<num_sms(), kThreads, Cfg<true>::kSmemBytes, stream>>>(tA, tB, tY, a);
+  return check_launch("grouped_gemm");
 }
 
 }  // namespace fp8bq

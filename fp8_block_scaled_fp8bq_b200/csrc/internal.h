@@ -9,6 +9,10 @@
 
 namespace fp8bq {
 
+// Largest expert count of fp8bq_grouped_gemm (the device scheduler keeps the
+// offsets and the tile prefix of all experts in shared memory).
+constexpr int kMaxExperts = 1024;
+
 // Number of SMs of the current device (cached per device).
 int num_sms();
 
@@ -23,8 +27,15 @@ fp8bq_status check_launch(const char *what);
 bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
                   uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
+// 3-D variant: dims {d0 (innermost), d1, d2}, byte strides of dims 1 and 2, box {box0, box1, 1}.
+bool make_tmap_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                  uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
+                  CUtensorMapSwizzle swizzle);
+
 // Per translation unit: read and clear its device error word.
 cudaError_t take_device_error_gemm(unsigned long long *v);
+cudaError_t take_device_error_decode(unsigned long long *v);
+cudaError_t take_device_error_native(unsigned long long *v);
 
 // Launchers (arguments already validated).
 fp8bq_status launch_encode(const float *x, int64_t n, uint8_t *q, cudaStream_t stream);
@@ -34,5 +45,15 @@ fp8bq_status launch_recalibrate(const fp8bq_weight_desc *descs, int n, int mode,
 fp8bq_status launch_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
                          int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K, int mode,
                          int variant, cudaStream_t stream);
+fp8bq_status launch_gemm_native(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                                int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                                cudaStream_t stream);
+size_t decode_workspace_size(int64_t M, int64_t N, int64_t K);
+fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, int64_t ldw, const float *sw, void *y,
+                                int64_t ldy, int64_t M, int64_t N, int64_t K, int mode, void *ws, size_t ws_bytes,
+                                cudaStream_t stream);
+fp8bq_status launch_grouped_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                                 const float *sw, const int32_t *offsets, int E, int64_t rows, int64_t N, int64_t K,
+                                 void *y, int64_t ldy, cudaStream_t stream);
 
 }  // namespace fp8bq

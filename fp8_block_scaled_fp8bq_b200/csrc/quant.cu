@@ -10,166 +10,20 @@
 // These kernels are HBM-bound (2 bytes read, 1 byte written per element):
 // 16-byte vector loads of bf16, an integer max over |x| bit patterns (for
 // non-negative bf16 the bit order is the value order, so the amax is exact),
-// one IEEE division per element (FP32 scales) or a multiply by the exact
-// reciprocal power of two (POW2 scales), and the hardware E4M3 conversion with
+// a correctly rounded quotient per element (one multiply and two fmas with FP32
+// scales, one multiply by the exact reciprocal with POW2 scales; see
+// tile_scale), and the hardware E4M3 conversion with
 // round-to-nearest-even and saturation (cvt.rn.satfinite.e4m3x2.f32).
-#include <cuda_fp8.h>
-
 #include <algorithm>
 
 #include "device.cuh"
 #include "internal.h"
+#include "quant.cuh"
 
 namespace fp8bq {
 namespace {
 
-// ---------------------------------------------------------------------------
-// Scales
-// ---------------------------------------------------------------------------
-// Smallest e with amax <= 448 * 2^e, clamped to [-127, 127].  With
-// amax = f * 2^E, f in [1, 2): 448 * 2^e = 1.75 * 2^(e+8), so e = E - 8 when
-// f <= 1.75 and e = E - 7 otherwise.  amax > 0.
-__device__ __forceinline__ int pow2_exponent(float amax) {
-  uint32_t b = __float_as_uint(amax);
-  int ef = (int)(b >> 23);
-  uint32_t frac = b & 0x7FFFFFu;
-  int E;
-  if (ef == 0) {                        // denormal: normalize the fraction
-    int p = 31 - __clz((int)frac);      // leading one, 0..22
-    E = p - 149;
-    frac = (frac << (23 - p)) & 0x7FFFFFu;
-  } else {
-    E = ef - 127;
-  }
-  int e = (frac <= 0x600000u) ? E - 8 : E - 7;
-  return max(-127, min(127, e));
-}
-
-// 2^e for e in [-127, 127], exactly (2^-127 is a binary32 denormal).
-__device__ __forceinline__ float exp2_exact(int e) {
-  return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
-}
-
-template <int MODE>
-__device__ __forceinline__ void tile_scale(float amax, float &s, float &inv) {
-  if (!(amax > 0.f)) {
-    s = 1.f;
-    inv = 1.f;
-  } else if (MODE == FP8BQ_SCALE_FP32) {
-    s = __fdiv_rn(amax, 448.f);
-    inv = 0.f;  // unused: the FP32 path divides
-  } else {
-    int e = pow2_exponent(amax);
-    s = exp2_exact(e);
-    inv = exp2_exact(-e);
-  }
-}
-
-// The binary32 quotient x / s, correctly rounded.  For a power-of-two scale the
-// product with the exact reciprocal is the same single rounding.
-template <int MODE>
-__device__ __forceinline__ float quotient(float x, float s, float inv) {
-  if (MODE == FP8BQ_SCALE_FP32) return __fdiv_rn(x, s);
-  return x * inv;
-}
-
-__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
-  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
-}
-
-// 8 bf16 (one 16-byte vector) -> 8 E4M3 codes (8 bytes).
-template <int MODE>
-__device__ __forceinline__ uint2 encode8(uint4 v, float s, float inv) {
-  uint2 r;
-  r.x = e4m3x2(quotient<MODE>(bf16_lo(v.x), s, inv), quotient<MODE>(bf16_hi(v.x), s, inv)) |
-        (e4m3x2(quotient<MODE>(bf16_lo(v.y), s, inv), quotient<MODE>(bf16_hi(v.y), s, inv)) << 16);
-  r.y = e4m3x2(quotient<MODE>(bf16_lo(v.z), s, inv), quotient<MODE>(bf16_hi(v.z), s, inv)) |
-        (e4m3x2(quotient<MODE>(bf16_lo(v.w), s, inv), quotient<MODE>(bf16_hi(v.w), s, inv)) << 16);
-  return r;
-}
-
-// max |x| of 8 bf16 as a bf16 bit pattern (exact for finite values).
-__device__ __forceinline__ uint32_t absmax_bits8(uint4 v) {
-  uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu), __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
-  return max(m & 0xFFFFu, m >> 16);
-}
-
-__device__ __forceinline__ float bits_to_amax(uint32_t b16) { return __uint_as_float(b16 << 16); }
-
-// ---------------------------------------------------------------------------
-// Activation quantization, 1x128 tiles
-// ---------------------------------------------------------------------------
-// Block = 8 warps; a half-warp owns one 1x128 tile (16 lanes x 8 elements);
-// each half-warp handles U rows of one K-block, all loads issued first.
-// Block covers rows [blockIdx.x * 16U, +16U) of K-block blockIdx.y.
-template <int MODE, int U>
-__global__ void __launch_bounds__(256) quant_act_vec_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
-                                                            int64_t ldx, uint8_t *__restrict__ q, int64_t ldq,
-                                                            float *__restrict__ sa, int64_t ldsa) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hl = lane & 15, half = lane >> 4;
-  const int64_t kb = blockIdx.y;
-  const int64_t k = kb * 128 + hl * 8;
-  const bool kin = k < K;  // K % 8 == 0 here: a vector is wholly in or out
-  const int64_t rbase = (int64_t)blockIdx.x * (16 * U) + warp * (2 * U) + half;
-
-  uint4 v[U];
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int64_t r = rbase + 2 * u;
-    v[u] = (kin && r < M) ? ld_nc_v4(x + r * ldx + k) : make_uint4(0, 0, 0, 0);
-  }
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int64_t r = rbase + 2 * u;
-    uint32_t m = absmax_bits8(v[u]);
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 8));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    float s, inv;
-    tile_scale<MODE>(bits_to_amax(m), s, inv);
-    if (r < M) {
-      if (kin) *reinterpret_cast<uint2 *>(q + r * ldq + k) = encode8<MODE>(v[u], s, inv);
-      if (hl == 0) sa[kb * ldsa + r] = s;
-    }
-  }
-}
-
-// Any alignment: one half-warp per tile, element j of lane hl is k0 + hl + 16 j.
-template <int MODE>
-__global__ void __launch_bounds__(256) quant_act_scalar_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
-                                                               int64_t ldx, uint8_t *__restrict__ q, int64_t ldq,
-                                                               float *__restrict__ sa, int64_t ldsa) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hl = lane & 15, half = lane >> 4;
-  const int64_t kb = blockIdx.y;
-  const int64_t r = (int64_t)blockIdx.x * 16 + warp * 2 + half;
-  uint16_t e[8];
-  uint32_t m = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int64_t k = kb * 128 + hl + 16 * j;
-    e[j] = (r < M && k < K) ? x[r * ldx + k] : (uint16_t)0;
-    m = max(m, (uint32_t)(e[j] & 0x7FFFu));
-  }
-  m = max(m, __shfl_xor_sync(0xffffffffu, m, 8));
-  m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
-  m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-  m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-  float s, inv;
-  tile_scale<MODE>(bits_to_amax(m), s, inv);
-  if (r >= M) return;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int64_t k = kb * 128 + hl + 16 * j;
-    if (k < K) {
-      const float f = __uint_as_float((uint32_t)e[j] << 16);
-      q[r * ldq + k] = (uint8_t)(e4m3x2(quotient<MODE>(f, s, inv), 0.f) & 0xFFu);
-    }
-  }
-  if (hl == 0) sa[kb * ldsa + r] = s;
-}
+using namespace qdev;
 
 // ---------------------------------------------------------------------------
 // Weight quantization / recalibration, 128x128 tiles
@@ -216,14 +70,13 @@ __device__ __forceinline__ void quant_tile_vec(const TileTensor &T, int64_t nb, 
   m = red[0];
 #pragma unroll
   for (int w = 1; w < 8; ++w) m = max(m, red[w]);
-  float s, inv;
-  tile_scale<MODE>(bits_to_amax(m), s, inv);
+  const TileScale ts = tile_scale<MODE>(bits_to_amax(m));
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int64_t n = nb * 128 + r0 + 16 * i;
-    if (kin && n < T.N) *reinterpret_cast<uint2 *>(T.q + n * T.ldq + k) = encode8<MODE>(v[i], s, inv);
+    if (kin && n < T.N) *reinterpret_cast<uint2 *>(T.q + n * T.ldq + k) = encode8<MODE>(v[i], ts);
   }
-  if (t == 0) T.s[nb * T.KB + kb] = s;
+  if (t == 0) T.s[nb * T.KB + kb] = ts.s;
   __syncthreads();  // red[] is reused by the next tile
 }
 
@@ -242,21 +95,20 @@ __device__ __forceinline__ void quant_tile_scalar(const TileTensor &T, int64_t n
   m = red[0];
 #pragma unroll
   for (int w = 1; w < 8; ++w) m = max(m, red[w]);
-  float s, inv;
-  tile_scale<MODE>(bits_to_amax(m), s, inv);
+  const TileScale ts = tile_scale<MODE>(bits_to_amax(m));
   for (int idx = t; idx < 128 * 128; idx += 256) {
     const int64_t n = nb * 128 + (idx >> 7), k = kb * 128 + (idx & 127);
     if (n < T.N && k < T.K) {
       const float f = __uint_as_float((uint32_t)T.w[n * T.ldw + k] << 16);
-      T.q[n * T.ldq + k] = (uint8_t)(e4m3x2(quotient<MODE>(f, s, inv), 0.f) & 0xFFu);
+      T.q[n * T.ldq + k] = (uint8_t)(e4m3x2(quotient<MODE>(f, ts), 0.f) & 0xFFu);
     }
   }
-  if (t == 0) T.s[nb * T.KB + kb] = s;
+  if (t == 0) T.s[nb * T.KB + kb] = ts.s;
   __syncthreads();
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(256) recalibrate_kernel(const __grid_constant__ RecalParams p) {
+__global__ void __launch_bounds__(256, 4) recalibrate_kernel(const __grid_constant__ RecalParams p) {
   __shared__ uint32_t red[8];
   for (int64_t tile = blockIdx.x; tile < p.total; tile += gridDim.x) {
     int lo = 0, hi = p.n - 1;  // last tensor whose first tile is <= tile

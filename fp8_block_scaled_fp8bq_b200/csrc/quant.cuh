@@ -1,0 +1,209 @@
+// E4M3 quantization device code shared by the quantizer kernels and the
+// decode prologue: tile scales, the correctly rounded element quotient, the
+// E4M3 conversion, and the 1x128 activation tile kernel.
+//
+// Method: "NVIDIA NeMo RL Achieves 48% Speedup With End-to-End FP8 Precision
+// Training", section "Technical breakthrough" (block-wise E4M3; activations
+// 1x128, weights 128x128); power-of-2 scales from section "Why this matters
+// for AI economics".
+#pragma once
+
+#include <cuda_fp8.h>
+
+#include "device.cuh"
+#include "../../include/fp8bq.h"
+
+namespace fp8bq {
+namespace qdev {
+
+// ---------------------------------------------------------------------------
+// Scales
+// ---------------------------------------------------------------------------
+// Smallest e with amax <= 448 * 2^e, clamped to [-127, 127].  With
+// amax = f * 2^E, f in [1, 2): 448 * 2^e = 1.75 * 2^(e+8), so e = E - 8 when
+// f <= 1.75 and e = E - 7 otherwise.  amax > 0.
+__device__ __forceinline__ int pow2_exponent(float amax) {
+  uint32_t b = __float_as_uint(amax);
+  int ef = (int)(b >> 23);
+  uint32_t frac = b & 0x7FFFFFu;
+  int E;
+  if (ef == 0) {                        // denormal: normalize the fraction
+    int p = 31 - __clz((int)frac);      // leading one, 0..22
+    E = p - 149;
+    frac = (frac << (23 - p)) & 0x7FFFFFu;
+  } else {
+    E = ef - 127;
+  }
+  int e = (frac <= 0x600000u) ? E - 8 : E - 7;
+  return max(-127, min(127, e));
+}
+
+// 2^e for e in [-127, 127], exactly (2^-127 is a binary32 denormal).
+__device__ __forceinline__ float exp2_exact(int e) {
+  return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// Per-tile constants of the element quotient x / s.
+//   FP32 scales: s = amax / 448; r = RN(1/s).  When s >= 2^-60 the quotient is
+//     computed with Markstein's correction (P. Markstein, "Computation of
+//     elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+//     Dev. 34(1), 1990): q0 = RN(x r), the residual x - q0 s is formed exactly
+//     by one fma, and q1 = RN(q0 + residual * r) is the correctly rounded
+//     quotient.  Below 2^-60 (tiles whose amax is under ~4e-16) the residual
+//     could underflow, so those tiles use the IEEE division.  A GPU test
+//     compares the codes this produces with the oracle's (an IEEE division)
+//     for every pair (tile amax, element) of bf16 values.
+//   POW2 scales: s = 2^e and r = 2^-e exactly; x * r is the single rounding of
+//     the exact quotient, i.e. the same as the division.
+struct TileScale {
+  float s;     // the scale
+  float r;     // reciprocal (exact for POW2, RN(1/s) for FP32)
+  bool exact;  // FP32 only: use the IEEE division for this tile
+};
+
+template <int MODE>
+__device__ __forceinline__ TileScale tile_scale(float amax) {
+  TileScale t;
+  if (!(amax > 0.f)) {
+    t.s = 1.f;
+    t.r = 1.f;
+    t.exact = false;
+  } else if (MODE == FP8BQ_SCALE_FP32) {
+    t.s = __fdiv_rn(amax, 448.f);
+    t.r = __frcp_rn(t.s);
+    t.exact = !(t.s >= 8.673617379884035e-19f);  // 2^-60
+  } else {
+    const int e = pow2_exponent(amax);
+    t.s = exp2_exact(e);
+    t.r = exp2_exact(-e);
+    t.exact = false;
+  }
+  return t;
+}
+
+// The binary32 quotient x / s, correctly rounded.
+template <int MODE>
+__device__ __forceinline__ float quotient(float x, const TileScale &t) {
+  if (MODE == FP8BQ_SCALE_POW2) return __fmul_rn(x, t.r);
+  if (t.exact) return __fdiv_rn(x, t.s);
+  const float q0 = __fmul_rn(x, t.r);
+  const float res = __fmaf_rn(-q0, t.s, x);
+  const float q1 = __fmaf_rn(res, t.r, q0);
+  // x / s has the sign of x (s > 0); the correction step turns -0 into +0, so
+  // the sign is taken from x.
+  return __uint_as_float((__float_as_uint(q1) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
+}
+
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+}
+
+// 8 bf16 (one 16-byte vector) -> 8 E4M3 codes (8 bytes).
+template <int MODE>
+__device__ __forceinline__ uint2 encode8(uint4 v, const TileScale &t) {
+  uint2 r;
+  r.x = e4m3x2(quotient<MODE>(bf16_lo(v.x), t), quotient<MODE>(bf16_hi(v.x), t)) |
+        (e4m3x2(quotient<MODE>(bf16_lo(v.y), t), quotient<MODE>(bf16_hi(v.y), t)) << 16);
+  r.y = e4m3x2(quotient<MODE>(bf16_lo(v.z), t), quotient<MODE>(bf16_hi(v.z), t)) |
+        (e4m3x2(quotient<MODE>(bf16_lo(v.w), t), quotient<MODE>(bf16_hi(v.w), t)) << 16);
+  return r;
+}
+
+// max |x| of 8 bf16 as a bf16 bit pattern (exact for finite values).
+__device__ __forceinline__ uint32_t absmax_bits8(uint4 v) {
+  uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu), __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+__device__ __forceinline__ float bits_to_amax(uint32_t b16) { return __uint_as_float(b16 << 16); }
+
+// ---------------------------------------------------------------------------
+// Activation quantization, 1x128 tiles
+// ---------------------------------------------------------------------------
+// Block = 8 warps; a half-warp owns one 1x128 tile (16 lanes x 8 elements);
+// each half-warp handles U rows of one K-block, all loads issued first.
+// Block (bx, by) covers rows [bx * 16U, +16U) of K-block by.
+template <int MODE, int U>
+__device__ __forceinline__ void quant_act_vec_block(int64_t bx, int64_t by, const uint16_t *__restrict__ x,
+                                                    int64_t M, int64_t K, int64_t ldx, uint8_t *__restrict__ q,
+                                                    int64_t ldq, float *__restrict__ sa, int64_t ldsa) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hl = lane & 15, half = lane >> 4;
+  const int64_t kb = by;
+  const int64_t k = kb * 128 + hl * 8;
+  const bool kin = k < K;  // K % 8 == 0 here: a vector is wholly in or out
+  const int64_t rbase = bx * (16 * U) + warp * (2 * U) + half;
+
+  uint4 v[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int64_t r = rbase + 2 * u;
+    v[u] = (kin && r < M) ? ld_nc_v4(x + r * ldx + k) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int64_t r = rbase + 2 * u;
+    uint32_t m = absmax_bits8(v[u]);
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 8));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    const TileScale ts = tile_scale<MODE>(bits_to_amax(m));
+    if (r < M) {
+      if (kin) *reinterpret_cast<uint2 *>(q + r * ldq + k) = encode8<MODE>(v[u], ts);
+      if (hl == 0) sa[kb * ldsa + r] = ts.s;
+    }
+  }
+}
+
+// Any alignment: one half-warp per tile, element j of lane hl is k0 + hl + 16 j.
+// Block (bx, by) covers rows [bx * 16, +16) of K-block by.
+template <int MODE>
+__device__ __forceinline__ void quant_act_scalar_block(int64_t bx, int64_t by, const uint16_t *__restrict__ x,
+                                                       int64_t M, int64_t K, int64_t ldx, uint8_t *__restrict__ q,
+                                                       int64_t ldq, float *__restrict__ sa, int64_t ldsa) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hl = lane & 15, half = lane >> 4;
+  const int64_t kb = by;
+  const int64_t r = bx * 16 + warp * 2 + half;
+  uint16_t e[8];
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int64_t k = kb * 128 + hl + 16 * j;
+    e[j] = (r < M && k < K) ? x[r * ldx + k] : (uint16_t)0;
+    m = max(m, (uint32_t)(e[j] & 0x7FFFu));
+  }
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 8));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  const TileScale ts = tile_scale<MODE>(bits_to_amax(m));
+  if (r >= M) return;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int64_t k = kb * 128 + hl + 16 * j;
+    if (k < K) {
+      const float f = __uint_as_float((uint32_t)e[j] << 16);
+      q[r * ldq + k] = (uint8_t)(e4m3x2(quotient<MODE>(f, ts), 0.f) & 0xFFu);
+    }
+  }
+  if (hl == 0) sa[kb * ldsa + r] = ts.s;
+}
+
+template <int MODE, int U>
+__global__ void __launch_bounds__(256) quant_act_vec_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
+                                                            int64_t ldx, uint8_t *__restrict__ q, int64_t ldq,
+                                                            float *__restrict__ sa, int64_t ldsa) {
+  quant_act_vec_block<MODE, U>(blockIdx.x, blockIdx.y, x, M, K, ldx, q, ldq, sa, ldsa);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(256) quant_act_scalar_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
+                                                               int64_t ldx, uint8_t *__restrict__ q, int64_t ldq,
+                                                               float *__restrict__ sa, int64_t ldsa) {
+  quant_act_scalar_block<MODE>(blockIdx.x, blockIdx.y, x, M, K, ldx, q, ldq, sa, ldsa);
+}
+
+}  // namespace qdev
+}  // namespace fp8bq

@@ -97,3 +97,16 @@ def test_recalibrate_validation(L):
     assert L.fp8bq_recalibrate(arr, 2, 1, None) == INVALID
     assert L.fp8bq_recalibrate(arr, -1, 1, None) == INVALID
     assert L.fp8bq_recalibrate(arr, 0, 1, None) == 0
+
+
+def test_grouped_validation(L):
+    f = L.fp8bq_grouped_gemm
+
+    def call(E=4, rows=256, N=256, K=256, lda=256, ldsa=256, ldy=256, off=FAKE):
+        return f(FAKE, lda, FAKE, ldsa, FAKE, FAKE, off, E, rows, N, K, FAKE, ldy, 0, None)
+    assert call(E=0) == INVALID
+    assert call(E=1025) == UNSUPPORTED
+    assert call(off=None) == INVALID
+    assert call(N=260, ldy=264) == UNSUPPORTED                            # N % 8
+    assert call(K=200, lda=208) == UNSUPPORTED                            # K % 128
+    assert call(rows=0) == 0

@@ -52,29 +52,42 @@ def test_e4m3_encoder_all_fp32_patterns():
         assert ok.all(), "first mismatch at pattern 0x%08x" % int(pats[np.argmin(ok)])
 
 
-@pytest.mark.parametrize("mode", MODES)
-def test_division_sweep_over_tile_amax(mode):
-    """Rows whose amax is a chosen bf16 value and whose other elements run over
-    every bf16 pattern below it: the quotient x/s for many (amax, x) pairs."""
-    rng = np.random.default_rng(7)
-    amax_bits = np.unique(np.concatenate([
-        np.arange(1, 0x7F80, 97, dtype=np.uint16), np.array([1, 2, 0x7F, 0x80, 0x3F80, 0x43E0, 0x7F7F], np.uint16),
-        rng.integers(0x0080, 0x7F80, 200).astype(np.uint16)]))
-    allx = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
-    allx = allx[(allx & 0x7FFF) < 0x7F80]                 # finite patterns only
-    K = 128
-    rows = []
-    for a in amax_bits:
-        ok = allx[(allx & 0x7FFF) <= a]
-        for i in range(0, ok.size, K - 1):
-            chunk = ok[i:i + K - 1]
-            row = np.zeros(K, dtype=np.uint16)
-            row[0] = a
-            row[1:1 + chunk.size] = chunk
-            rows.append(row)
-    xb = np.stack(rows)
-    x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
-    check_act(x, mode)
+def _rows_for_amax(amaxes):
+    """1x128 tiles whose element 0 is the amax a and whose other 127 elements run,
+    across consecutive rows, over every bf16 pattern x with |x| <= a (both signs)."""
+    a = np.asarray(amaxes, dtype=np.int64)
+    R = -(-2 * (a + 1) // 127)                              # rows needed per amax
+    row_a = np.repeat(a, R)
+    row_i = np.arange(int(R.sum()), dtype=np.int64) - np.repeat(np.cumsum(R) - R, R)
+    t = row_i[:, None] * 127 + np.arange(127, dtype=np.int64)[None, :]
+    A = row_a[:, None]
+    x = np.where(t <= A, t, np.where(t < 2 * (A + 1), (t - (A + 1)) | 0x8000, 0))
+    return np.concatenate([row_a[:, None], x], axis=1).astype(np.uint16)
+
+
+@pytest.mark.slow
+def test_quotient_every_amax_element_pair():
+    """Exhaustive over the quantizer's arithmetic domain: for every finite positive
+    bf16 tile amax a and every finite bf16 element x with |x| <= a, the code of
+    x / s(a) equals the oracle's.  (The scale depends only on a, so this covers
+    every quotient the quantizers can ever form.)"""
+    all_a = np.arange(1, 0x7F80, dtype=np.uint32)
+    # chunks of about 2^25 elements
+    cuts = [0]
+    acc = 0
+    for i, a in enumerate(all_a):
+        acc += 2 * (int(a) + 1)
+        if acc >= (1 << 25):
+            cuts.append(i + 1)
+            acc = 0
+    cuts.append(all_a.size)
+    for c0, c1 in zip(cuts[:-1], cuts[1:]):
+        if c1 <= c0:
+            continue
+        xb = _rows_for_amax(all_a[c0:c1])
+        x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
+        for mode in MODES:
+            check_act(x, mode)
 
 
 @pytest.mark.parametrize("mode", MODES)
