@@ -59,6 +59,7 @@ SIGNATURES = {
     "fp8bq_gemm_ex": (I32, [P, I64, P, I64, P, I64, P, P, I64, I64, I64, I64, I32, I32, P]),
     "fp8bq_gemm_decode_workspace_size": (SZ, [I64, I64, I64]),
     "fp8bq_gemm_decode": (I32, [P, I64, P, I64, P, P, I64, I64, I64, I64, I32, P, SZ, P]),
+    "fp8bq_gemm_decode_noalloc": (I32, [P, I64, P, I64, P, P, I64, I64, I64, I64, I32, P]),
     "fp8bq_grouped_gemm": (I32, [P, I64, P, I64, P, P, P, I32, I64, I64, I64, P, I64, I32, P]),
 }
 

@@ -209,6 +209,28 @@ FP8BQ_API fp8bq_status fp8bq_gemm_decode(const void *x, int64_t ldx,
                                int mode, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * fp8bq_gemm_decode without a workspace, for callers that cannot allocate
+ * device memory when they call (a C or Fortran host program linking this
+ * library without a framework's memory pool, or a serving loop that must not
+ * allocate once running).  The pages have no counterpart: this is a calling
+ * convenience, not part of the method.
+ *   Arguments, result and requirements are those of fp8bq_gemm_decode.  The
+ *   scratch is a fixed 32 MiB array in device memory that the library holds on
+ *   every GPU that loads it until the process exits; a shape whose workspace
+ *   (fp8bq_gemm_decode_workspace_size) exceeds 32 MiB returns
+ *   FP8BQ_ERR_WORKSPACE and launches nothing.  Nothing is allocated.
+ *   The first call on a device looks up the array's device address (a CUDA
+ *   runtime call); make that first call outside any stream capture.
+ *   All calls share the one array: calls that may run at the same time on the
+ *   GPU (different streams, or different host threads) race on it and must be
+ *   ordered by the caller.  Each call rewrites the parts it reads.
+ */
+FP8BQ_API fp8bq_status fp8bq_gemm_decode_noalloc(const void *x, int64_t ldx,
+                                                 const uint8_t *qw, int64_t ldw, const float *sw,
+                                                 void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                                                 int mode, void *stream);
+
+/*
  * Grouped (mixture-of-experts) GEMM ("Real-world performance gains": the
  * recipe on a mixture-of-experts model): rows [offsets[e], offsets[e+1]) of the
  * expert-sorted activations are multiplied by expert e's weight.
