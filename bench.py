@@ -409,7 +409,7 @@ def reference(args):
     print(json.dumps(line), flush=True)
 
 
-CASES = (["gemm:" + n for n in NAMES] + ["decode:" + n for n in NAMES] +
+CASES = (["gemm:" + n for n in NAMES] + ["decode:" + n for n in NAMES] + ["cublas:" + n for n in NAMES] +
          ["quant_act:4096", "quant_act:14336", "recalibrate:layer", "quant_weight:gate_up", "moe:up", "moe:down"])
 
 
@@ -442,6 +442,20 @@ def run_case(args):
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         variant = fq.GEMM_NATIVE_POW2 if args.native else fq.GEMM_PROMOTE
         fn = lambda: fq.gemm(qa, sa, qw, sw, mode, out=y, variant=variant)  # noqa: E731
+        work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
+    elif kind == "cublas":
+        # context only: cuBLASLt FP8 GEMM through torch._scaled_mm on the same shape
+        # (per-tensor scales; blockwise scales if this torch build accepts them)
+        N, K = wl.LLAMA8B_SHAPES[what]
+        a = wl.activations(M, K, seed=1, device=dev).to(torch.float8_e4m3fn)
+        b = wl.weights(N, K, seed=2, device=dev).mul(20).to(torch.float8_e4m3fn)
+        if args.pow2:   # blockwise: 1x128 for a, 128x128 for b
+            sa_ = torch.ones((M, K // 128), dtype=torch.float32, device=dev)
+            sb_ = torch.ones((K // 128, (N + 127) // 128), dtype=torch.float32, device=dev).t()
+        else:
+            sa_ = torch.ones((), dtype=torch.float32, device=dev)
+            sb_ = torch.ones((), dtype=torch.float32, device=dev)
+        fn = lambda: torch._scaled_mm(a, b.t(), scale_a=sa_, scale_b=sb_, out_dtype=torch.bfloat16)  # noqa: E731
         work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
     elif kind == "decode":
         N, K = wl.LLAMA8B_SHAPES[what]

@@ -8,25 +8,27 @@
 // 128x128).  In generation the linear layers see a handful of tokens, so the
 // time goes into streaming the weight from HBM.
 //
-// Design.  Two launches:
+// Design (M <= 64), three launches:
 //   1. prologue: 1x128 quantization of X into the workspace (the same device
-//      code as fp8bq_quant_act) and zeroing of the split-K counters;
+//      code as fp8bq_quant_act);
 //   2. the GEMM, with the operands swapped so that the tensor cores do useful
 //      work at small M: the weight is the 128-row MMA operand and the tokens
-//      are the MMA's N dimension (NT = M rounded up to 16, 32 or 64; rows
-//      past M are TMA zero-fill).  For M > 64 the per-token promotion would
-//      cost more than the weight stream, so step 2 is the prefill GEMM on the
-//      quantized activation instead.  A unit of work is one 128-row
-//      weight block times one contiguous range of K-blocks (split-K chosen on
-//      the host so the units fill the SMs).  Per K-block: TMA loads of the
-//      weight tile (16 KB), the activation-code tile and that K-block's row
-//      scales into a deep stage ring; 4 x tcgen05.mma 128xNTx32 into one of
-//      two TMEM buffers; the epilogue warps (weight row = TMEM lane, token =
-//      column) add P * (sa[kb][token] * sw[nb][kb]) into FP32 registers.
-//   A unit writes bf16 directly when the K range is not split; otherwise it
-//   writes an FP32 partial to the workspace and bumps a per-weight-block
-//   counter, and the unit that arrives last sums the partials in split order
-//   (deterministic) and writes bf16.
+//      are the MMA's N dimension (NT = M rounded up to 16, 32 or 64; rows past
+//      M are TMA zero-fill).  The NB x KB grid of (128-row weight block,
+//      128-deep K-block) work items is cut, in weight-block-major order, into
+//      one contiguous equal share per CTA, so every SM streams the same number
+//      of weight bytes whatever NB is.  Per work item: TMA loads of the weight
+//      tile (16 KB), the activation-code tile and that K-block's row scales
+//      into a deep stage ring; 4 x tcgen05.mma 128xNTx32 into one of two TMEM
+//      buffers; the epilogue warps (weight row = TMEM lane, token = column)
+//      add P * (sa[kb][token] * sw[nb][kb]) into FP32 registers.  A weight
+//      block whose whole K range lies inside one share is written as bf16 at
+//      once; a share's first and last weight blocks, when cut, go to FP32
+//      partial slots in the workspace;
+//   3. reduce: for each cut weight block, the partial slots of the CTAs that
+//      share it are added in CTA order (deterministic) and written as bf16.
+// For M > 64 the per-token promotion costs more than the weight stream, so
+// step 2 is the prefill GEMM on the quantized activation instead.
 #include <cuda_bf16.h>
 #include <string.h>
 
@@ -46,11 +48,7 @@ constexpr int kDLowRegs = 56;
 constexpr int kDHighRegs = 224;
 static_assert(128 * kDLowRegs + 256 * kDHighRegs <= kDThreads * kDLaunchRegs, "register split");
 constexpr int kMaxDecodeM = 256;
-// Above this many tokens the swapped kernel's per-column promotion costs more
-// than the weight stream: quantize into the workspace and run the prefill GEMM
-// (128-row tiles, per-row scales) instead.
 constexpr int kSwapMaxM = 64;
-constexpr int kMaxSplit = 16;
 constexpr int kDEpiWarps = 8;
 constexpr int kStageBudget = 212992;
 
@@ -65,7 +63,6 @@ struct DCfg {
   static constexpr int kStages = kFit < 8 ? kFit : 8;
   static constexpr int kCW = NT / 2;         // token columns per epilogue warpgroup
   static constexpr int kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
-  static constexpr int kCH = kCW < 32 ? kCW : 32;  // columns per TMEM load round
   static constexpr int kSmemBytes = kStages * (kABytes + kBBytes + kSSlot) + 256 + 1024;
   static_assert(kStages >= 3 && kSmemBytes <= 232448, "decode shared memory budget");
 };
@@ -73,31 +70,27 @@ struct DCfg {
 struct DecodeArgs {
   const float *sw;
   int32_t M, N, KB, NB;
-  int32_t S;      // K-splits per weight block
-  int32_t units;  // NB * S
-  float *part;    // [S][M][N] partials (S > 1)
-  int32_t *cnt;   // [NB] arrival counters, zeroed by the prologue
+  int64_t W;      // NB * KB work items
+  int32_t G;      // CTAs (shares)
+  float *part;    // [G][2][M][128] partial slots
   uint16_t *y;    // bf16 bits
   int64_t ldy;
 };
 
+// First work item of CTA c's share.
+__host__ __device__ __forceinline__ int64_t share_begin(int64_t c, int64_t W, int64_t G) { return c * W / G; }
+
+// The CTA whose share holds work item p.
+__host__ __device__ __forceinline__ int64_t share_of(int64_t p, int64_t W, int64_t G) {
+  int64_t c = p * G / W;
+  while (c + 1 < G && share_begin(c + 1, W, G) <= p) ++c;
+  while (c > 0 && share_begin(c, W, G) > p) --c;
+  return c;
+}
+
 __device__ __forceinline__ uint16_t bf16_bits(float v) {
   __nv_bfloat16 b = __float2bfloat16_rn(v);
   return *reinterpret_cast<uint16_t *>(&b);
-}
-
-// Named barrier among the 256 epilogue threads that also ORs a predicate.
-__device__ __forceinline__ bool epi_barrier_or(bool p) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred q, o;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.or.pred o, 1, 256, q;\n\t"
-      "selp.u32 %0, 1, 0, o;\n\t}\n"
-      : "=r"(r)
-      : "r"((uint32_t)p)
-      : "memory");
-  return r != 0;
 }
 
 // CH consecutive TMEM columns of this warp's 32 lanes into r[0..CH).
@@ -105,11 +98,8 @@ template <int CH>
 __device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t *r) {
   if constexpr (CH == 8) {
     tmem_ld_32x32b_x8(taddr, r);
-  } else if constexpr (CH == 16) {
-    tmem_ld_32x32b_x16(taddr, r);
   } else {
-#pragma unroll
-    for (int c = 0; c < CH / 32; ++c) tmem_ld_32x32b_x32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * c));
+    tmem_ld_32x32b_x16(taddr, r);
   }
 }
 
@@ -131,10 +121,11 @@ __global__ void __launch_bounds__(kDThreads, 1)
   uint64_t *drain = tempty + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  volatile int *last_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int S = args.S, KB = args.KB;
+  const int KB = args.KB;
+  const int64_t p_begin = share_begin(blockIdx.x, args.W, args.G);
+  const int64_t p_end = share_begin(blockIdx.x + 1, args.W, args.G);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -147,7 +138,6 @@ __global__ void __launch_bounds__(kDThreads, 1)
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
-    *last_flag = 0;
     fence_mbarrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -171,24 +161,21 @@ __global__ void __launch_bounds__(kDThreads, 1)
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
-        const int nb = u / S, kc = u - nb * S;
-        const int kb0 = (int)((int64_t)kc * KB / S), kb1 = (int)((int64_t)(kc + 1) * KB / S);
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, kSiteProducerEmpty)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[stage], C::kTx);
-          tma_load_2d(sA + stage * C::kABytes, &tmW, &full[stage], kb * DBK, nb * DBM);
-          tma_load_2d(sB + stage * C::kBBytes, &tmX, &full[stage], kb * DBK, 0);
-          tma_load_2d(sS + stage * C::kSSlot, &tmS, &full[stage], 0, kb);
-          armed |= 1u << stage;
-          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
+      for (int64_t p = p_begin; p < p_end; ++p) {
+        const int nb = (int)(p / KB), kb = (int)(p - (int64_t)nb * KB);
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, kSiteProducerEmpty)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[stage], C::kTx);
+        tma_load_2d(sA + stage * C::kABytes, &tmW, &full[stage], kb * DBK, nb * DBM);
+        tma_load_2d(sB + stage * C::kBBytes, &tmX, &full[stage], kb * DBK, 0);
+        tma_load_2d(sS + stage * C::kSSlot, &tmS, &full[stage], 0, kb);
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1;
         }
       }
       if (!ok) {
@@ -201,33 +188,29 @@ __global__ void __launch_bounds__(kDThreads, 1)
       int stage = 0, buf = 0;
       uint32_t phase = 0, bphase = 0;
       bool ok = true, issued = false;
-      for (int u = blockIdx.x; u < args.units && ok; u += gridDim.x) {
-        const int nb = u / S, kc = u - nb * S;
-        const int kb0 = (int)((int64_t)kc * KB / S), kb1 = (int)((int64_t)(kc + 1) * KB / S);
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&tempty[buf], bphase ^ 1, abort_flag, kSiteMmaTmemEmpty) ||
-              !mbar_wait(&full[stage], phase, abort_flag, kSiteMmaFull)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d = tmem_base + (uint32_t)(buf * NT);
-          const uint32_t a0 = smem_addr(sA + stage * C::kABytes);
-          const uint32_t b0 = smem_addr(sB + stage * C::kBBytes);
+      for (int64_t p = p_begin; p < p_end; ++p) {
+        if (!mbar_wait(&tempty[buf], bphase ^ 1, abort_flag, kSiteMmaTmemEmpty) ||
+            !mbar_wait(&full[stage], phase, abort_flag, kSiteMmaFull)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(buf * NT);
+        const uint32_t a0 = smem_addr(sA + stage * C::kABytes);
+        const uint32_t b0 = smem_addr(sB + stage * C::kBBytes);
 #pragma unroll
-          for (int k = 0; k < DBK / 32; ++k)
-            mma_f8f6f4(d, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k), idesc, k > 0 ? 1u : 0u);
-          mma_commit(&empty[stage]);
-          mma_commit(&tfull[buf]);
-          issued = true;
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
-          if (++buf == 2) {
-            buf = 0;
-            bphase ^= 1;
-          }
+        for (int k = 0; k < DBK / 32; ++k)
+          mma_f8f6f4(d, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k), idesc, k > 0 ? 1u : 0u);
+        mma_commit(&empty[stage]);
+        mma_commit(&tfull[buf]);
+        issued = true;
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+        if (++buf == 2) {
+          buf = 0;
+          bphase ^= 1;
         }
       }
       if (!ok && issued) {
@@ -240,110 +223,75 @@ __global__ void __launch_bounds__(kDThreads, 1)
     // ------------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     const int h = (warp - 4) >> 2;
-    const int c0 = h * C::kCW;  // first token column of this warpgroup
+    const int c0 = h * C::kCW;          // first token column of this warpgroup
+    const int r = quarter * 32 + lane;  // weight row within the block = output column
     int stage = 0, buf = 0;
-    uint32_t phase = 0, bphase = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
-      const int nb = u / S, kc = u - nb * S;
-      const int kb0 = (int)((int64_t)kc * KB / S), kb1 = (int)((int64_t)(kc + 1) * KB / S);
-      const int n = nb * DBM + quarter * 32 + lane;  // weight row = output column
-      const float *swp = args.sw + (int64_t)nb * KB;
-      float acc[C::kCW];
+    uint32_t bphase = 0;
+    float acc[C::kCW];
 #pragma unroll
-      for (int j = 0; j < C::kCW; ++j) acc[j] = 0.f;
-      float w0 = __ldg(swp + kb0), w1 = (kb0 + 1 < kb1) ? __ldg(swp + kb0 + 1) : 0.f;
-      for (int kb = kb0; kb < kb1 && ok; ++kb) {
-        const float w = w0;
-        w0 = w1;
-        if (kb + 2 < kb1) w1 = __ldg(swp + kb + 2);
-        const bool got = mbar_wait(&tfull[buf], bphase, abort_flag, kSiteEpiTmemFull);
-        if (!__all_sync(0xffffffffu, got)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * NT + c0);
-        const float4 *sc4 = reinterpret_cast<const float4 *>(sS + stage * C::kSSlot) + c0 / 4;
-#pragma unroll
-        for (int c = 0; c < C::kCW / C::kCH; ++c) {
-          uint32_t r[C::kCH];
-          load_cols<C::kCH>(taddr + c * C::kCH, r);
-          tmem_ld_wait();
-          if (c == C::kCW / C::kCH - 1) {  // the TMEM buffer has been read
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
-          }
-#pragma unroll
-          for (int j = 0; j < C::kCH / 4; ++j) {
-            const float4 s4 = sc4[c * C::kCH / 4 + j];
-            float *a = &acc[c * C::kCH + 4 * j];
-            a[0] = fmaf(__uint_as_float(r[4 * j + 0]), s4.x * w, a[0]);
-            a[1] = fmaf(__uint_as_float(r[4 * j + 1]), s4.y * w, a[1]);
-            a[2] = fmaf(__uint_as_float(r[4 * j + 2]), s4.z * w, a[2]);
-            a[3] = fmaf(__uint_as_float(r[4 * j + 3]), s4.w * w, a[3]);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);  // the stage's scales have been read
-        if (++stage == C::kStages) {
-          stage = 0;
-          phase ^= 1;
-        }
-        if (++buf == 2) {
-          buf = 0;
-          bphase ^= 1;
-        }
+    for (int j = 0; j < C::kCW; ++j) acc[j] = 0.f;
+    // sw is [NB][KB] row-major, so work item p's weight scale is sw[p]; the
+    // next two are loaded ahead
+    float w0 = p_begin < p_end ? __ldg(args.sw + p_begin) : 0.f;
+    float w1 = p_begin + 1 < p_end ? __ldg(args.sw + p_begin + 1) : 0.f;
+    for (int64_t p = p_begin; p < p_end; ++p) {
+      const int nb = (int)(p / KB), kb = (int)(p - (int64_t)nb * KB);
+      const float w = w0;
+      w0 = w1;
+      if (p + 2 < p_end) w1 = __ldg(args.sw + p + 2);
+      const bool got = mbar_wait(&tfull[buf], bphase, abort_flag, kSiteEpiTmemFull);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * NT + c0);
+      const float4 *sc4 = reinterpret_cast<const float4 *>(sS + stage * C::kSSlot) + c0 / 4;
+      uint32_t v[C::kCW];
+      if constexpr (C::kCW <= 16) {
+        load_cols<C::kCW>(taddr, v);
+      } else {
+        load_cols<16>(taddr, v);
+        load_cols<16>(taddr + 16, v + 16);
       }
-      (void)phase;
-      if (S == 1) {
-        if (!ok) break;
-        if (n < args.N) {
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
 #pragma unroll
-          for (int j = 0; j < C::kCW; ++j)
-            if (c0 + j < args.M) args.y[(int64_t)(c0 + j) * args.ldy + n] = bf16_bits(acc[j]);
-        }
-        continue;
+      for (int j = 0; j < C::kCW / 4; ++j) {
+        const float4 s4 = sc4[j];
+        acc[4 * j + 0] = fmaf(__uint_as_float(v[4 * j + 0]), s4.x * w, acc[4 * j + 0]);
+        acc[4 * j + 1] = fmaf(__uint_as_float(v[4 * j + 1]), s4.y * w, acc[4 * j + 1]);
+        acc[4 * j + 2] = fmaf(__uint_as_float(v[4 * j + 2]), s4.z * w, acc[4 * j + 2]);
+        acc[4 * j + 3] = fmaf(__uint_as_float(v[4 * j + 3]), s4.w * w, acc[4 * j + 3]);
       }
-      // split K: partial out, then the last unit of this weight block reduces
-      if (ok && n < args.N) {
-#pragma unroll
-        for (int j = 0; j < C::kCW; ++j)
-          if (c0 + j < args.M) args.part[((int64_t)kc * args.M + (c0 + j)) * args.N + n] = acc[j];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);  // the stage's scales have been read
+      if (++stage == C::kStages) stage = 0;
+      if (++buf == 2) {
+        buf = 0;
+        bphase ^= 1;
       }
-      __threadfence();
-      const bool stop1 = epi_barrier_or(!ok);
-      if (stop1) break;
-      if (warp == 4 && lane == 0) *last_flag = (atomicAdd(args.cnt + nb, 1) == S - 1) ? 1 : 0;
-      epi_barrier_or(false);
-      if (*last_flag) {
-        // Sum the S partials in split order (the same order whichever unit
-        // arrives last); this unit's own partial is still in registers.  The
-        // loads of one split are independent, so all of them are in flight
-        // together.
-        __threadfence();
-        float tot[C::kCW];
-#pragma unroll
-        for (int j = 0; j < C::kCW; ++j) tot[j] = 0.f;
-        for (int s = 0; s < S; ++s) {
-          if (s == kc) {
-#pragma unroll
-            for (int j = 0; j < C::kCW; ++j) tot[j] += acc[j];
-          } else if (n < args.N) {
-            const float *src = args.part + (int64_t)s * args.M * args.N + n;
+      // end of this weight block's run inside the share: flush it
+      if (kb == KB - 1 || p + 1 == p_end) {
+        const int64_t run0 = (p - kb > p_begin) ? p - kb : p_begin;  // first work item of the run
+        const bool whole = (run0 == p - kb) && kb == KB - 1;
+        const int n = nb * DBM + r;
+        if (whole) {
+          if (n < args.N) {
 #pragma unroll
             for (int j = 0; j < C::kCW; ++j)
-              if (c0 + j < args.M) tot[j] += __ldcg(src + (int64_t)(c0 + j) * args.N);
+              if (c0 + j < args.M) args.y[(int64_t)(c0 + j) * args.ldy + n] = bf16_bits(acc[j]);
           }
-        }
-        if (n < args.N) {
+        } else {
+          // slot 0: the run holding the share's first item; slot 1: the last run
+          const int which = (run0 == p_begin) ? 0 : 1;
+          float *dst = args.part + ((int64_t)(blockIdx.x * 2 + which) * args.M) * DBM + r;
 #pragma unroll
           for (int j = 0; j < C::kCW; ++j)
-            if (c0 + j < args.M) args.y[(int64_t)(c0 + j) * args.ldy + n] = bf16_bits(tot[j]);
+            if (c0 + j < args.M) dst[(int64_t)(c0 + j) * DBM] = acc[j];
         }
+#pragma unroll
+        for (int j = 0; j < C::kCW; ++j) acc[j] = 0.f;
       }
-      if (epi_barrier_or(*abort_flag != 0)) break;  // also keeps last_flag stable until all have read it
     }
   }
 
@@ -355,22 +303,38 @@ __global__ void __launch_bounds__(kDThreads, 1)
   }
 }
 
-// Prologue: 1x128 quantization of X into the workspace, counters zeroed.
+// Adds the partial slots of the CTAs that share a weight block, in CTA order.
+// Block (nb, m): weight block nb, token m, one thread per weight row; blocks
+// held wholly by one CTA were written directly and are skipped.
+__global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeArgs a) {
+  const int nb = blockIdx.x, m = blockIdx.y;
+  const int r = threadIdx.x;
+  const int64_t first = (int64_t)nb * a.KB, last = first + a.KB - 1;
+  const int64_t c0 = share_of(first, a.W, a.G), c1 = share_of(last, a.W, a.G);
+  if (c0 == c1) return;
+  const int n = nb * DBM + r;
+  if (n >= a.N) return;
+  float sum = 0.f;
+  for (int64_t c = c0; c <= c1; ++c) {
+    const int which = share_begin(c, a.W, a.G) >= first ? 0 : 1;
+    sum += a.part[((c * 2 + which) * a.M + m) * DBM + r];
+  }
+  a.y[(int64_t)m * a.ldy + n] = bf16_bits(sum);
+}
+
+// Prologue: 1x128 quantization of X into the workspace.
 template <int MODE, bool VEC>
 __global__ void __launch_bounds__(256) decode_prologue_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
                                                               int64_t ldx, uint8_t *__restrict__ q,
-                                                              float *__restrict__ sa, int64_t ldsa,
-                                                              int32_t *__restrict__ cnt, int ncnt) {
-  if (blockIdx.x == 0 && blockIdx.y == 0)
-    for (int i = threadIdx.x; i < ncnt; i += blockDim.x) cnt[i] = 0;
-  if constexpr (VEC) qdev::quant_act_vec_block<MODE, 4>(blockIdx.x, blockIdx.y, x, M, K, ldx, q, K, sa, ldsa);
+                                                              float *__restrict__ sa, int64_t ldsa) {
+  if constexpr (VEC) qdev::quant_act_vec_block<MODE>(blockIdx.x, blockIdx.y, x, M, K, ldx, q, K, sa, ldsa);
   else qdev::quant_act_scalar_block<MODE>(blockIdx.x, blockIdx.y, x, M, K, ldx, q, K, sa, ldsa);
 }
 
 struct Plan {
-  int NT, S, NB, KB;
-  int64_t ldsa;
-  size_t off_q, off_sa, off_part, off_cnt, total;
+  int NT, NB, KB, G;
+  int64_t W, ldsa;
+  size_t off_q, off_sa, off_part, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -381,35 +345,18 @@ int pick_nt(int64_t M) {
   return 64;
 }
 
-// Split-K count: minimise (weight bytes / SM-fill efficiency) + partial traffic.
-int pick_split(int64_t M, int64_t N, int64_t K, int NB, int KB, int sms) {
-  double best = 1e300;
-  int best_s = 1;
-  for (int s = 1; s <= std::min(KB, kMaxSplit); ++s) {
-    const int64_t units = (int64_t)NB * s;
-    const int64_t waves = (units + sms - 1) / sms;
-    const double eff = (double)units / (double)(waves * sms);
-    const double cost = (double)N * K / eff + (s > 1 ? 8.0 * s * M * N : 0.0);
-    if (cost < best * (1.0 - 1e-9)) {
-      best = cost;
-      best_s = s;
-    }
-  }
-  return best_s;
-}
-
 Plan make_plan(int64_t M, int64_t N, int64_t K) {
   Plan p;
   p.NT = M <= kSwapMaxM ? pick_nt(M) : 0;  // 0: the prefill GEMM
   p.NB = (int)((N + 127) / 128);
   p.KB = (int)(K / 128);
-  p.S = p.NT ? pick_split(M, N, K, p.NB, p.KB, num_sms()) : 1;
+  p.W = (int64_t)p.NB * p.KB;
+  p.G = (int)std::min<int64_t>(p.W, num_sms());
   p.ldsa = (M + 3) / 4 * 4;
   p.off_q = 0;
   p.off_sa = align256((size_t)(M * K));
   p.off_part = p.off_sa + align256((size_t)p.KB * p.ldsa * 4);
-  p.off_cnt = p.off_part + (p.S > 1 ? align256((size_t)p.S * M * N * 4) : 0);
-  p.total = p.off_cnt + align256((size_t)p.NB * 4);
+  p.total = p.off_part + (p.NT ? align256((size_t)p.G * 2 * M * DBM * 4) : 0);
   return p;
 }
 
@@ -436,9 +383,11 @@ fp8bq_status launch_decode_nt(const CUtensorMap &tW, const CUtensorMap &tX, cons
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
     ready = 1;
   }
-  const int grid = std::min(a.units, num_sms());
-  decode_kernel<NT><<<grid, kDThreads, DCfg<NT>::kSmemBytes, stream>>>(tW, tX, tS, a);
-  return check_launch("gemm_decode");
+  decode_kernel<NT><<<a.G, kDThreads, DCfg<NT>::kSmemBytes, stream>>>(tW, tX, tS, a);
+  fp8bq_status st = check_launch("gemm_decode");
+  if (st != FP8BQ_OK) return st;
+  decode_reduce_kernel<<<dim3((unsigned)a.NB, (unsigned)a.M), 128, 0, stream>>>(a);
+  return check_launch("gemm_decode reduce");
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -462,28 +411,27 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
   uint8_t *q = wsb + p.off_q;
   float *sa = reinterpret_cast<float *>(wsb + p.off_sa);
   float *part = reinterpret_cast<float *>(wsb + p.off_part);
-  int32_t *cnt = reinterpret_cast<int32_t *>(wsb + p.off_cnt);
 
-  // 1. quantize X (and zero the counters)
+  // 1. quantize X
   const uint16_t *xs = static_cast<const uint16_t *>(x);
   const bool vec = aligned(x, 16) && ldx % 8 == 0;  // K % 128 == 0 already
   if (vec) {
     dim3 grid((unsigned)((M + 63) / 64), (unsigned)p.KB);
     if (mode == FP8BQ_SCALE_FP32)
-      decode_prologue_kernel<FP8BQ_SCALE_FP32, true><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, sa, p.ldsa, cnt, p.NB);
+      decode_prologue_kernel<FP8BQ_SCALE_FP32, true><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, sa, p.ldsa);
     else
-      decode_prologue_kernel<FP8BQ_SCALE_POW2, true><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, sa, p.ldsa, cnt, p.NB);
+      decode_prologue_kernel<FP8BQ_SCALE_POW2, true><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, sa, p.ldsa);
   } else {
     dim3 grid((unsigned)((M + 15) / 16), (unsigned)p.KB);
     if (mode == FP8BQ_SCALE_FP32)
-      decode_prologue_kernel<FP8BQ_SCALE_FP32, false><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, sa, p.ldsa, cnt, p.NB);
+      decode_prologue_kernel<FP8BQ_SCALE_FP32, false><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, sa, p.ldsa);
     else
-      decode_prologue_kernel<FP8BQ_SCALE_POW2, false><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, sa, p.ldsa, cnt, p.NB);
+      decode_prologue_kernel<FP8BQ_SCALE_POW2, false><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, sa, p.ldsa);
   }
   fp8bq_status st = check_launch("gemm_decode prologue");
   if (st != FP8BQ_OK) return st;
 
-  // 2. the GEMM
+  // 2. the GEMM (and 3. the reduction of cut weight blocks)
   if (p.NT == 0)
     return launch_gemm(q, K, sa, p.ldsa, qw, ldw, sw, y, ldy, M, N, K, mode, FP8BQ_GEMM_AUTO, stream);
   CUtensorMap tW, tX, tS;
@@ -500,10 +448,9 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
   a.N = (int32_t)N;
   a.KB = p.KB;
   a.NB = p.NB;
-  a.S = p.S;
-  a.units = p.NB * p.S;
+  a.W = p.W;
+  a.G = p.G;
   a.part = part;
-  a.cnt = cnt;
   a.y = static_cast<uint16_t *>(y);
   a.ldy = ldy;
   switch (p.NT) {

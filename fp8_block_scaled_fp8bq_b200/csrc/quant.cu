@@ -158,12 +158,11 @@ fp8bq_status launch_quant_act(const void *x, int64_t M, int64_t K, int64_t ldx, 
   const uint16_t *xs = static_cast<const uint16_t *>(x);
   const bool vec = aligned(x, 16) && ldx % 8 == 0 && K % 8 == 0 && aligned(q, 8) && ldq % 8 == 0;
   if (vec) {
-    constexpr int U = 4;
-    dim3 grid((unsigned)((M + 16 * U - 1) / (16 * U)), (unsigned)KB);
+    dim3 grid((unsigned)((M + 63) / 64), (unsigned)KB);
     if (mode == FP8BQ_SCALE_FP32)
-      quant_act_vec_kernel<FP8BQ_SCALE_FP32, U><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, ldq, sa, ldsa);
+      quant_act_vec_kernel<FP8BQ_SCALE_FP32><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, ldq, sa, ldsa);
     else
-      quant_act_vec_kernel<FP8BQ_SCALE_POW2, U><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, ldq, sa, ldsa);
+      quant_act_vec_kernel<FP8BQ_SCALE_POW2><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, ldq, sa, ldsa);
   } else {
     dim3 grid((unsigned)((M + 15) / 16), (unsigned)KB);
     if (mode == FP8BQ_SCALE_FP32)

@@ -98,14 +98,35 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
 }
 
+// Two quotients at once with the packed FP32 instructions (the same IEEE
+// operations, two lanes per instruction); fma(q0, -s, x) forms the same exact
+// residual as fma(-q0, s, x).
+template <int MODE>
+__device__ __forceinline__ float2 quotient2(float2 x, const TileScale &t) {
+  const float2 r2 = make_float2(t.r, t.r);
+  if (MODE == FP8BQ_SCALE_POW2) return __fmul2_rn(x, r2);
+  if (t.exact) return make_float2(__fdiv_rn(x.x, t.s), __fdiv_rn(x.y, t.s));
+  const float2 q0 = __fmul2_rn(x, r2);
+  const float2 res = __ffma2_rn(q0, make_float2(-t.s, -t.s), x);
+  const float2 q1 = __ffma2_rn(res, r2, q0);
+  return make_float2(
+      __uint_as_float((__float_as_uint(q1.x) & 0x7FFFFFFFu) | (__float_as_uint(x.x) & 0x80000000u)),
+      __uint_as_float((__float_as_uint(q1.y) & 0x7FFFFFFFu) | (__float_as_uint(x.y) & 0x80000000u)));
+}
+
+// Two bf16 packed in a 32-bit word (lower address in the low half) -> E4M3x2.
+template <int MODE>
+__device__ __forceinline__ uint32_t encode2(uint32_t w, const TileScale &t) {
+  const float2 q = quotient2<MODE>(make_float2(bf16_lo(w), bf16_hi(w)), t);
+  return e4m3x2(q.x, q.y);
+}
+
 // 8 bf16 (one 16-byte vector) -> 8 E4M3 codes (8 bytes).
 template <int MODE>
 __device__ __forceinline__ uint2 encode8(uint4 v, const TileScale &t) {
   uint2 r;
-  r.x = e4m3x2(quotient<MODE>(bf16_lo(v.x), t), quotient<MODE>(bf16_hi(v.x), t)) |
-        (e4m3x2(quotient<MODE>(bf16_lo(v.y), t), quotient<MODE>(bf16_hi(v.y), t)) << 16);
-  r.y = e4m3x2(quotient<MODE>(bf16_lo(v.z), t), quotient<MODE>(bf16_hi(v.z), t)) |
-        (e4m3x2(quotient<MODE>(bf16_lo(v.w), t), quotient<MODE>(bf16_hi(v.w), t)) << 16);
+  r.x = encode2<MODE>(v.x, t) | (encode2<MODE>(v.y, t) << 16);
+  r.y = encode2<MODE>(v.z, t) | (encode2<MODE>(v.w, t) << 16);
   return r;
 }
 
@@ -120,39 +141,36 @@ __device__ __forceinline__ float bits_to_amax(uint32_t b16) { return __uint_as_f
 // ---------------------------------------------------------------------------
 // Activation quantization, 1x128 tiles
 // ---------------------------------------------------------------------------
-// Block = 8 warps; a half-warp owns one 1x128 tile (16 lanes x 8 elements);
-// each half-warp handles U rows of one K-block, all loads issued first.
-// Block (bx, by) covers rows [bx * 16U, +16U) of K-block by.
-template <int MODE, int U>
+// Block = 8 warps = 64 tiles: rows [bx * 64, +64) of K-block by.  Four lanes
+// share a tile: lane qd holds the tile's 16-byte chunks qd, qd+4, qd+8, qd+12
+// (32 elements), so each load instruction reads 64 contiguous bytes per row and
+// each store writes 32; the tile amax takes two shuffles and every lane's
+// scale computation is spread over 32 elements.
+template <int MODE>
 __device__ __forceinline__ void quant_act_vec_block(int64_t bx, int64_t by, const uint16_t *__restrict__ x,
                                                     int64_t M, int64_t K, int64_t ldx, uint8_t *__restrict__ q,
                                                     int64_t ldq, float *__restrict__ sa, int64_t ldsa) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hl = lane & 15, half = lane >> 4;
+  const int qd = lane & 3;
+  const int64_t r = bx * 64 + warp * 8 + (lane >> 2);
   const int64_t kb = by;
-  const int64_t k = kb * 128 + hl * 8;
-  const bool kin = k < K;  // K % 8 == 0 here: a vector is wholly in or out
-  const int64_t rbase = bx * (16 * U) + warp * (2 * U) + half;
-
-  uint4 v[U];
+  uint4 v[4];
 #pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int64_t r = rbase + 2 * u;
-    v[u] = (kin && r < M) ? ld_nc_v4(x + r * ldx + k) : make_uint4(0, 0, 0, 0);
+  for (int j = 0; j < 4; ++j) {
+    const int64_t k = kb * 128 + (j * 4 + qd) * 8;  // K % 8 == 0 here: a vector is wholly in or out
+    v[j] = (r < M && k < K) ? ld_nc_v4(x + r * ldx + k) : make_uint4(0, 0, 0, 0);
   }
+  uint32_t m = max(max(absmax_bits8(v[0]), absmax_bits8(v[1])), max(absmax_bits8(v[2]), absmax_bits8(v[3])));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  const TileScale ts = tile_scale<MODE>(bits_to_amax(m));
+  if (r < M) {
 #pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int64_t r = rbase + 2 * u;
-    uint32_t m = absmax_bits8(v[u]);
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 8));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    const TileScale ts = tile_scale<MODE>(bits_to_amax(m));
-    if (r < M) {
-      if (kin) *reinterpret_cast<uint2 *>(q + r * ldq + k) = encode8<MODE>(v[u], ts);
-      if (hl == 0) sa[kb * ldsa + r] = ts.s;
+    for (int j = 0; j < 4; ++j) {
+      const int64_t k = kb * 128 + (j * 4 + qd) * 8;
+      if (k < K) *reinterpret_cast<uint2 *>(q + r * ldq + k) = encode8<MODE>(v[j], ts);
     }
+    if (qd == 0) sa[kb * ldsa + r] = ts.s;
   }
 }
 
@@ -191,11 +209,11 @@ __device__ __forceinline__ void quant_act_scalar_block(int64_t bx, int64_t by, c
   if (hl == 0) sa[kb * ldsa + r] = ts.s;
 }
 
-template <int MODE, int U>
+template <int MODE>
 __global__ void __launch_bounds__(256) quant_act_vec_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
                                                             int64_t ldx, uint8_t *__restrict__ q, int64_t ldq,
                                                             float *__restrict__ sa, int64_t ldsa) {
-  quant_act_vec_block<MODE, U>(blockIdx.x, blockIdx.y, x, M, K, ldx, q, ldq, sa, ldsa);
+  quant_act_vec_block<MODE>(blockIdx.x, blockIdx.y, x, M, K, ldx, q, ldq, sa, ldsa);
 }
 
 template <int MODE>
