@@ -449,12 +449,21 @@ def run_case(args):
         N, K = wl.LLAMA8B_SHAPES[what]
         a = wl.activations(M, K, seed=1, device=dev).to(torch.float8_e4m3fn)
         b = wl.weights(N, K, seed=2, device=dev).mul(20).to(torch.float8_e4m3fn)
-        if args.pow2:   # blockwise: 1x128 for a, 128x128 for b
-            sa_ = torch.ones((M, K // 128), dtype=torch.float32, device=dev)
-            sb_ = torch.ones((K // 128, (N + 127) // 128), dtype=torch.float32, device=dev).t()
-        else:
-            sa_ = torch.ones((), dtype=torch.float32, device=dev)
-            sb_ = torch.ones((), dtype=torch.float32, device=dev)
+        sa_ = torch.ones((), dtype=torch.float32, device=dev)
+        sb_ = torch.ones((), dtype=torch.float32, device=dev)
+        if args.pow2:
+            # blockwise: 1x128 for a (outer-dim-major), 128x128 for b; the layouts
+            # torch documents in its error text; fall back to per-tensor if refused
+            cand_a = torch.ones((K // 128, M), dtype=torch.float32, device=dev).t()
+            for cand_b in (torch.ones(((N + 127) // 128, K // 128), dtype=torch.float32, device=dev).t(),
+                           torch.ones((K // 128, (N + 127) // 128), dtype=torch.float32, device=dev)):
+                try:
+                    torch._scaled_mm(a, b.t(), scale_a=cand_a, scale_b=cand_b, out_dtype=torch.bfloat16)
+                    sa_, sb_ = cand_a, cand_b
+                    print(json.dumps({"case": args.case, "cublas_scaling": "blockwise 1x128 x 128x128"}))
+                    break
+                except RuntimeError as e:
+                    print(json.dumps({"case": args.case, "cublas_refused": str(e).splitlines()[0][:120]}))
         fn = lambda: torch._scaled_mm(a, b.t(), scale_a=sa_, scale_b=sb_, out_dtype=torch.bfloat16)  # noqa: E731
         work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
     elif kind == "decode":

@@ -206,7 +206,8 @@ fp8bq_status fp8bq_recalibrate(const fp8bq_weight_desc *descs, int n, int mode, 
 fp8bq_status fp8bq_gemm_ex(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
                            int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                            int mode, int variant, void *stream) {
-  if (variant < FP8BQ_GEMM_AUTO || variant > FP8BQ_GEMM_NATIVE_POW2) return FP8BQ_ERR_INVALID_ARG;
+  if ((variant < FP8BQ_GEMM_AUTO || variant > FP8BQ_GEMM_NATIVE_POW2) && variant != FP8BQ_GEMM_SELFTEST_TIMEOUT)
+    return FP8BQ_ERR_INVALID_ARG;
   if (variant == FP8BQ_GEMM_NATIVE_POW2 && mode != FP8BQ_SCALE_POW2) return FP8BQ_ERR_INVALID_ARG;
   fp8bq_status st = check_gemm_operands(qa, lda, sa, ldsa, qw, ldw, sw, y, ldy, M, N, K, mode);
   if (st != FP8BQ_OK || M == 0 || N == 0) return st;

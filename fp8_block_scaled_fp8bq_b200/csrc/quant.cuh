@@ -81,17 +81,17 @@ __device__ __forceinline__ TileScale tile_scale(float amax) {
   return t;
 }
 
-// The binary32 quotient x / s, correctly rounded.
+// The binary32 quotient x / s, correctly rounded.  The residual is formed as
+// q0 s - x (exact by one fma) and subtracted in the correcting fma, which keeps
+// the sign of zero: x = -0 gives q0 = -0, residual +0 and q1 = -0 + -0 = -0,
+// while x = +0 gives +0.
 template <int MODE>
 __device__ __forceinline__ float quotient(float x, const TileScale &t) {
   if (MODE == FP8BQ_SCALE_POW2) return __fmul_rn(x, t.r);
   if (t.exact) return __fdiv_rn(x, t.s);
   const float q0 = __fmul_rn(x, t.r);
-  const float res = __fmaf_rn(-q0, t.s, x);
-  const float q1 = __fmaf_rn(res, t.r, q0);
-  // x / s has the sign of x (s > 0); the correction step turns -0 into +0, so
-  // the sign is taken from x.
-  return __uint_as_float((__float_as_uint(q1) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
+  const float res = __fmaf_rn(q0, t.s, -x);
+  return __fmaf_rn(-res, t.r, q0);
 }
 
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
@@ -99,19 +99,15 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
 }
 
 // Two quotients at once with the packed FP32 instructions (the same IEEE
-// operations, two lanes per instruction); fma(q0, -s, x) forms the same exact
-// residual as fma(-q0, s, x).
+// operations as quotient(), two lanes per instruction).
 template <int MODE>
 __device__ __forceinline__ float2 quotient2(float2 x, const TileScale &t) {
   const float2 r2 = make_float2(t.r, t.r);
   if (MODE == FP8BQ_SCALE_POW2) return __fmul2_rn(x, r2);
   if (t.exact) return make_float2(__fdiv_rn(x.x, t.s), __fdiv_rn(x.y, t.s));
   const float2 q0 = __fmul2_rn(x, r2);
-  const float2 res = __ffma2_rn(q0, make_float2(-t.s, -t.s), x);
-  const float2 q1 = __ffma2_rn(res, r2, q0);
-  return make_float2(
-      __uint_as_float((__float_as_uint(q1.x) & 0x7FFFFFFFu) | (__float_as_uint(x.x) & 0x80000000u)),
-      __uint_as_float((__float_as_uint(q1.y) & 0x7FFFFFFFu) | (__float_as_uint(x.y) & 0x80000000u)));
+  const float2 res = __ffma2_rn(q0, make_float2(t.s, t.s), make_float2(-x.x, -x.y));
+  return __ffma2_rn(make_float2(-res.x, -res.y), r2, q0);
 }
 
 // Two bf16 packed in a 32-bit word (lower address in the low half) -> E4M3x2.

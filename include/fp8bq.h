@@ -181,7 +181,12 @@ FP8BQ_API fp8bq_status fp8bq_gemm(const uint8_t *qa, int64_t lda, const float *s
 typedef enum {
     FP8BQ_GEMM_AUTO = 0,          /* what fp8bq_gemm does */
     FP8BQ_GEMM_PROMOTE = 1,       /* FP32 promotion of every K-block partial */
-    FP8BQ_GEMM_NATIVE_POW2 = 2    /* native block-scaled MMA (POW2 scales only) */
+    FP8BQ_GEMM_NATIVE_POW2 = 2,   /* native block-scaled MMA (POW2 scales only) */
+    FP8BQ_GEMM_SELFTEST_TIMEOUT = 99  /* failure-detection self-test: the promotion kernel runs
+                                         with its TMA producer disabled, so its MMA issuer's
+                                         bounded wait runs out (about 1 s); the call returns
+                                         FP8BQ_OK, y is not written, and the next
+                                         fp8bq_get_device_error reports FP8BQ_ERR_TIMEOUT */
 } fp8bq_gemm_variant;
 
 FP8BQ_API fp8bq_status fp8bq_gemm_ex(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa,
