@@ -440,7 +440,7 @@ def run_case(args):
         qa, sa = fq.quant_act(x, mode)
         qw, sw = fq.quant_weight(w, mode)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        variant = fq.GEMM_NATIVE_POW2 if args.native else fq.GEMM_PROMOTE
+        variant = fq.GEMM_NATIVE_POW2 if args.native else (fq.GEMM_PROMOTE_PAIR if args.pair else fq.GEMM_PROMOTE)
         fn = lambda: fq.gemm(qa, sa, qw, sw, mode, out=y, variant=variant)  # noqa: E731
         work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
     elif kind == "cublas":
@@ -542,6 +542,7 @@ def main():
     ap.add_argument("--pow2", action="store_true", help="power-of-2 scales for --case")
     ap.add_argument("--graph", action="store_true", help="--case: time a CUDA graph of --steps calls")
     ap.add_argument("--native", action="store_true", help="--case gemm with --pow2: native block-scaled MMA")
+    ap.add_argument("--pair", action="store_true", help="--case gemm: the CTA-pair promotion kernel")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)

@@ -22,6 +22,7 @@ SCALE_POW2 = 1
 GEMM_AUTO = 0
 GEMM_PROMOTE = 1
 GEMM_NATIVE_POW2 = 2
+GEMM_PROMOTE_PAIR = 3
 GEMM_SELFTEST_TIMEOUT = 99
 
 _HERE = os.path.dirname(os.path.abspath(__file__))

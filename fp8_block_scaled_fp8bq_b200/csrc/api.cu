@@ -140,7 +140,8 @@ fp8bq_status fp8bq_get_device_error(uint64_t *code) {
   unsigned long long v = 0, w = 0;
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-  cudaError_t (*takers[])(unsigned long long *) = {take_device_error_gemm, take_device_error_decode, take_device_error_native};
+  cudaError_t (*takers[])(unsigned long long *) = {take_device_error_gemm, take_device_error_decode, take_device_error_native,
+                                                       take_device_error_pair};
   for (auto take : takers) {
     e = take(&w);
     if (e != cudaSuccess) return cuda_fail(e, "read device error word");
@@ -206,7 +207,7 @@ fp8bq_status fp8bq_recalibrate(const fp8bq_weight_desc *descs, int n, int mode, 
 fp8bq_status fp8bq_gemm_ex(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
                            int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                            int mode, int variant, void *stream) {
-  if ((variant < FP8BQ_GEMM_AUTO || variant > FP8BQ_GEMM_NATIVE_POW2) && variant != FP8BQ_GEMM_SELFTEST_TIMEOUT)
+  if ((variant < FP8BQ_GEMM_AUTO || variant > FP8BQ_GEMM_PROMOTE_PAIR) && variant != FP8BQ_GEMM_SELFTEST_TIMEOUT)
     return FP8BQ_ERR_INVALID_ARG;
   if (variant == FP8BQ_GEMM_NATIVE_POW2 && mode != FP8BQ_SCALE_POW2) return FP8BQ_ERR_INVALID_ARG;
   fp8bq_status st = check_gemm_operands(qa, lda, sa, ldsa, qw, ldw, sw, y, ldy, M, N, K, mode);

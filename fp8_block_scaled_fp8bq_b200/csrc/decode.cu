@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (lane == 0) mbar_arrive_relaxed(&tempty[buf]);
 #pragma unroll
       for (int j = 0; j < C::kCW / 4; ++j) {
         const float4 s4 = sc4[j];

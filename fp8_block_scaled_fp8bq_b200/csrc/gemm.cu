@@ -370,7 +370,7 @@ __device__ __forceinline__ void run_epilogue(const Smem &S, uint32_t tmem_base, 
         if (c == 1) {  // the buffer has been read: hand it back to the MMA warp
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&S.tempty[buf]);
+          if (lane == 0) mbar_arrive_relaxed(&S.tempty[buf]);
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j)
@@ -544,14 +544,15 @@ cudaError_t take_device_error_gemm(unsigned long long *v) { return take_tu_devic
 fp8bq_status launch_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
                          int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K, int mode,
                          int variant, cudaStream_t stream) {
-  (void)mode;
   if (M == 0 || N == 0) return FP8BQ_OK;
   if (K == 0) {
     cudaError_t e = cudaMemset2DAsync(y, (size_t)ldy * 2, 0, (size_t)N * 2, (size_t)M, stream);
     return e == cudaSuccess ? FP8BQ_OK : cuda_fail(e, "memset(y)");
   }
-  if (variant == FP8BQ_GEMM_NATIVE_POW2)
+  if (variant == FP8BQ_GEMM_NATIVE_POW2 || (variant == FP8BQ_GEMM_AUTO && mode == FP8BQ_SCALE_POW2))
     return launch_gemm_native(qa, lda, sa, ldsa, qw, ldw, sw, y, ldy, M, N, K, stream);
+  if (variant == FP8BQ_GEMM_PROMOTE_PAIR)
+    return launch_gemm_pair(qa, lda, sa, ldsa, qw, ldw, sw, y, ldy, M, N, K, stream);
   CUtensorMap tA, tB, tY;
   if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qa, (uint64_t)K, (uint64_t)M, (uint64_t)lda, BK, BM,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||

@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty);  // the next tile's MMAs may overwrite the accumulator
+      if (lane == 0) mbar_arrive_relaxed(tempty);  // the next tile's MMAs may overwrite the accumulator
 #pragma unroll
       for (int c = 0; c < 4; ++c) {  // four 32-column chunks
         if (lane == 0) bulk_wait_group_read0();

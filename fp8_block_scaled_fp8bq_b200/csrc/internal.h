@@ -36,6 +36,7 @@ bool make_tmap_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
 cudaError_t take_device_error_gemm(unsigned long long *v);
 cudaError_t take_device_error_decode(unsigned long long *v);
 cudaError_t take_device_error_native(unsigned long long *v);
+cudaError_t take_device_error_pair(unsigned long long *v);
 
 // Launchers (arguments already validated).
 fp8bq_status launch_encode(const float *x, int64_t n, uint8_t *q, cudaStream_t stream);
@@ -45,6 +46,10 @@ fp8bq_status launch_recalibrate(const fp8bq_weight_desc *descs, int n, int mode,
 fp8bq_status launch_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
                          int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K, int mode,
                          int variant, cudaStream_t stream);
+bool pair_gemm_available();
+fp8bq_status launch_gemm_pair(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                              int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                              cudaStream_t stream);
 fp8bq_status launch_gemm_native(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
                                 int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                                 cudaStream_t stream);

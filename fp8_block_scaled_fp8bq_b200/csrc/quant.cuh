@@ -47,9 +47,9 @@ __device__ __forceinline__ float exp2_exact(int e) {
 //   FP32 scales: s = amax / 448; r = RN(1/s).  When s >= 2^-60 the quotient is
 //     computed with Markstein's correction (P. Markstein, "Computation of
 //     elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
-//     Dev. 34(1), 1990): q0 = RN(x r), the residual x - q0 s is formed exactly
-//     by one fma, and q1 = RN(q0 + residual * r) is the correctly rounded
-//     quotient.  Below 2^-60 (tiles whose amax is under ~4e-16) the residual
+//     Dev. 34(1), 1990): q0 = RN(x r), the residual q0 s - x is formed
+//     exactly by one fma, and q1 = RN(q0 - residual * r) is the correctly
+//     rounded quotient (see quotient() for the sign of zero).  Below 2^-60 (tiles whose amax is under ~4e-16) the residual
 //     could underflow, so those tiles use the IEEE division.  A GPU test
 //     compares the codes this produces with the oracle's (an IEEE division)
 //     for every pair (tile amax, element) of bf16 values.

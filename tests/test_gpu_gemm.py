@@ -18,7 +18,7 @@ import oracle
 from helpers import assert_gemm_close, bf16_bits, bf16_to_f64, f32, need_gpu, u8
 
 pytestmark = pytest.mark.gpu
-VARIANTS = [fq.GEMM_PROMOTE]
+VARIANTS = [fq.GEMM_PROMOTE, fq.GEMM_PROMOTE_PAIR]
 
 
 @pytest.fixture(autouse=True)
@@ -139,3 +139,17 @@ def test_row_subset_gives_identical_rows():
     y2 = fq.gemm(qa2, sa2, qw, sw)
     torch.cuda.synchronize()
     assert torch.equal(y[128:256].view(torch.int16), y2.view(torch.int16))
+
+
+def test_pair_kernel_equals_one_sm_kernel():
+    """The CTA-pair kernel (256x256 tiles, paired MMA) and the one-SM kernel
+    compute every output from the same K-block partials in the same order."""
+    x = wl.activations(640, 1024, seed=21, device="cuda")
+    w = wl.weights(768, 1024, seed=22, device="cuda")
+    qa, sa = fq.quant_act(x)
+    qw, sw = fq.quant_weight(w)
+    y_pair = fq.gemm(qa, sa, qw, sw, variant=fq.GEMM_PROMOTE_PAIR)
+    y_one = fq.gemm(qa, sa, qw, sw, variant=fq.GEMM_PROMOTE)
+    torch.cuda.synchronize()
+    assert_gemm_close(bf16_to_f64(y_pair), bf16_to_f64(y_one), "pair vs one-SM")
+    assert torch.equal(y_pair.view(torch.int16), y_one.view(torch.int16))
