@@ -73,20 +73,32 @@ def load_peaks():
 
 def kernel_source_sha():
     h = hashlib.sha256()
-    for f in ("gemm.cu", "device.cuh"):
+    for f in ("gemm.cu", "device.cuh", "api.cu"):
         h.update(open(os.path.join(ROOT, "fp8_block_scaled_fp8bq_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def committed_traffic():
-    """DRAM bytes per GEMM launch from the committed ncu summary, if the kernel is unchanged."""
-    p = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    """DRAM bytes per GEMM launch from the committed ncu summary, if the kernel is unchanged.
+
+    The summary holds `key: value` lines; `source_sha` names the kernel sources
+    the counters were taken from and `dram_bytes_per_launch_step_avg` is the
+    mean over the step's four GEMM launches of dram__bytes_read.sum +
+    dram__bytes_write.sum."""
+    p = os.path.join(ROOT, "profiles", "gemm_traffic_llama8b_layer_M8192.txt")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
+    d = {}
+    for line in open(p):
+        if ":" in line and not line.startswith((" ", "#", "`")):
+            k, v = line.split(":", 1)
+            d[k.strip()] = v.strip()
     if d.get("source_sha") != kernel_source_sha():
         return None
-    return d.get("dram_bytes_per_launch_step_avg")
+    try:
+        return int(d["dram_bytes_per_launch_step_avg"])
+    except (KeyError, ValueError):
+        return None
 
 
 # --------------------------------------------------------------------------- clocks

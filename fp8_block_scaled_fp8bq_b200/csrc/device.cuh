@@ -398,6 +398,24 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) 
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Tile order of the persistent GEMMs.  Output tiles (mi, ni) of a num_m x
+// num_n grid are visited in bands of `band` consecutive indices of one
+// dimension (M when n_major == 0, N otherwise); inside a band that dimension
+// runs fastest.  The band's operand panels are re-read from L2 by every tile of
+// the band while the other operand streams through once per band.
+__device__ __forceinline__ void raster_tile(int t, int num_m, int num_n, int band, int n_major, int &mi, int &ni) {
+  const int along = n_major ? num_n : num_m;
+  const int across = n_major ? num_m : num_n;
+  const int per = band * across;
+  const int g = t / per;
+  const int first = g * band;
+  const int width = min(along - first, band);
+  const int r = t - g * per;
+  const int i = first + r % width, j = r / width;
+  mi = n_major ? j : i;
+  ni = n_major ? i : j;
+}
+
 __device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"

@@ -71,7 +71,6 @@ constexpr int kLowRegs = 56;
 constexpr int kHighRegs = 224;
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int kTmemCols = 2 * BN;
-constexpr int kGroupM = 16;
 constexpr int kBarBytes = 256;
 
 // Per-warp bf16 staging: dense = 32 rows x 64 columns in the TMA 128-byte
@@ -91,6 +90,7 @@ struct GemmArgs {
   int64_t ldsa;
   int32_t M, N, KB, NB;     // grouped: M = total rows
   int32_t num_m, num_n;     // dense tile grid; grouped: num_n only
+  int32_t band, n_major;    // dense tile order (raster_tile)
   // grouped only
   const int32_t *offsets;   // [E+1], device
   int32_t E;
@@ -106,16 +106,13 @@ struct Tile {
 };
 
 __device__ __forceinline__ Tile dense_tile(int t, const GemmArgs &a) {
-  const int per_group = kGroupM * a.num_n;
-  const int g = t / per_group;
-  const int first_m = g * kGroupM;
-  const int gm = min(a.num_m - first_m, kGroupM);
-  const int r = t - g * per_group;
+  int mi, ni;
+  raster_tile(t, a.num_m, a.num_n, a.band, a.n_major, mi, ni);
   Tile tl;
   tl.e = 0;
-  tl.row0 = (first_m + r % gm) * BM;
+  tl.row0 = mi * BM;
   tl.row_end = a.M;
-  tl.nb = r / gm;
+  tl.nb = ni;
   return tl;
 }
 
@@ -573,6 +570,7 @@ fp8bq_status launch_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_
   a.NB = (int32_t)((N + 127) / 128);
   a.num_m = (int32_t)((M + BM - 1) / BM);
   a.num_n = (int32_t)((N + BN - 1) / BN);
+  choose_raster(M, N, K, BM, BN, &a.band, &a.n_major);
   a.selftest = variant == FP8BQ_GEMM_SELFTEST_TIMEOUT ? 1 : 0;
   const int64_t tiles = (int64_t)a.num_m * a.num_n;
   const int grid = (int)std::min<int64_t>(tiles, num_sms());

@@ -58,7 +58,6 @@ static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "regis
 constexpr int kTmemCols = 512;
 constexpr int kAccCols = BN;       // one 128 x 256 FP32 accumulator
 constexpr int kSFCols = 12;        // per stage: SFA 4 + SFB 8 TMEM columns
-constexpr int kGroupM = 16;
 constexpr int kSmemBytes =
     kStages * (kABytes + kBBytes) + kStages * kSFBytes + kEpiWarps * kEpiBufBytes + 256 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -70,16 +69,11 @@ struct NativeArgs {
   int64_t ldsa;
   int32_t M, N, KB, NB;
   int32_t num_m, num_n;
+  int32_t band, n_major;  // tile order (raster_tile)
 };
 
 __device__ __forceinline__ void tile_mn(int t, const NativeArgs &a, int &mb, int &nb) {
-  const int per_group = kGroupM * a.num_n;
-  const int g = t / per_group;
-  const int first_m = g * kGroupM;
-  const int gm = min(a.num_m - first_m, kGroupM);
-  const int r = t - g * per_group;
-  mb = first_m + r % gm;
-  nb = r / gm;
+  raster_tile(t, a.num_m, a.num_n, a.band, a.n_major, mb, nb);
 }
 
 // UE8M0 of a power-of-two fp32 scale: its exponent field (2^-127, a binary32
@@ -357,6 +351,7 @@ fp8bq_status launch_gemm_native(const uint8_t *qa, int64_t lda, const float *sa,
   a.NB = (int32_t)((N + 127) / 128);
   a.num_m = (int32_t)((M + BM - 1) / BM);
   a.num_n = (int32_t)((N + BN - 1) / BN);
+  choose_raster(M, N, K, BM, BN, &a.band, &a.n_major);
   const int64_t tiles = (int64_t)a.num_m * a.num_n;
   const int grid = (int)std::min<int64_t>(tiles, num_sms());
   gemm_native_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tA, tB, tY, a);

@@ -54,7 +54,6 @@ constexpr int kLowRegs = 56;
 constexpr int kHighRegs = 224;
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int kTmemCols = 2 * PBN;
-constexpr int kGroupM = 8;
 constexpr int kSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiBufBytes + 256 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -64,16 +63,11 @@ struct PairArgs {
   int64_t ldsa;
   int32_t M, N, KB, NB;
   int32_t num_m, num_n;  // pair tiles (256 x 256)
+  int32_t band, n_major;  // tile order (raster_tile)
 };
 
 __device__ __forceinline__ void pair_tile(int t, const PairArgs &a, int &pm, int &nb) {
-  const int per_group = kGroupM * a.num_n;
-  const int g = t / per_group;
-  const int first_m = g * kGroupM;
-  const int gm = min(a.num_m - first_m, kGroupM);
-  const int r = t - g * per_group;
-  pm = first_m + r % gm;
-  nb = r / gm;
+  raster_tile(t, a.num_m, a.num_n, a.band, a.n_major, pm, nb);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -381,6 +375,7 @@ fp8bq_status launch_gemm_pair(const uint8_t *qa, int64_t lda, const float *sa, i
   a.NB = (int32_t)((N + 127) / 128);
   a.num_m = (int32_t)((M + PBM - 1) / PBM);
   a.num_n = (int32_t)((N + PBN - 1) / PBN);
+  choose_raster(M, N, K, PBM, PBN, &a.band, &a.n_major);
   int dev = 0;
   cudaGetDevice(&dev);
   const int64_t tiles = (int64_t)a.num_m * a.num_n;

@@ -32,6 +32,12 @@ bool make_tmap_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
                   CUtensorMapSwizzle swizzle);
 
+// Tile order of a persistent GEMM over an M x N output in bm x bn tiles with
+// depth K (bytes per operand row = K): picks the banded dimension and the band
+// width (see raster_tile) that minimise the operand bytes read from DRAM when
+// a band's panels of one operand stay in L2.
+void choose_raster(int64_t M, int64_t N, int64_t K, int bm, int bn, int32_t *band, int32_t *n_major);
+
 // Per translation unit: read and clear its device error word.
 cudaError_t take_device_error_gemm(unsigned long long *v);
 cudaError_t take_device_error_decode(unsigned long long *v);

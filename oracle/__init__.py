@@ -69,6 +69,10 @@ def lib():
         L.o_f64_to_bf16.argtypes = [ctypes.c_double]
         L.o_f64_to_bf16_array.restype = None
         L.o_f64_to_bf16_array.argtypes = [P, I64, P]
+        L.o_silu.restype = ctypes.c_double
+        L.o_silu.argtypes = [ctypes.c_double]
+        L.o_swiglu_bf16.restype = None
+        L.o_swiglu_bf16.argtypes = [P, P, I64, P]
         L.o_num_threads.restype = ctypes.c_int
         L.o_num_threads.argtypes = []
         _lib = L
@@ -232,3 +236,44 @@ def f64_to_bf16(v):
     out = np.empty(v.shape, dtype=np.uint16)
     lib().o_f64_to_bf16_array(_p(v), v.size, _p(out))
     return out
+
+
+# --- gate/up activation (SwiGLU) and the fused gate+up -> H codes composition
+
+def silu(g):
+    """silu(g) = g / (1 + e^-g) in double."""
+    return lib().o_silu(float(g))
+
+
+def swiglu_bf16(g_bits, u_bits):
+    """h = bf16_RNE(silu(g) * u) elementwise on bf16 bit patterns (double arithmetic)."""
+    g = _c(np.asarray(g_bits, dtype=np.uint16), np.uint16)
+    u = _c(np.asarray(u_bits, dtype=np.uint16), np.uint16)
+    if g.shape != u.shape:
+        raise ValueError("gate and up shapes differ")
+    h = np.empty(g.shape, dtype=np.uint16)
+    lib().o_swiglu_bf16(_p(g), _p(u), g.size, _p(h))
+    return h
+
+
+def split_gate_up(y_bits):
+    """De-interleave a gate+up output [R, 2I] whose 128-column blocks alternate
+    gate block j, up block j (j = 0..I/128-1) into (g [R, I], u [R, I])."""
+    y = np.asarray(y_bits)
+    R, N2 = y.shape
+    if N2 % 256:
+        raise ValueError("the gate+up width must be a multiple of 256")
+    blocks = y.reshape(R, N2 // 256, 2, 128)
+    return (np.ascontiguousarray(blocks[:, :, 0, :].reshape(R, N2 // 2)),
+            np.ascontiguousarray(blocks[:, :, 1, :].reshape(R, N2 // 2)))
+
+
+def swiglu_quant_from_y(y64, mode):
+    """The fused epilogue's definition, from the gate+up GEMM's FP64 result
+    [R, 2I]: round to bf16 (the GEMM's output), h = swiglu_bf16(g, u), then the
+    1x128 activation quantization of h.  Returns (codes [R, I], scales [I/128, R],
+    h bits [R, I])."""
+    g, u = split_gate_up(f64_to_bf16(y64))
+    h = swiglu_bf16(g, u)
+    q, s = quant_act(h, mode)
+    return q, s, h

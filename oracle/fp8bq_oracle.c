@@ -435,4 +435,23 @@ O_API void o_f64_to_bf16_array(const double *v, int64_t n, uint16_t *out)
     for (i = 0; i < n; ++i) out[i] = o_f64_to_bf16(v[i]);
 }
 
+/*
+ * The gated feed-forward activation between the gate+up projection and the
+ * down projection of a Llama-style block.  The pages name Llama 3.1 8B
+ * (section "Technical breakthrough"), whose feed-forward block is SwiGLU
+ * (N. Shazeer, "GLU Variants Improve Transformer", 2020):
+ *     h = silu(g) * u,   silu(g) = g * sigmoid(g) = g / (1 + e^-g),
+ * with g the gate projection and u the up projection.  The same section keeps
+ * non-linear functions in BF16: g and u are the BF16 outputs of the FP8 GEMM
+ * and h is rounded to BF16 once; the arithmetic here is double.
+ */
+O_API double o_silu(double g) { return g / (1.0 + exp(-g)); }
+
+O_API void o_swiglu_bf16(const uint16_t *g, const uint16_t *u, int64_t n, uint16_t *h)
+{
+    int64_t i;
+#pragma omp parallel for schedule(static)
+    for (i = 0; i < n; ++i) h[i] = o_f64_to_bf16(o_silu((double)o_bf16(g[i])) * (double)o_bf16(u[i]));
+}
+
 O_API int o_num_threads(void) { return omp_get_max_threads(); }
