@@ -73,6 +73,11 @@ def lib():
         L.o_silu.argtypes = [ctypes.c_double]
         L.o_swiglu_bf16.restype = None
         L.o_swiglu_bf16.argtypes = [P, P, I64, P]
+        L.o_adamw_step.restype = None
+        L.o_adamw_step.argtypes = [P, P, P, P, I64, ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                   ctypes.c_float, I64]
+        L.o_f32_to_bf16_array.restype = None
+        L.o_f32_to_bf16_array.argtypes = [P, I64, P]
         L.o_num_threads.restype = ctypes.c_int
         L.o_num_threads.argtypes = []
         _lib = L
@@ -277,3 +282,36 @@ def swiglu_quant_from_y(y64, mode):
     h = swiglu_bf16(g, u)
     q, s = quant_act(h, mode)
     return q, s, h
+
+
+# --- optimizer step + recalibration -------------------------------------------
+
+def adamw_step(p, g, m, v, lr, beta1, beta2, eps, weight_decay, step):
+    """One binary32 AdamW step; returns new (p, m, v) (inputs are not modified)."""
+    p = np.array(_c(p, np.float32), copy=True)
+    m = np.array(_c(m, np.float32), copy=True)
+    v = np.array(_c(v, np.float32), copy=True)
+    g = _c(g, np.float32)
+    if not (p.shape == g.shape == m.shape == v.shape):
+        raise ValueError("shapes differ")
+    lib().o_adamw_step(_p(p), _p(g), _p(m), _p(v), p.size, float(lr), float(beta1), float(beta2), float(eps),
+                       float(weight_decay), int(step))
+    return p, m, v
+
+
+def f32_to_bf16(x):
+    """binary32 -> bf16 bit patterns, round to nearest even."""
+    x = _c(np.asarray(x, dtype=np.float32), np.float32)
+    out = np.empty(x.shape, dtype=np.uint16)
+    lib().o_f32_to_bf16_array(_p(x), x.size, _p(out))
+    return out
+
+
+def adamw_recalibrate(p, g, m, v, lr, beta1, beta2, eps, weight_decay, step, mode):
+    """The fused optimizer step + recalibration, by composition: the AdamW step
+    on the FP32 master weight [N, K], its bf16 copy, and the 128x128
+    quantization of that copy.  Returns (p, m, v, w_bits, q, s)."""
+    p1, m1, v1 = adamw_step(p, g, m, v, lr, beta1, beta2, eps, weight_decay, step)
+    w = f32_to_bf16(p1)
+    q, s = quant_weight(w, mode)
+    return p1, m1, v1, w, q, s

@@ -454,4 +454,47 @@ O_API void o_swiglu_bf16(const uint16_t *g, const uint16_t *u, int64_t n, uint16
     for (i = 0; i < n; ++i) h[i] = o_f64_to_bf16(o_silu((double)o_bf16(g[i])) * (double)o_bf16(u[i]));
 }
 
+/*
+ * One optimizer step of an FP32 master weight, the step after which the
+ * scales are recalibrated (section "Real-world performance gains": the policy
+ * weights change every training step).  The pages do not name the optimizer;
+ * the reading is AdamW (I. Loshchilov, F. Hutter, "Decoupled Weight Decay
+ * Regularization", ICLR 2019, Algorithm 2, with Adam's bias-corrected moments
+ * of D. Kingma, J. Ba, "Adam", ICLR 2015) on binary32 state, the usual
+ * mixed-precision recipe.  Every operation below is one IEEE binary32
+ * operation, in this order (no contraction, -ffp-contract=off):
+ *   m' = b1 m + (1 - b1) g
+ *   v' = b2 v + ((1 - b2) g) g
+ *   m^ = m' / bc1,  v^ = v' / bc2,   bc_i = 1 - b_i^t  (double pow, rounded to binary32)
+ *   p' = p - lr (m^ / (sqrt(v^) + eps) + wd p)
+ */
+O_API void o_adamw_step(float *p, const float *g, float *m, float *v, int64_t n, float lr, float b1, float b2,
+                        float eps, float wd, int64_t step)
+{
+    const float bc1 = (float)(1.0 - pow((double)b1, (double)step));
+    const float bc2 = (float)(1.0 - pow((double)b2, (double)step));
+    const float c1 = 1.0f - b1, c2 = 1.0f - b2;
+    int64_t i;
+#pragma omp parallel for schedule(static)
+    for (i = 0; i < n; ++i) {
+        float mi = b1 * m[i] + c1 * g[i];
+        float vi = b2 * v[i] + (c2 * g[i]) * g[i];
+        float mh = mi / bc1;
+        float vh = vi / bc2;
+        float d = sqrtf(vh) + eps;
+        float u = mh / d + wd * p[i];
+        p[i] = p[i] - lr * u;
+        m[i] = mi;
+        v[i] = vi;
+    }
+}
+
+/* binary32 -> bf16, round to nearest even (exact through double). */
+O_API void o_f32_to_bf16_array(const float *x, int64_t n, uint16_t *out)
+{
+    int64_t i;
+#pragma omp parallel for schedule(static)
+    for (i = 0; i < n; ++i) out[i] = o_f64_to_bf16((double)x[i]);
+}
+
 O_API int o_num_threads(void) { return omp_get_max_threads(); }
