@@ -73,6 +73,8 @@ def lib():
         L.o_silu.argtypes = [ctypes.c_double]
         L.o_swiglu_bf16.restype = None
         L.o_swiglu_bf16.argtypes = [P, P, I64, P]
+        L.o_gemm_wgrad_rows.restype = None
+        L.o_gemm_wgrad_rows.argtypes = [P, I64, P, I64, P, I64, P, I64, I64, I64, I64, P, I64, P]
         L.o_adamw_step.restype = None
         L.o_adamw_step.argtypes = [P, P, P, P, I64, ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                                    ctypes.c_float, I64]
@@ -315,3 +317,43 @@ def adamw_recalibrate(p, g, m, v, lr, beta1, beta2, eps, weight_decay, step, mod
     w = f32_to_bf16(p1)
     q, s = quant_weight(w, mode)
     return p1, m1, v1, w, q, s
+
+
+# --- backward pass of the linear layer ----------------------------------------
+
+def quant_act_t(x_bits, mode):
+    """1x128 quantization along the token axis, transposed: bf16 X [M, K] ->
+    (codes of X^T [K, M], scales [ceil(M/128), K]).  The quantization of X^T
+    over 1x128 tiles of its rows (tokens are the contraction of the
+    weight-gradient GEMM)."""
+    x = _c(x_bits, np.uint16)
+    return quant_act(np.ascontiguousarray(x.T), mode)
+
+
+def gemm_dgrad(q_dy, s_dy, qw, sw, rows=None):
+    """dX = dY . W in double from 1x128 codes of dY [M, N] and the 128x128 codes
+    of W [N, K]: the forward GEMM's definition with W^T as the second operand
+    (a square tile's scale applies to its transpose unchanged)."""
+    return gemm(q_dy, s_dy, np.ascontiguousarray(np.asarray(qw).T), np.ascontiguousarray(np.asarray(sw).T),
+                rows=rows)
+
+
+def gemm_wgrad(qa, sa, qb, sb, rows=None):
+    """dW[n, k] = sum_m deq(dY^T)[n, m] deq(X^T)[k, m] in double; qa [N, M], sa [MB, >=N],
+    qb [K, M], sb [MB, >=K] (1x128 tiles along m on both operands)."""
+    qa = _c(qa, np.uint8)
+    sa = _c(sa, np.float32)
+    qb = _c(qb, np.uint8)
+    sb = _c(sb, np.float32)
+    N, M = qa.shape
+    K = qb.shape[0]
+    if rows is None:
+        r = None
+        R = N
+    else:
+        r = _c(np.asarray(rows, dtype=np.int64), np.int64)
+        R = r.size
+    y = np.empty((R, K), dtype=np.float64)
+    lib().o_gemm_wgrad_rows(_p(qa), M, _p(sa), sa.shape[1], _p(qb), M, _p(sb), sb.shape[1], N, K, M,
+                            None if r is None else _p(r), R, _p(y))
+    return y

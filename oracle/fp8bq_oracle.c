@@ -406,6 +406,42 @@ O_API void o_grouped_gemm_rows(const uint8_t *qa, int64_t lda, const float *sa, 
     }
 }
 
+/*
+ * The weight-gradient GEMM of a linear layer's backward pass, by definition:
+ * dW[n][k] = sum over tokens m of dY[m][n] X[m][k], both operands quantized
+ * over 1x128 tiles along the token axis (the contraction), given transposed:
+ * a = codes of dY^T [N][lda] with scales sa[mb*ldsa + n], b = codes of X^T
+ * [K][ldb] with scales sb[mb*ldsb + k].  Accumulated in double in ascending m,
+ * for the rows listed in rows[0..R) (rows == NULL: all N rows).  y is [R or N][K].
+ * Training in FP8 (section "Technical breakthrough": FP8 in both generation and
+ * training) multiplies activations and gradients block-wise in the backward
+ * pass as well; the 1x128 activation granularity is applied along the
+ * contraction, the plainest reading for two activation-like operands.
+ */
+O_API void o_gemm_wgrad_rows(const uint8_t *a, int64_t lda, const float *sa, int64_t ldsa,
+                             const uint8_t *b, int64_t ldb, const float *sb, int64_t ldsb,
+                             int64_t N, int64_t K, int64_t M,
+                             const int64_t *rows, int64_t R, double *y)
+{
+    int64_t nrows = rows ? R : N;
+    int64_t i;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (i = 0; i < nrows; ++i) {
+        int64_t n = rows ? rows[i] : i;
+        int64_t k;
+        for (k = 0; k < K; ++k) {
+            double acc = 0.0;
+            int64_t m;
+            for (m = 0; m < M; ++m) {
+                double da = o_e4m3_decode(a[n * lda + m]) * (double)sa[(m / 128) * ldsa + n];
+                double db = o_e4m3_decode(b[k * ldb + m]) * (double)sb[(m / 128) * ldsb + k];
+                acc += da * db;
+            }
+            y[i * K + k] = acc;
+        }
+    }
+}
+
 /* bf16 round-to-nearest-even of a double (single rounding).  NaN -> 0x7FC0. */
 O_API uint16_t o_f64_to_bf16(double v)
 {
