@@ -73,7 +73,7 @@ def load_peaks():
 
 def kernel_source_sha():
     h = hashlib.sha256()
-    for f in ("gemm.cu", "device.cuh", "api.cu"):
+    for f in ("gemm.cu", "gemm_promote.cuh", "device.cuh", "api.cu"):
         h.update(open(os.path.join(ROOT, "fp8_block_scaled_fp8bq_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -422,7 +422,9 @@ def reference(args):
 
 
 CASES = (["gemm:" + n for n in NAMES] + ["decode:" + n for n in NAMES] + ["cublas:" + n for n in NAMES] +
-         ["quant_act:4096", "quant_act:14336", "recalibrate:layer", "quant_weight:gate_up", "moe:up", "moe:down"])
+         ["quant_act:4096", "quant_act:14336", "recalibrate:layer", "quant_weight:gate_up", "moe:up", "moe:down",
+          "swiglu:gate_up", "moe_swiglu:up", "adamw_recal:layer", "quant_act_t:4096", "quant_act_t:14336",
+          "transpose_weight:gate_up"] + ["dgrad:" + n for n in NAMES] + ["wgrad:" + n for n in NAMES])
 
 
 def decode_bytes(M, N, K):
@@ -452,7 +454,8 @@ def run_case(args):
         qa, sa = fq.quant_act(x, mode)
         qw, sw = fq.quant_weight(w, mode)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        variant = fq.GEMM_NATIVE_POW2 if args.native else (fq.GEMM_PROMOTE_PAIR if args.pair else fq.GEMM_PROMOTE)
+        variant = (fq.GEMM_NATIVE_POW2 if args.native else fq.GEMM_PROMOTE_PAIR if args.pair
+                   else fq.GEMM_PROMOTE_PAIR_N128 if args.pair128 else fq.GEMM_PROMOTE)
         fn = lambda: fq.gemm(qa, sa, qw, sw, mode, out=y, variant=variant)  # noqa: E731
         work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
     elif kind == "cublas":
@@ -500,6 +503,86 @@ def run_case(args):
         fn = lambda: fq.grouped_gemm(qa, sa, qw, sw, off, mode, out=y)  # noqa: E731
         work, unit = moe_bytes(R, E, N, K) / 1e9, "GB/s"
         print(json.dumps({"case": args.case, "flops": 2.0 * R * N * K}))
+    elif kind == "swiglu":
+        # fused gate+up: the Llama gate+up weight [2I, K] taken as interleaved,
+        # H codes [M, I] and scales out (no bf16 H)
+        N, K = wl.LLAMA8B_SHAPES[what]
+        x = wl.activations(M, K, seed=1, device=dev)
+        w = wl.weights(N, K, seed=2, device=dev)
+        qa, sa = fq.quant_act(x, mode)
+        qw, sw = fq.quant_weight(w, mode)
+        qh = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
+        sh = torch.empty(fq.act_scale_shape(M, N // 2), dtype=torch.float32, device=dev)
+        fn = lambda: fq.gemm_swiglu_quant(qa, sa, qw, sw, mode, qh=qh, sh=sh)  # noqa: E731
+        work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
+    elif kind == "moe_swiglu":
+        moe = wl.moe_layer(seed=0, device=dev)
+        x, w = moe["x_" + what], moe["w_" + what]
+        E, N, K = w.shape
+        R = x.shape[0]
+        qa, sa = fq.quant_act(x, mode)
+        qw, sw = fq.quant_weight(w.reshape(E * N, K), mode)
+        qw, sw = qw.view(E, N, K), sw.view(E, N // 128, K // 128)
+        off = moe["offsets"].to(torch.int32).to(dev)
+        qh = torch.empty((R, N // 2), dtype=torch.uint8, device=dev)
+        sh = torch.empty(fq.act_scale_shape(R, N // 2), dtype=torch.float32, device=dev)
+        fn = lambda: fq.grouped_gemm_swiglu_quant(qa, sa, qw, sw, off, mode, qh=qh, sh=sh)  # noqa: E731
+        # bytes: A codes + scales, W codes + scales, H codes + scales
+        work = (R * K + 4 * R * (K // 128) + E * N * K + 4 * E * (N // 128) * (K // 128) + R * N // 2
+                + 4 * R * (N // 256)) / 1e9
+        unit = "GB/s"
+        print(json.dumps({"case": args.case, "flops": 2.0 * R * N * K}))
+    elif kind == "quant_act_t":
+        K = int(what)
+        x = wl.activations(M, K, seed=1, device=dev)
+        qt = torch.empty((K, M), dtype=torch.uint8, device=dev)
+        st = torch.empty((fq.ceil_div(M, 128), K), dtype=torch.float32, device=dev)
+        fn = lambda: fq.quant_act_t(x, mode, qt=qt, st=st)  # noqa: E731
+        work, unit = quant_act_bytes(M, K) / 1e9, "GB/s"
+    elif kind == "transpose_weight":
+        N, K = wl.LLAMA8B_SHAPES[what]
+        q, sw = fq.quant_weight(wl.weights(N, K, seed=2, device=dev), mode)
+        qt = torch.empty((K, N), dtype=torch.uint8, device=dev)
+        swt = torch.empty((sw.shape[1], sw.shape[0]), dtype=torch.float32, device=dev)
+        fn = lambda: fq.transpose_weight(q, sw, qt=qt, swt=swt)  # noqa: E731
+        work, unit = 2.0 * N * K / 1e9, "GB/s"
+    elif kind == "dgrad":
+        # dX [M, K] = dY [M, N] . W [N, K] through W^T's codes
+        N, K = wl.LLAMA8B_SHAPES[what]
+        dy = wl.activations(M, N, seed=1, device=dev)
+        q_dy, s_dy = fq.quant_act(dy, mode)
+        qwt, swt = fq.transpose_weight(*fq.quant_weight(wl.weights(N, K, seed=2, device=dev), mode))
+        dx = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.gemm_dgrad(q_dy, s_dy, qwt, swt, mode, out=dx)  # noqa: E731
+        work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
+    elif kind == "wgrad":
+        # dW [N, K] = dY^T X over M tokens
+        N, K = wl.LLAMA8B_SHAPES[what]
+        qa, sa = fq.quant_act_t(wl.activations(M, N, seed=1, device=dev), mode)
+        qb, sb = fq.quant_act_t(wl.activations(M, K, seed=2, device=dev), mode)
+        dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.gemm_wgrad(qa, sa, qb, sb, M, mode, out=dw)  # noqa: E731
+        work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
+    elif kind == "adamw_recal":
+        # AdamW on fp32 master weights + moments of the four Llama-8B-shaped
+        # linears, fused with the bf16 copy and the 128x128 recalibration
+        tensors = []
+        nbytes = 0
+        for i, (N, K) in enumerate(wl.LLAMA8B_SHAPES.values()):
+            g = torch.Generator(device=dev).manual_seed(300 + i)
+            p = torch.randn((N, K), generator=g, device=dev) * 0.02
+            gr = torch.randn((N, K), generator=g, device=dev) * 1e-3
+            m = torch.randn((N, K), generator=g, device=dev) * 1e-4
+            v = torch.rand((N, K), generator=g, device=dev) * 1e-6
+            w = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+            q = torch.empty((N, K), dtype=torch.uint8, device=dev)
+            s_ = torch.empty(((N + 127) // 128, (K + 127) // 128), dtype=torch.float32, device=dev)
+            tensors.append((p, gr, m, v, w, q, s_))
+            # read p, g, m, v; write p, m, v, w, q, scales
+            nbytes += N * K * (16 + 12 + 2 + 1) + 4 * ((N + 127) // 128) * ((K + 127) // 128)
+        fn = lambda: fq.adamw_recalibrate(tensors, lr=1e-5, beta1=0.9, beta2=0.95, eps=1e-8,  # noqa: E731
+                                          weight_decay=0.1, step=100, mode=mode)
+        work, unit = nbytes / 1e9, "GB/s"
     elif kind == "quant_act":
         K = int(what)
         x = wl.activations(M, K, seed=1, device=dev)
@@ -555,6 +638,8 @@ def main():
     ap.add_argument("--graph", action="store_true", help="--case: time a CUDA graph of --steps calls")
     ap.add_argument("--native", action="store_true", help="--case gemm with --pow2: native block-scaled MMA")
     ap.add_argument("--pair", action="store_true", help="--case gemm: the CTA-pair promotion kernel")
+    ap.add_argument("--pair128", action="store_true",
+                    help="--case gemm: the CTA-pair promotion kernel with 256x128 tiles")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)

@@ -23,6 +23,7 @@ GEMM_AUTO = 0
 GEMM_PROMOTE = 1
 GEMM_NATIVE_POW2 = 2
 GEMM_PROMOTE_PAIR = 3
+GEMM_PROMOTE_PAIR_N128 = 4
 GEMM_SELFTEST_TIMEOUT = 99
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -46,6 +47,17 @@ class WeightDesc(ctypes.Structure):
                 ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("ldw", ctypes.c_int64), ("ldq", ctypes.c_int64)]
 
 
+class AdamWDesc(ctypes.Structure):
+    _fields_ = [("param", ctypes.c_void_p), ("grad", ctypes.c_void_p), ("exp_avg", ctypes.c_void_p),
+                ("exp_avg_sq", ctypes.c_void_p), ("w", ctypes.c_void_p), ("q", ctypes.c_void_p),
+                ("s", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
+class AdamWConfig(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int64)]
+
+
 # name -> (restype, argtypes); the full list of the C ABI's entry points.
 P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
 SIGNATURES = {
@@ -63,6 +75,13 @@ SIGNATURES = {
     "fp8bq_gemm_decode": (I32, [P, I64, P, I64, P, P, I64, I64, I64, I64, I32, P, SZ, P]),
     "fp8bq_gemm_decode_noalloc": (I32, [P, I64, P, I64, P, P, I64, I64, I64, I64, I32, P]),
     "fp8bq_grouped_gemm": (I32, [P, I64, P, I64, P, P, P, I32, I64, I64, I64, P, I64, I32, P]),
+    "fp8bq_quant_act_t": (I32, [P, I64, I64, I64, P, I64, P, I64, I32, P]),
+    "fp8bq_transpose_weight": (I32, [P, I64, I64, I64, P, P, I64, P, P]),
+    "fp8bq_gemm_wgrad": (I32, [P, I64, P, I64, P, I64, P, I64, P, I64, I64, I64, I64, I32, P]),
+    "fp8bq_adamw_recalibrate": (I32, [ctypes.POINTER(AdamWDesc), I32, ctypes.POINTER(AdamWConfig), I32, P]),
+    "fp8bq_gemm_swiglu_quant": (I32, [P, I64, P, I64, P, I64, P, P, I64, P, I64, P, I64, I64, I64, I64, I32, P]),
+    "fp8bq_grouped_gemm_swiglu_quant": (I32, [P, I64, P, I64, P, P, P, I32, I64, I64, I64, P, I64, P, I64, P, I64,
+                                              I32, P]),
 }
 
 _lib = None
@@ -156,6 +175,67 @@ def recalibrate(tensors, mode=SCALE_POW2, stream=None):
     _check(lib().fp8bq_recalibrate(arr, len(tensors), mode, _stream(stream)), "fp8bq_recalibrate")
 
 
+def quant_act_t(x, mode=SCALE_FP32, qt=None, st=None, stream=None):
+    """Token-axis 1x128 quantization of bf16 x [M, K] with transposed output ->
+    (codes of x^T uint8 [K, ldqt>=M], scales fp32 [ceil(M/128), ldst>=K])."""
+    M, K = x.shape
+    if qt is None:
+        qt = torch.empty((K, ceil_div(max(M, 1), 16) * 16), dtype=torch.uint8, device=x.device)
+    if st is None:
+        st = torch.empty((ceil_div(M, 128), ceil_div(max(K, 1), 4) * 4), dtype=torch.float32, device=x.device)
+    _check(lib().fp8bq_quant_act_t(_ptr(x), M, K, _ld(x), _ptr(qt), _ld(qt), _ptr(st), st.stride(0), mode,
+                                   _stream(stream)), "fp8bq_quant_act_t")
+    return qt, st
+
+
+def transpose_weight(q, sw, qt=None, swt=None, stream=None):
+    """Codes and tile scales of W^T from those of W [N, K] (no requantization)."""
+    N, K = q.shape
+    if qt is None:
+        qt = torch.empty((K, N), dtype=torch.uint8, device=q.device)
+    if swt is None:
+        swt = torch.empty((sw.shape[1], sw.shape[0]), dtype=torch.float32, device=q.device)
+    _check(lib().fp8bq_transpose_weight(_ptr(q), N, K, _ld(q), _ptr(sw), _ptr(qt), _ld(qt), _ptr(swt),
+                                        _stream(stream)), "fp8bq_transpose_weight")
+    return qt, swt
+
+
+def gemm_dgrad(q_dy, s_dy, qwt, swt, mode=SCALE_FP32, out=None, stream=None):
+    """dX = dY . W from dY's 1x128 codes and W^T's codes (transpose_weight)."""
+    return gemm(q_dy, s_dy, qwt, swt, mode, out=out, stream=stream)
+
+
+def gemm_wgrad(qa, sa, qb, sb, M, mode=SCALE_FP32, out=None, stream=None):
+    """dW [N, K] = dY^T X from the token-axis codes of dY^T (qa [N, >=M], sa) and
+    X^T (qb [K, >=M], sb); M = tokens."""
+    N, K = qa.shape[0], qb.shape[0]
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device=qa.device)
+    _check(lib().fp8bq_gemm_wgrad(_ptr(qa), _ld(qa), _ptr(sa), sa.stride(0), _ptr(qb), _ld(qb), _ptr(sb),
+                                  sb.stride(0), _ptr(out), _ld(out), N, K, M, mode, _stream(stream)),
+           "fp8bq_gemm_wgrad")
+    return out
+
+
+def adamw_recalibrate(tensors, lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=1, mode=SCALE_POW2,
+                      stream=None):
+    """One AdamW step on fp32 master weights fused with their 128x128 recalibration.
+
+    tensors: [(param, grad, exp_avg, exp_avg_sq, w_bf16_or_None, q, s), ...], all
+    dense [N, K] (s [ceil(N/128), ceil(K/128)]); updated in place."""
+    arr = (AdamWDesc * len(tensors))()
+    for i, (p, g, m, v, w, q, s) in enumerate(tensors):
+        N, K = p.shape
+        for t in (p, g, m, v, q) + ((w,) if w is not None else ()):
+            if t.shape != (N, K) or not t.is_contiguous():
+                raise ValueError("dense [N, K] tensors expected")
+        arr[i] = AdamWDesc(p.data_ptr(), g.data_ptr(), m.data_ptr(), v.data_ptr(),
+                           w.data_ptr() if w is not None else None, q.data_ptr(), s.data_ptr(), N, K)
+    cfg = AdamWConfig(lr, beta1, beta2, eps, weight_decay, step)
+    _check(lib().fp8bq_adamw_recalibrate(arr, len(tensors), ctypes.byref(cfg), mode, _stream(stream)),
+           "fp8bq_adamw_recalibrate")
+
+
 def gemm(qa, sa, qw, sw, mode=SCALE_FP32, out=None, variant=GEMM_AUTO, stream=None):
     """Block-scaled FP8 GEMM: bf16 [M, N] = deq(qa) . deq(qw)^T."""
     M, K = qa.shape
@@ -194,6 +274,59 @@ def grouped_gemm(qa, sa, qw, sw, offsets, mode=SCALE_FP32, out=None, stream=None
     _check(lib().fp8bq_grouped_gemm(_ptr(qa), _ld(qa), _ptr(sa), sa.stride(0), _ptr(qw), _ptr(sw), _ptr(offsets),
                                     E, R, N, K, _ptr(out), _ld(out), mode, _stream(stream)), "fp8bq_grouped_gemm")
     return out
+
+
+def interleave_gate_up(w_gate, w_up):
+    """Storage layout of a gated feed-forward block's gate+up weight for
+    gemm_swiglu_quant: [..., 2I, K] with 128-row blocks alternating gate block j,
+    up block j.  A one-time layout step when the weights are created; the
+    recalibration then quantizes the interleaved tensor in place every step."""
+    if w_gate.shape != w_up.shape or w_gate.shape[-2] % 128:
+        raise ValueError("gate and up must have the same shape with a multiple of 128 rows")
+    *lead, I, K = w_gate.shape
+    g = w_gate.reshape(*lead, I // 128, 1, 128, K)
+    u = w_up.reshape(*lead, I // 128, 1, 128, K)
+    return torch.cat([g, u], dim=-3).reshape(*lead, 2 * I, K).contiguous()
+
+
+def gemm_swiglu_quant(qa, sa, qw, sw, mode=SCALE_FP32, qh=None, sh=None, h=None, want_h=False, stream=None):
+    """Gate+up GEMM with H = bf16(silu(g) * u) and its 1x128 quantization in the epilogue.
+
+    qw/sw: the interleaved gate+up weight [2I, K] (see interleave_gate_up).
+    Returns (qh uint8 [M, I], sh fp32 [I/128, ldsh], h bf16 [M, I] or None)."""
+    M, K = qa.shape
+    I = qw.shape[0] // 2
+    if qh is None:
+        qh = torch.empty((M, I), dtype=torch.uint8, device=qa.device)
+    if sh is None:
+        sh = torch.empty(act_scale_shape(M, I), dtype=torch.float32, device=qa.device)
+    if h is None and want_h:
+        h = torch.empty((M, I), dtype=torch.bfloat16, device=qa.device)
+    _check(lib().fp8bq_gemm_swiglu_quant(_ptr(qa), _ld(qa), _ptr(sa), sa.stride(0), _ptr(qw), _ld(qw), _ptr(sw),
+                                         _ptr(qh), _ld(qh), _ptr(sh), sh.stride(0), _ptr(h),
+                                         _ld(h) if h is not None else 0, M, I, K, mode, _stream(stream)),
+           "fp8bq_gemm_swiglu_quant")
+    return qh, sh, h
+
+
+def grouped_gemm_swiglu_quant(qa, sa, qw, sw, offsets, mode=SCALE_FP32, qh=None, sh=None, h=None, want_h=False,
+                              stream=None):
+    """Grouped (mixture-of-experts) form of gemm_swiglu_quant; qw [E, 2I, K] interleaved per expert."""
+    R, K = qa.shape
+    E, N2, _ = qw.shape
+    I = N2 // 2
+    if qh is None:
+        qh = torch.empty((R, I), dtype=torch.uint8, device=qa.device)
+    if sh is None:
+        sh = torch.empty(act_scale_shape(R, I), dtype=torch.float32, device=qa.device)
+    if h is None and want_h:
+        h = torch.empty((R, I), dtype=torch.bfloat16, device=qa.device)
+    _check(lib().fp8bq_grouped_gemm_swiglu_quant(_ptr(qa), _ld(qa), _ptr(sa), sa.stride(0), _ptr(qw), _ptr(sw),
+                                                 _ptr(offsets), E, R, I, K, _ptr(qh), _ld(qh), _ptr(sh),
+                                                 sh.stride(0), _ptr(h), _ld(h) if h is not None else 0, mode,
+                                                 _stream(stream)),
+           "fp8bq_grouped_gemm_swiglu_quant")
+    return qh, sh, h
 
 
 def device_error():

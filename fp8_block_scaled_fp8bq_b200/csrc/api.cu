@@ -122,13 +122,9 @@ bool bad_mode(int mode) { return mode != FP8BQ_SCALE_FP32 && mode != FP8BQ_SCALE
 
 constexpr int64_t kMaxDim = (int64_t)1 << 31;
 
-fp8bq_status check_gemm_operands(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
-                                 int64_t ldw, const float *sw, const void *y, int64_t ldy, int64_t M, int64_t N,
-                                 int64_t K, int mode) {
-  if (M < 0 || N < 0 || K < 0 || bad_mode(mode)) return FP8BQ_ERR_INVALID_ARG;
-  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
-  if (M == 0 || N == 0) return FP8BQ_OK;
-  if (y == nullptr || ldy < N || !aligned(y, 16) || ldy % 8 != 0) return FP8BQ_ERR_INVALID_ARG;
+// The GEMM's inputs (M, N > 0): codes and scales of both operands.
+fp8bq_status check_gemm_inputs(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                               int64_t ldw, const float *sw, int64_t M, int64_t K) {
   if (K == 0) return FP8BQ_OK;
   if (K % 128 != 0) return FP8BQ_ERR_UNSUPPORTED;
   if (!qa || !sa || !qw || !sw) return FP8BQ_ERR_INVALID_ARG;
@@ -136,6 +132,33 @@ fp8bq_status check_gemm_operands(const uint8_t *qa, int64_t lda, const float *sa
   if (!aligned(qa, 16) || !aligned(qw, 16) || lda % 16 != 0 || ldw % 16 != 0) return FP8BQ_ERR_INVALID_ARG;
   if (!aligned(sa, 16) || !aligned(sw, 4) || ldsa % 4 != 0) return FP8BQ_ERR_INVALID_ARG;
   return FP8BQ_OK;
+}
+
+fp8bq_status check_gemm_operands(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                                 int64_t ldw, const float *sw, const void *y, int64_t ldy, int64_t M, int64_t N,
+                                 int64_t K, int mode) {
+  if (M < 0 || N < 0 || K < 0 || bad_mode(mode)) return FP8BQ_ERR_INVALID_ARG;
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return FP8BQ_OK;
+  if (y == nullptr || ldy < N || !aligned(y, 16) || ldy % 8 != 0) return FP8BQ_ERR_INVALID_ARG;
+  return check_gemm_inputs(qa, lda, sa, ldsa, qw, ldw, sw, M, K);
+}
+
+// The fused gate+up epilogue's operands: W_gu has 2I rows; the outputs are the
+// H codes [M][ldqh], the H scales [I/128][ldsh] (the activation-scale layout the
+// next GEMM reads) and the optional bf16 H [M][ldh].
+fp8bq_status check_swiglu_operands(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                                   int64_t ldw, const float *sw, const uint8_t *qh, int64_t ldqh, const float *sh,
+                                   int64_t ldsh, const void *h, int64_t ldh, int64_t M, int64_t I, int64_t K,
+                                   int mode) {
+  if (M < 0 || I < 0 || K < 0 || bad_mode(mode)) return FP8BQ_ERR_INVALID_ARG;
+  if (M >= kMaxDim || 2 * I >= kMaxDim || K >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
+  if (M == 0 || I == 0) return FP8BQ_OK;
+  if (I % 128 != 0) return FP8BQ_ERR_UNSUPPORTED;
+  if (!qh || ldqh < I || ldqh % 16 != 0 || !aligned(qh, 16)) return FP8BQ_ERR_INVALID_ARG;
+  if (!sh || ldsh < M || ldsh % 4 != 0 || !aligned(sh, 16)) return FP8BQ_ERR_INVALID_ARG;
+  if (h != nullptr && (ldh < I || ldh % 8 != 0 || !aligned(h, 16))) return FP8BQ_ERR_INVALID_ARG;
+  return check_gemm_inputs(qa, lda, sa, ldsa, qw, ldw, sw, M, K);
 }
 
 }  // namespace
@@ -162,8 +185,9 @@ fp8bq_status fp8bq_get_device_error(uint64_t *code) {
   unsigned long long v = 0, w = 0;
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-  cudaError_t (*takers[])(unsigned long long *) = {take_device_error_gemm, take_device_error_decode, take_device_error_native,
-                                                       take_device_error_pair};
+  cudaError_t (*takers[])(unsigned long long *) = {take_device_error_gemm, take_device_error_decode,
+                                                    take_device_error_native, take_device_error_pair,
+                                                    take_device_error_swiglu, take_device_error_wgrad};
   for (auto take : takers) {
     e = take(&w);
     if (e != cudaSuccess) return cuda_fail(e, "read device error word");
@@ -229,7 +253,7 @@ fp8bq_status fp8bq_recalibrate(const fp8bq_weight_desc *descs, int n, int mode, 
 fp8bq_status fp8bq_gemm_ex(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
                            int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                            int mode, int variant, void *stream) {
-  if ((variant < FP8BQ_GEMM_AUTO || variant > FP8BQ_GEMM_PROMOTE_PAIR) && variant != FP8BQ_GEMM_SELFTEST_TIMEOUT)
+  if ((variant < FP8BQ_GEMM_AUTO || variant > FP8BQ_GEMM_PROMOTE_PAIR_N128) && variant != FP8BQ_GEMM_SELFTEST_TIMEOUT)
     return FP8BQ_ERR_INVALID_ARG;
   if (variant == FP8BQ_GEMM_NATIVE_POW2 && mode != FP8BQ_SCALE_POW2) return FP8BQ_ERR_INVALID_ARG;
   fp8bq_status st = check_gemm_operands(qa, lda, sa, ldsa, qw, ldw, sw, y, ldy, M, N, K, mode);
@@ -270,6 +294,95 @@ fp8bq_status fp8bq_grouped_gemm(const uint8_t *qa, int64_t lda, const float *sa,
   if (st != FP8BQ_OK || total_rows == 0 || N == 0) return st;
   return launch_grouped_gemm(qa, lda, sa, ldsa, qw, sw, offsets, E, total_rows, N, K, y, ldy,
                              static_cast<cudaStream_t>(stream));
+}
+
+fp8bq_status fp8bq_gemm_swiglu_quant(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa,
+                                     const uint8_t *qw, int64_t ldw, const float *sw, uint8_t *qh, int64_t ldqh,
+                                     float *sh, int64_t ldsh, void *h, int64_t ldh, int64_t M, int64_t I, int64_t K,
+                                     int mode, void *stream) {
+  fp8bq_status st = check_swiglu_operands(qa, lda, sa, ldsa, qw, ldw, sw, qh, ldqh, sh, ldsh, h, ldh, M, I, K, mode);
+  if (st != FP8BQ_OK || M == 0 || I == 0) return st;
+  return launch_gemm_swiglu(qa, lda, sa, ldsa, qw, ldw, sw, qh, ldqh, sh, ldsh, h, ldh, M, I, K, mode,
+                            static_cast<cudaStream_t>(stream));
+}
+
+fp8bq_status fp8bq_grouped_gemm_swiglu_quant(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa,
+                                             const uint8_t *qw, const float *sw, const int32_t *offsets, int E,
+                                             int64_t total_rows, int64_t I, int64_t K, uint8_t *qh, int64_t ldqh,
+                                             float *sh, int64_t ldsh, void *h, int64_t ldh, int mode, void *stream) {
+  if (E < 1 || E > kMaxExperts || total_rows < 0) return E > kMaxExperts ? FP8BQ_ERR_UNSUPPORTED : FP8BQ_ERR_INVALID_ARG;
+  if (!offsets || !aligned(offsets, 4)) return FP8BQ_ERR_INVALID_ARG;
+  if ((int64_t)E * 2 * I >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
+  fp8bq_status st =
+      check_swiglu_operands(qa, lda, sa, ldsa, qw, K, sw, qh, ldqh, sh, ldsh, h, ldh, total_rows, I, K, mode);
+  if (st != FP8BQ_OK || total_rows == 0 || I == 0) return st;
+  return launch_grouped_gemm_swiglu(qa, lda, sa, ldsa, qw, sw, offsets, E, total_rows, I, K, qh, ldqh, sh, ldsh, h,
+                                    ldh, mode, static_cast<cudaStream_t>(stream));
+}
+
+fp8bq_status fp8bq_quant_act_t(const void *x, int64_t M, int64_t K, int64_t ldx, uint8_t *qt, int64_t ldqt, float *st,
+                               int64_t ldst, int mode, void *stream) {
+  if (M < 0 || K < 0 || bad_mode(mode)) return FP8BQ_ERR_INVALID_ARG;
+  if (M >= kMaxDim || K >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
+  if (M == 0 || K == 0) return FP8BQ_OK;
+  if (K % 8 != 0) return FP8BQ_ERR_UNSUPPORTED;
+  if (!x || !qt || !st) return FP8BQ_ERR_INVALID_ARG;
+  if (ldx < K || ldx % 8 != 0 || !aligned(x, 16)) return FP8BQ_ERR_INVALID_ARG;
+  if (ldqt < M || ldqt % 16 != 0 || !aligned(qt, 16)) return FP8BQ_ERR_INVALID_ARG;
+  if (ldst < K || ldst % 4 != 0 || !aligned(st, 16)) return FP8BQ_ERR_INVALID_ARG;
+  return launch_quant_act_t(x, M, K, ldx, qt, ldqt, st, ldst, mode, static_cast<cudaStream_t>(stream));
+}
+
+fp8bq_status fp8bq_transpose_weight(const uint8_t *q, int64_t N, int64_t K, int64_t ldq, const float *sw, uint8_t *qt,
+                                    int64_t ldqt, float *swt, void *stream) {
+  if (N < 0 || K < 0) return FP8BQ_ERR_INVALID_ARG;
+  if (N >= kMaxDim || K >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
+  if (N == 0 || K == 0) return FP8BQ_OK;
+  if (N % 16 != 0 || K % 16 != 0) return FP8BQ_ERR_UNSUPPORTED;
+  if (!q || !sw || !qt || !swt) return FP8BQ_ERR_INVALID_ARG;
+  if (ldq < K || ldq % 16 != 0 || !aligned(q, 16) || ldqt < N || ldqt % 16 != 0 || !aligned(qt, 16))
+    return FP8BQ_ERR_INVALID_ARG;
+  if (!aligned(sw, 4) || !aligned(swt, 4)) return FP8BQ_ERR_INVALID_ARG;
+  return launch_transpose_weight(q, N, K, ldq, sw, qt, ldqt, swt, static_cast<cudaStream_t>(stream));
+}
+
+fp8bq_status fp8bq_gemm_wgrad(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qb,
+                              int64_t ldb, const float *sb, int64_t ldsb, void *y, int64_t ldy, int64_t N, int64_t K,
+                              int64_t M, int mode, void *stream) {
+  if (N < 0 || K < 0 || M < 0 || bad_mode(mode)) return FP8BQ_ERR_INVALID_ARG;
+  if (N >= kMaxDim || K >= kMaxDim || M >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
+  if (N == 0 || K == 0) return FP8BQ_OK;
+  if (y == nullptr || ldy < K || !aligned(y, 16) || ldy % 8 != 0) return FP8BQ_ERR_INVALID_ARG;
+  if (M == 0) return launch_gemm_wgrad(qa, lda, sa, ldsa, qb, ldb, sb, ldsb, y, ldy, N, K, M, static_cast<cudaStream_t>(stream));
+  if (M % 128 != 0 || K % 4 != 0) return FP8BQ_ERR_UNSUPPORTED;
+  if (!qa || !sa || !qb || !sb) return FP8BQ_ERR_INVALID_ARG;
+  if (lda < M || ldb < M || lda % 16 != 0 || ldb % 16 != 0 || !aligned(qa, 16) || !aligned(qb, 16))
+    return FP8BQ_ERR_INVALID_ARG;
+  if (ldsa < N || ldsa % 4 != 0 || !aligned(sa, 16)) return FP8BQ_ERR_INVALID_ARG;
+  if (ldsb < K || ldsb % 4 != 0 || !aligned(sb, 16)) return FP8BQ_ERR_INVALID_ARG;
+  return launch_gemm_wgrad(qa, lda, sa, ldsa, qb, ldb, sb, ldsb, y, ldy, N, K, M, static_cast<cudaStream_t>(stream));
+}
+
+fp8bq_status fp8bq_adamw_recalibrate(const fp8bq_adamw_desc *descs, int n, const fp8bq_adamw_config *cfg, int mode,
+                                     void *stream) {
+  if (n < 0 || bad_mode(mode) || cfg == nullptr) return FP8BQ_ERR_INVALID_ARG;
+  if (!(cfg->beta1 >= 0.f && cfg->beta1 < 1.f && cfg->beta2 >= 0.f && cfg->beta2 < 1.f && cfg->eps >= 0.f) ||
+      cfg->step < 1)
+    return FP8BQ_ERR_INVALID_ARG;
+  if (n == 0) return FP8BQ_OK;
+  if (!descs) return FP8BQ_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    const fp8bq_adamw_desc &d = descs[i];
+    if (d.N < 0 || d.K < 0) return FP8BQ_ERR_INVALID_ARG;
+    if (d.N >= kMaxDim || d.K >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
+    if (d.N == 0 || d.K == 0) continue;
+    if (d.K % 4 != 0) return FP8BQ_ERR_UNSUPPORTED;
+    if (!d.param || !d.grad || !d.exp_avg || !d.exp_avg_sq || !d.q || !d.s) return FP8BQ_ERR_INVALID_ARG;
+    if (!aligned(d.param, 16) || !aligned(d.grad, 16) || !aligned(d.exp_avg, 16) || !aligned(d.exp_avg_sq, 16) ||
+        !aligned(d.w, 8) || !aligned(d.q, 4) || !aligned(d.s, 4))
+      return FP8BQ_ERR_INVALID_ARG;
+  }
+  return launch_adamw_recalibrate(descs, n, cfg, mode, static_cast<cudaStream_t>(stream));
 }
 
 fp8bq_status fp8bq_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw, int64_t ldw,

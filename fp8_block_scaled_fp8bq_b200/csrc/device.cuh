@@ -37,6 +37,7 @@ enum WaitSite : unsigned {
   kSiteMmaTmemEmpty = 3,
   kSiteEpiTmemFull = 4,
   kSiteDrain = 5,
+  kSitePairExchange = 6,
 };
 
 __device__ __forceinline__ void record_error(unsigned where) {

@@ -39,13 +39,8 @@ namespace {
 
 constexpr int CBM = 128;                 // A rows per CTA
 constexpr int PBM = 2 * CBM;             // rows per pair tile
-constexpr int PBN = 256;                 // columns per tile
-constexpr int CBN = PBN / 2;             // B rows per CTA
 constexpr int BK = 128;
-constexpr int kStages = 6;
 constexpr int kABytes = CBM * BK;
-constexpr int kBBytes = CBN * BK;
-constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kEpiWarps = 8;
 constexpr int kEpiBufBytes = 32 * 128;   // 32 rows x 64 bf16, 128-byte swizzle
 constexpr int kThreads = 384;
@@ -53,9 +48,23 @@ constexpr int kLaunchRegs = 168;
 constexpr int kLowRegs = 56;
 constexpr int kHighRegs = 224;
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split");
-constexpr int kTmemCols = 2 * PBN;
-constexpr int kSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiBufBytes + 256 + 1024;
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+constexpr int kTmemCols = 512;
+
+// Tile shapes: PBN = 256 (two 256-column TMEM buffers) or PBN = 128 (four
+// 128-column buffers, so the MMA can run three K-blocks ahead of the
+// promotion warps instead of one).
+template <int PBN>
+struct PairCfg {
+  static constexpr int CBN = PBN / 2;                 // B rows per CTA
+  static constexpr int kBBytes = CBN * BK;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = PBN == 256 ? 6 : 8;
+  static constexpr int kBufs = kTmemCols / PBN;       // TMEM accumulator buffers
+  static constexpr int kWarpCols = PBN / 2;           // columns per epilogue warp
+  static constexpr int kSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiBufBytes + 256 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(2 * kStages + 2 * kBufs + 1 <= 28, "barrier area");
+};
 
 struct PairArgs {
   const float *sa;
@@ -81,9 +90,13 @@ __device__ __forceinline__ void settle() {
   for (int i = 0; i < 64; ++i) __nanosleep(1000);
 }
 
+template <int PBN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmY, const PairArgs args) {
+  using C = PairCfg<PBN>;
+  constexpr int CBN = C::CBN, kBBytes = C::kBBytes, kStageBytes = C::kStageBytes, kStages = C::kStages;
+  constexpr int kBufs = C::kBufs, kWarpCols = C::kWarpCols;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = base;
@@ -93,8 +106,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *full = bars;
   uint64_t *empty = full + kStages;
   uint64_t *tfull = empty + kStages;
-  uint64_t *tempty = tfull + 2;
-  uint64_t *drain = tempty + 2;
+  uint64_t *tempty = tfull + kBufs;
+  uint64_t *drain = tempty + kBufs;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -109,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kBufs; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 2 * kEpiWarps);
     }
@@ -186,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             stage = 0;
             phase ^= 1;
           }
-          if (++buf == 2) {
+          if (++buf == kBufs) {
             buf = 0;
             bphase ^= 1;
           }
@@ -207,6 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quarter * 32 + lane;
     uint8_t *ebuf = sEpi + ew * kEpiBufBytes;
     const uint32_t tempty0 = mapa_shared(smem_addr(&tempty[0]), 0);
+    constexpr int kPairs = kWarpCols / 2;  // accumulator pairs per thread
     int buf = 0;
     uint32_t bphase = 0;
     for (int t = pair; t < total; t += npairs) {
@@ -214,13 +228,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       pair_tile(t, args, pm, nb);
       const int r0 = pm * PBM + (int)rank * CBM;  // this CTA's first row
       const int m = r0 + row;
-      const int wn = nb * 2 + half;
+      const int wn = PBN == 256 ? nb * 2 + half : nb;  // the warp's weight block
       const bool live = m < args.M && wn < args.NB;
       const float *sa_p = args.sa + m;
       const float *sw_p = args.sw + (int64_t)wn * KB;
-      float2 acc[64];
+      float2 acc[kPairs];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.f, 0.f);
+      for (int j = 0; j < kPairs; ++j) acc[j] = make_float2(0.f, 0.f);
       float a0 = 0.f, w0 = 0.f, a1 = 0.f, w1 = 0.f;
       if (live) {
         a0 = __ldg(sa_p);
@@ -246,14 +260,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * PBN + half * 128);
+        const uint32_t taddr =
+            tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * PBN + half * kWarpCols);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < kWarpCols / 64; ++c) {
           uint32_t r[64];
           tmem_ld_32x32b_x32(taddr + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
           tmem_ld_32x32b_x32(taddr + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_ld_wait();
-          if (c == 1) {  // this warp's part of the buffer has been read
+          if (c == kWarpCols / 64 - 1) {  // this warp's part of the buffer has been read
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -266,14 +281,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc[32 * c + j] =
                 __ffma2_rn(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])), sc2, acc[32 * c + j]);
         }
-        if (++buf == 2) {
+        if (++buf == kBufs) {
           buf = 0;
           bphase ^= 1;
         }
       }
       if (!ok) break;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < kWarpCols / 64; ++c) {
         if (lane == 0) bulk_wait_group_read0();
         __syncwarp();
         uint8_t *rowp = ebuf + lane * 128;
@@ -290,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          const int x = nb * PBN + half * 128 + c * 64;
+          const int x = nb * PBN + half * kWarpCols + c * 64;
           const int y = r0 + quarter * 32;
           if (x < args.N && y < args.M) {
             tma_store_2d(&tmY, ebuf, x, y);
@@ -312,26 +327,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-int g_pready[64] = {0};
-int g_pmax_clusters[64] = {0};
+int g_pready[2][64] = {};         // [tile shape][device]: 0 unknown, 1 ready, -1 refused
+int g_pmax_clusters[2][64] = {};
 
-}  // namespace
-
-bool pair_gemm_available() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  if (g_pready[dev] == 0) {
+template <int PBN>
+bool pair_ready(int dev) {
+  constexpr int si = PBN == 256 ? 0 : 1;
+  if (g_pready[si][dev] == 0) {
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, gemm_pair_kernel) != cudaSuccess || fa.numRegs != kLaunchRegs ||
-        cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-            cudaSuccess) {
-      g_pready[dev] = -1;
+    if (cudaFuncGetAttributes(&fa, gemm_pair_kernel<PBN>) != cudaSuccess || fa.numRegs != kLaunchRegs ||
+        cudaFuncSetAttribute(gemm_pair_kernel<PBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PairCfg<PBN>::kSmemBytes) != cudaSuccess) {
+      g_pready[si][dev] = -1;
       return false;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 128);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.dynamicSmemBytes = PairCfg<PBN>::kSmemBytes;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
@@ -340,28 +353,29 @@ bool pair_gemm_available() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int nclusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&nclusters, gemm_pair_kernel, &cfg) != cudaSuccess || nclusters < 1) {
+    if (cudaOccupancyMaxActiveClusters(&nclusters, gemm_pair_kernel<PBN>, &cfg) != cudaSuccess || nclusters < 1) {
       cudaGetLastError();
-      g_pready[dev] = -1;
+      g_pready[si][dev] = -1;
       return false;
     }
-    g_pmax_clusters[dev] = nclusters;
-    g_pready[dev] = 1;
+    g_pmax_clusters[si][dev] = nclusters;
+    g_pready[si][dev] = 1;
   }
-  return g_pready[dev] == 1;
+  return g_pready[si][dev] == 1;
 }
 
-cudaError_t take_device_error_pair(unsigned long long *v) { return take_tu_device_error(v); }
-
-fp8bq_status launch_gemm_pair(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
-                              int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                              cudaStream_t stream) {
-  if (!pair_gemm_available()) return FP8BQ_ERR_UNSUPPORTED;
+template <int PBN>
+fp8bq_status launch_pair(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                         int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                         cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || !pair_ready<PBN>(dev))
+    return FP8BQ_ERR_UNSUPPORTED;
   CUtensorMap tA, tB, tY;
   if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qa, (uint64_t)K, (uint64_t)M, (uint64_t)lda, BK, CBM,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, (uint64_t)K, (uint64_t)N, (uint64_t)ldw, BK, CBN,
-                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, (uint64_t)K, (uint64_t)N, (uint64_t)ldw, BK,
+                    PairCfg<PBN>::CBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M, (uint64_t)ldy * 2, 64, 32,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return FP8BQ_ERR_INVALID_ARG;
@@ -376,14 +390,13 @@ fp8bq_status launch_gemm_pair(const uint8_t *qa, int64_t lda, const float *sa, i
   a.num_m = (int32_t)((M + PBM - 1) / PBM);
   a.num_n = (int32_t)((N + PBN - 1) / PBN);
   choose_raster(M, N, K, PBM, PBN, &a.band, &a.n_major);
-  int dev = 0;
-  cudaGetDevice(&dev);
   const int64_t tiles = (int64_t)a.num_m * a.num_n;
-  const int pairs = (int)std::min<int64_t>(tiles, std::min(g_pmax_clusters[dev], num_sms() / 2));
+  const int si = PBN == 256 ? 0 : 1;
+  const int pairs = (int)std::min<int64_t>(tiles, std::min(g_pmax_clusters[si][dev], num_sms() / 2));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = PairCfg<PBN>::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -392,9 +405,26 @@ fp8bq_status launch_gemm_pair(const uint8_t *qa, int64_t lda, const float *sa, i
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, tA, tB, tY, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<PBN>, tA, tB, tY, a);
   if (e != cudaSuccess) return cuda_fail(e, "gemm_pair launch");
   return check_launch("gemm_pair");
+}
+
+}  // namespace
+
+bool pair_gemm_available() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  return pair_ready<256>(dev) && pair_ready<128>(dev);
+}
+
+cudaError_t take_device_error_pair(unsigned long long *v) { return take_tu_device_error(v); }
+
+fp8bq_status launch_gemm_pair(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                              int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                              int tile_n, cudaStream_t stream) {
+  if (tile_n == 128) return launch_pair<128>(qa, lda, sa, ldsa, qw, ldw, sw, y, ldy, M, N, K, stream);
+  return launch_pair<256>(qa, lda, sa, ldsa, qw, ldw, sw, y, ldy, M, N, K, stream);
 }
 
 }  // namespace fp8bq

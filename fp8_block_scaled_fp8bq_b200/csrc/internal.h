@@ -43,6 +43,8 @@ cudaError_t take_device_error_gemm(unsigned long long *v);
 cudaError_t take_device_error_decode(unsigned long long *v);
 cudaError_t take_device_error_native(unsigned long long *v);
 cudaError_t take_device_error_pair(unsigned long long *v);
+cudaError_t take_device_error_swiglu(unsigned long long *v);
+cudaError_t take_device_error_wgrad(unsigned long long *v);
 
 // Launchers (arguments already validated).
 fp8bq_status launch_encode(const float *x, int64_t n, uint8_t *q, cudaStream_t stream);
@@ -55,7 +57,7 @@ fp8bq_status launch_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_
 bool pair_gemm_available();
 fp8bq_status launch_gemm_pair(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
                               int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                              cudaStream_t stream);
+                              int tile_n, cudaStream_t stream);
 fp8bq_status launch_gemm_native(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
                                 int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                                 cudaStream_t stream);
@@ -66,5 +68,21 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
 fp8bq_status launch_grouped_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
                                  const float *sw, const int32_t *offsets, int E, int64_t rows, int64_t N, int64_t K,
                                  void *y, int64_t ldy, cudaStream_t stream);
+fp8bq_status launch_gemm_swiglu(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
+                                int64_t ldw, const float *sw, uint8_t *qh, int64_t ldqh, float *sh, int64_t ldsh,
+                                void *h, int64_t ldh, int64_t M, int64_t I, int64_t K, int mode, cudaStream_t stream);
+fp8bq_status launch_grouped_gemm_swiglu(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa,
+                                        const uint8_t *qw, const float *sw, const int32_t *offsets, int E,
+                                        int64_t rows, int64_t I, int64_t K, uint8_t *qh, int64_t ldqh, float *sh,
+                                        int64_t ldsh, void *h, int64_t ldh, int mode, cudaStream_t stream);
+fp8bq_status launch_adamw_recalibrate(const fp8bq_adamw_desc *descs, int n, const fp8bq_adamw_config *cfg, int mode,
+                                      cudaStream_t stream);
+fp8bq_status launch_quant_act_t(const void *x, int64_t M, int64_t K, int64_t ldx, uint8_t *qt, int64_t ldqt, float *st,
+                                int64_t ldst, int mode, cudaStream_t stream);
+fp8bq_status launch_transpose_weight(const uint8_t *q, int64_t N, int64_t K, int64_t ldq, const float *sw,
+                                     uint8_t *qt, int64_t ldqt, float *swt, cudaStream_t stream);
+fp8bq_status launch_gemm_wgrad(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qb,
+                               int64_t ldb, const float *sb, int64_t ldsb, void *y, int64_t ldy, int64_t N, int64_t K,
+                               int64_t M, cudaStream_t stream);
 
 }  // namespace fp8bq

@@ -186,6 +186,8 @@ typedef enum {
                                      128x256 tile */
     FP8BQ_GEMM_NATIVE_POW2 = 2,   /* native block-scaled MMA (POW2 scales only) */
     FP8BQ_GEMM_PROMOTE_PAIR = 3,  /* FP32 promotion on CTA pairs (paired MMA, 256x256 tiles) */
+    FP8BQ_GEMM_PROMOTE_PAIR_N128 = 4,  /* FP32 promotion on CTA pairs, 256x128 tiles and four
+                                          TMEM accumulator buffers */
     FP8BQ_GEMM_SELFTEST_TIMEOUT = 99  /* failure-detection self-test: the promotion kernel runs
                                          with its TMA producer disabled, so its MMA issuer's
                                          bounded wait runs out (about 1 s); the call returns
@@ -258,6 +260,155 @@ FP8BQ_API fp8bq_status fp8bq_grouped_gemm(const uint8_t *qa, int64_t lda, const 
                                 const int32_t *offsets, int E, int64_t total_rows,
                                 int64_t N, int64_t K, void *y, int64_t ldy,
                                 int mode, void *stream);
+
+/*
+ * Gate+up projection of a gated (SwiGLU) feed-forward block with the
+ * activation and the down projection's input quantization in the GEMM's
+ * epilogue.  "Technical breakthrough" runs the linear layers in FP8 and keeps
+ * non-linear functions in BF16; the Llama 3.1 8B model it names has SwiGLU
+ * feed-forward blocks.  "Real-world performance gains" names the quantization
+ * kernels as an overhead of the FP8 linear layers; this call removes the
+ * separate activation and quantization passes over the [M][I] intermediate.
+ * Computes, for every row m and feature i < I:
+ *   g = bf16(Y[m][gate column of i]),  u = bf16(Y[m][up column of i]),
+ *       with Y = X W_gu^T the block-scaled GEMM of fp8bq_gemm (FP32 promotion);
+ *   H[m][i] = bf16(silu(g) * u),  silu(g) = g / (1 + e^-g)  (FP32 arithmetic,
+ *       one rounding to bf16);
+ *   (qh, sh) = the 1x128 activation quantization of H (fp8bq_quant_act's
+ *       definition, scale mode `mode`).
+ *   qa, sa   activation codes [M][lda] and scales [K/128][ldsa], as fp8bq_gemm.
+ *   qw, sw   W_gu codes [2I][ldw] and scales [2I/128][K/128]: the gate and up
+ *            weights ([I][K] each) with their 128-row blocks interleaved: rows
+ *            [256 j, 256 j + 128) are gate rows [128 j, 128 j + 128) and rows
+ *            [256 j + 128, 256 j + 256) the up rows of the same features.
+ *            (Quantizing W_gu with fp8bq_quant_weight gives the same codes and
+ *            scales as quantizing gate and up separately.)
+ *   qh       E4M3 codes of H [M][ldqh];  sh  fp32 scales [I/128][ldsh] with
+ *            the scale of tile (m, j) at sh[j * ldsh + m] -- the activation
+ *            layout, so (qh, sh) is the down projection's (qa, sa) as is.
+ *   h        optional bf16 H [M][ldh] (NULL: not written).
+ * The scale arguments of the input GEMM may be FP32 or power-of-2 values in
+ * either mode (both run the FP32 promotion); `mode` selects the kind of scale
+ * produced for H.
+ * Requirements: as fp8bq_gemm for the inputs (K % 128 == 0); I % 128 == 0;
+ * ldqh >= I, ldqh % 16 == 0, qh 16-byte aligned; ldsh >= M, ldsh % 4 == 0,
+ * sh 16-byte aligned; h: ldh >= I, ldh % 8 == 0, 16-byte aligned.  K = 0 gives
+ * H = 0 (codes 0, scales 1).  Asynchronous on `stream`; allocates nothing.
+ */
+FP8BQ_API fp8bq_status fp8bq_gemm_swiglu_quant(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa,
+                                               const uint8_t *qw, int64_t ldw, const float *sw,
+                                               uint8_t *qh, int64_t ldqh, float *sh, int64_t ldsh,
+                                               void *h, int64_t ldh, int64_t M, int64_t I, int64_t K,
+                                               int mode, void *stream);
+
+/*
+ * Grouped (mixture-of-experts) form of fp8bq_gemm_swiglu_quant: rows
+ * [offsets[e], offsets[e+1]) use expert e's interleaved gate+up weight.
+ *   qw  E4M3 [E][2I][K], dense, each expert's rows interleaved as above;
+ *   sw  fp32 [E][2I/128][K/128];  offsets as fp8bq_grouped_gemm.
+ *   qh, sh, h over total_rows rows, as fp8bq_gemm_swiglu_quant.
+ * Rows not covered by [offsets[0], offsets[E]) are not written.
+ * Requirements: as fp8bq_gemm_swiglu_quant and fp8bq_grouped_gemm.
+ */
+FP8BQ_API fp8bq_status fp8bq_grouped_gemm_swiglu_quant(const uint8_t *qa, int64_t lda, const float *sa,
+                                                       int64_t ldsa, const uint8_t *qw, const float *sw,
+                                                       const int32_t *offsets, int E, int64_t total_rows,
+                                                       int64_t I, int64_t K, uint8_t *qh, int64_t ldqh, float *sh,
+                                                       int64_t ldsh, void *h, int64_t ldh, int mode,
+                                                       void *stream);
+
+/*
+ * Backward pass of the FP8 linear layer Y = X W^T ("Technical breakthrough":
+ * FP8 in training as well as generation; 1x128 tiles for activations, 128x128
+ * for weights).  With dY [M][N] the output gradient:
+ *   dX = dY W   : fp8bq_gemm(codes/scales of dY from fp8bq_quant_act,
+ *                            W^T codes/scales from fp8bq_transpose_weight)
+ *   dW = dY^T X : fp8bq_gemm_wgrad(dY^T and X^T codes/scales from
+ *                            fp8bq_quant_act_t)
+ */
+
+/*
+ * 1x128 quantization along the token axis with transposed output: tile
+ * (k, mb) is X[128 mb .. 128 mb + 127][k] (the last one may be shorter).
+ *   x    bf16 [M][ldx]
+ *   qt   E4M3 codes of X^T [K][ldqt] (token-contiguous)
+ *   st   fp32 scales [ceil(M/128)][ldst], tile (k, mb) at st[mb * ldst + k]
+ * (qt, st) is therefore the 1x128 quantization of X^T in fp8bq_quant_act's
+ * layout.  Requirements: K % 8 == 0; x 16-byte aligned, ldx >= K, ldx % 8 == 0;
+ * qt 16-byte aligned, ldqt >= M, ldqt % 16 == 0; st 16-byte aligned,
+ * ldst >= K, ldst % 4 == 0.
+ */
+FP8BQ_API fp8bq_status fp8bq_quant_act_t(const void *x, int64_t M, int64_t K, int64_t ldx,
+                                         uint8_t *qt, int64_t ldqt, float *st, int64_t ldst,
+                                         int mode, void *stream);
+
+/*
+ * The transpose of a weight's 128x128-tile quantization: qt [K][ldqt] = q^T,
+ * swt [ceil(K/128)][ceil(N/128)] = sw^T (a square tile's scale applies to its
+ * transpose, so no element is requantized).  q [N][ldq], sw [ceil(N/128)][ceil(K/128)].
+ * Requirements: N % 16 == 0, K % 16 == 0; q and qt 16-byte aligned with
+ * ldq >= K, ldqt >= N, both multiples of 16.
+ */
+FP8BQ_API fp8bq_status fp8bq_transpose_weight(const uint8_t *q, int64_t N, int64_t K, int64_t ldq, const float *sw,
+                                              uint8_t *qt, int64_t ldqt, float *swt, void *stream);
+
+/*
+ * Weight-gradient GEMM: y[n][k] = sum_m deq(qa)[n][m] deq(qb)[k][m], bf16 out,
+ * FP32 promotion per 128-token block with the scale product sa * sb formed
+ * per output element.
+ *   qa, sa  codes of dY^T [N][lda] and scales [M/128][ldsa] (fp8bq_quant_act_t of dY)
+ *   qb, sb  codes of X^T [K][ldb] and scales [M/128][ldsb] (fp8bq_quant_act_t of X)
+ *   y       bf16 dW [N][ldy]
+ * Requirements: M % 128 == 0, K % 4 == 0; qa, qb 16-byte aligned, lda, ldb >= M
+ * and multiples of 16; sa, sb 16-byte aligned, ldsa >= N, ldsb >= K, both
+ * multiples of 4; y 16-byte aligned, ldy >= K, ldy % 8 == 0.  M = 0 writes zeros.
+ */
+FP8BQ_API fp8bq_status fp8bq_gemm_wgrad(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa,
+                                        const uint8_t *qb, int64_t ldb, const float *sb, int64_t ldsb,
+                                        void *y, int64_t ldy, int64_t N, int64_t K, int64_t M,
+                                        int mode, void *stream);
+
+/*
+ * One optimizer step fused with the recalibration it makes necessary
+ * ("Real-world performance gains": the weights change every training step, so
+ * their scales are recalibrated after each step; "Technical breakthrough":
+ * 128x128 weight tiles).  The pages do not name the optimizer; this is AdamW
+ * (Loshchilov & Hutter 2019; Adam's bias-corrected moments, Kingma & Ba 2015)
+ * on binary32 master weights and moments.  For every element, each step one
+ * correctly rounded binary32 operation, in this order:
+ *   m  = b1 m + (1 - b1) g
+ *   v  = b2 v + ((1 - b2) g) g
+ *   m^ = m / bc1,  v^ = v / bc2,  bc_i = 1 - b_i^step (computed in double on
+ *        the host and rounded to binary32; 1 - b_i in binary32)
+ *   p  = p - lr (m^ / (sqrt(v^) + eps) + weight_decay p)
+ * then w = bf16(p) (round to nearest even) and (q, s) = the 128x128
+ * quantization of w exactly as fp8bq_quant_weight.  Everything is read and
+ * written in one pass over the tensors.
+ */
+typedef struct {
+    float *param;            /* fp32 master weight [N][K], dense; updated in place */
+    const float *grad;       /* fp32 gradient [N][K], dense */
+    float *exp_avg;          /* fp32 first moment [N][K], dense; updated */
+    float *exp_avg_sq;       /* fp32 second moment [N][K], dense; updated */
+    void *w;                 /* bf16 weight [N][K] written, or NULL (not written) */
+    uint8_t *q;              /* E4M3 codes [N][K], dense */
+    float *s;                /* fp32 scales [ceil(N/128)][ceil(K/128)] */
+    int64_t N, K;
+} fp8bq_adamw_desc;
+
+typedef struct {
+    float lr, beta1, beta2, eps, weight_decay;
+    int64_t step;            /* the step being taken, >= 1 */
+} fp8bq_adamw_config;
+
+/*
+ * descs: host array of n tensors (copied into the launch parameters; may be
+ * freed on return).  Requirements: K % 4 == 0; param, grad, exp_avg,
+ * exp_avg_sq 16-byte aligned; w 8-byte aligned; q and s 4-byte aligned;
+ * 0 <= beta1, beta2 < 1; eps >= 0; step >= 1.  Tensors may not overlap.
+ */
+FP8BQ_API fp8bq_status fp8bq_adamw_recalibrate(const fp8bq_adamw_desc *descs, int n,
+                                               const fp8bq_adamw_config *cfg, int mode, void *stream);
 
 #ifdef __cplusplus
 }

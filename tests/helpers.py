@@ -50,3 +50,23 @@ def assert_gemm_close(y, ref, what=""):
 def need_gpu():
     """GPU tests fail (not skip) without a device: they must never pass vacuously."""
     assert torch.cuda.is_available(), "gpu-marked test run without a CUDA device"
+
+
+def oracle_act(x, mode, rows=None):
+    """The oracle's own 1x128 quantization of bf16 activations (only `rows`, if
+    given: each row's tiles depend on that row alone).  Returns (codes, scales)."""
+    import oracle
+    if rows is not None:
+        x = x[torch.as_tensor(rows, device=x.device)]
+    return oracle.quant_act(bf16_bits(x), mode)
+
+
+def oracle_weight(w, mode):
+    """The oracle's own 128x128 quantization of a bf16 weight [N, K] (or
+    [E, N, K], tile by tile per expert).  Returns (codes, scales)."""
+    import oracle
+    if w.dim() == 3:
+        E, N, K = w.shape
+        q, s = oracle.quant_weight(bf16_bits(w.reshape(E * N, K)), mode)
+        return q.reshape(E, N, K), s.reshape(E, N // 128, -(-K // 128))
+    return oracle.quant_weight(bf16_bits(w), mode)

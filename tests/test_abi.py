@@ -110,3 +110,53 @@ def test_grouped_validation(L):
     assert call(N=260, ldy=264) == UNSUPPORTED                            # N % 8
     assert call(K=200, lda=208) == UNSUPPORTED                            # K % 128
     assert call(rows=0) == 0
+
+
+def test_swiglu_validation(L):
+    f = L.fp8bq_gemm_swiglu_quant
+
+    def call(M=256, I=256, K=256, lda=256, ldsa=256, ldw=256, ldqh=256, ldsh=256, h=None, ldh=0, mode=0, qh=FAKE,
+             sh=FAKE):
+        return f(FAKE, lda, FAKE, ldsa, FAKE, ldw, FAKE, qh, ldqh, sh, ldsh, h, ldh, M, I, K, mode, None)
+    assert call(I=192, ldqh=192) == UNSUPPORTED                          # I % 128
+    assert call(K=200, lda=208, ldw=208) == UNSUPPORTED                  # K % 128
+    assert call(ldqh=128) == INVALID                                     # ldqh < I
+    assert call(ldqh=264) == INVALID                                     # ldqh % 16
+    assert call(qh=None) == INVALID
+    assert call(sh=None) == INVALID
+    assert call(ldsh=255) == INVALID                                     # ldsh < M
+    assert call(ldsh=258) == INVALID                                     # ldsh % 4
+    assert call(h=FAKE, ldh=128) == INVALID                              # ldh < I
+    assert call(h=FAKE, ldh=260) == INVALID                              # ldh % 8
+    assert call(h=ctypes.c_void_p(0x10008), ldh=256) == INVALID          # h alignment
+    assert call(lda=128) == INVALID                                      # lda < K
+    assert call(M=-1) == INVALID
+    assert call(mode=3) == INVALID
+    assert call(M=0) == 0 and call(I=0) == 0
+
+    g = L.fp8bq_grouped_gemm_swiglu_quant
+
+    def gcall(E=4, rows=256, I=256, K=256, off=FAKE, ldqh=256):
+        return g(FAKE, 256, FAKE, 256, FAKE, FAKE, off, E, rows, I, K, FAKE, ldqh, FAKE, 256, None, 0, 0, None)
+    assert gcall(E=0) == INVALID
+    assert gcall(E=1025) == UNSUPPORTED
+    assert gcall(off=None) == INVALID
+    assert gcall(I=192, ldqh=192) == UNSUPPORTED
+    assert gcall(ldqh=100) == INVALID
+    assert gcall(rows=0) == 0
+
+
+def test_interleave_gate_up_layout():
+    """Host-side layout helper of the fused gate+up call: 128-row blocks
+    alternate gate block j, up block j (values exact in bf16)."""
+    import torch
+    import fp8_block_scaled_fp8bq_b200 as fq
+    I, K = 256, 128
+    g = torch.arange(I, dtype=torch.float32)[:, None].expand(I, K).to(torch.bfloat16)
+    u = (-1 - torch.arange(I, dtype=torch.float32))[:, None].expand(I, K).to(torch.bfloat16)
+    col = fq.interleave_gate_up(g, u)[:, 0].float()
+    r = torch.arange(128, dtype=torch.float32)
+    assert torch.equal(col[0:128], r) and torch.equal(col[128:256], -1 - r)
+    assert torch.equal(col[256:384], 128 + r) and torch.equal(col[384:512], -129 - r)
+    e = fq.interleave_gate_up(g.reshape(1, I, K).expand(3, I, K), u.reshape(1, I, K).expand(3, I, K))
+    assert e.shape == (3, 2 * I, K) and torch.equal(e[2, :, 0].float(), col)

@@ -13,7 +13,7 @@ import torch
 import fp8_block_scaled_fp8bq_b200 as fq
 import fp8bq_workloads as wl
 import oracle
-from helpers import assert_gemm_close, bf16_bits, bf16_to_f64, f32, need_gpu, u8
+from helpers import oracle_weight, assert_gemm_close, bf16_bits, bf16_to_f64, f32, need_gpu, u8
 
 pytestmark = pytest.mark.gpu
 
@@ -27,14 +27,18 @@ def _gpu_and_clean_error_word():
 
 
 _W = {}
+_OW = {}
 
 
 def qweights(name, mode):
+    """GPU-quantized weight (codes, scales); the oracle's own quantization of
+    the same bf16 weight is kept beside it for check_decode."""
     key = (name, mode)
     if key not in _W:
         N, K = wl.LLAMA8B_SHAPES[name]
         w = wl.weights(N, K, seed=N * 3 + K, device="cuda")
         _W[key] = fq.quant_weight(w, mode)
+        _OW[_W[key][0].data_ptr()] = oracle_weight(w, mode)
     return _W[key]
 
 
@@ -43,7 +47,8 @@ def check_decode(x, qw, sw, mode):
     y = fq.gemm_decode(x, qw, sw, mode)
     torch.cuda.synchronize()
     qa, sa = oracle.quant_act(bf16_bits(x), mode)
-    ref = oracle.gemm(qa, sa, u8(qw), f32(sw), blockint=True)
+    oqw, osw = _OW[qw.data_ptr()]
+    ref = oracle.gemm(qa, sa, oqw, osw, blockint=True)
     assert_gemm_close(bf16_to_f64(y), ref, "decode M=%d" % M)
     return y
 

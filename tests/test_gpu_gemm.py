@@ -15,10 +15,10 @@ import torch
 import fp8_block_scaled_fp8bq_b200 as fq
 import fp8bq_workloads as wl
 import oracle
-from helpers import assert_gemm_close, bf16_bits, bf16_to_f64, f32, need_gpu, u8
+from helpers import oracle_act, oracle_weight, assert_gemm_close, bf16_bits, bf16_to_f64, f32, need_gpu, u8
 
 pytestmark = pytest.mark.gpu
-VARIANTS = [fq.GEMM_PROMOTE, fq.GEMM_PROMOTE_PAIR]
+VARIANTS = [fq.GEMM_PROMOTE, fq.GEMM_PROMOTE_PAIR, fq.GEMM_PROMOTE_PAIR_N128]
 
 
 @pytest.fixture(autouse=True)
@@ -87,7 +87,8 @@ def test_single_linear_within_tolerance(mode):
 @pytest.mark.parametrize("name", list(wl.LLAMA8B_SHAPES))
 def test_llama_prefill_full_size_sampled_rows(mode, name):
     """The bench's launch configuration (M = 8192) end to end on the GPU: quantize
-    X and W, GEMM; the oracle recomputes 16 sampled rows from the GPU's codes."""
+    X and W, GEMM; the oracle quantizes the same bf16 inputs itself (16 sampled
+    rows of X, all of W) and computes those rows."""
     N, K = wl.LLAMA8B_SHAPES[name]
     M = wl.PREFILL_TOKENS
     x = wl.activations(M, K, seed=N, device="cuda")
@@ -98,9 +99,9 @@ def test_llama_prefill_full_size_sampled_rows(mode, name):
     torch.cuda.synchronize()
     rows = np.sort(np.random.default_rng(N).choice(M, 16, replace=False))
     rows[0], rows[-1] = 0, M - 1
-    # the codes themselves are checked bit-exact elsewhere; here the oracle
-    # recomputes the GEMM from them
-    ref = oracle.gemm(u8(qa), f32(sa)[:, :M], u8(qw), f32(sw), rows=rows, blockint=True)
+    oqa, osa = oracle_act(x, mode, rows)
+    oqw, osw = oracle_weight(w, mode)
+    ref = oracle.gemm(oqa, osa, oqw, osw, blockint=True)
     got = bf16_to_f64(y[torch.from_numpy(rows).cuda()])
     assert_gemm_close(got, ref, name)
 
@@ -141,14 +142,16 @@ def test_row_subset_gives_identical_rows():
     assert torch.equal(y[128:256].view(torch.int16), y2.view(torch.int16))
 
 
-def test_pair_kernel_equals_one_sm_kernel():
-    """The CTA-pair kernel (256x256 tiles, paired MMA) and the one-SM kernel
-    compute every output from the same K-block partials in the same order."""
+@pytest.mark.parametrize("pair_variant", [fq.GEMM_PROMOTE_PAIR, fq.GEMM_PROMOTE_PAIR_N128])
+def test_pair_kernel_equals_one_sm_kernel(pair_variant):
+    """The CTA-pair kernels (256x256 or 256x128 tiles, paired MMA) and the
+    one-SM kernel compute every output from the same K-block partials in the
+    same order."""
     x = wl.activations(640, 1024, seed=21, device="cuda")
     w = wl.weights(768, 1024, seed=22, device="cuda")
     qa, sa = fq.quant_act(x)
     qw, sw = fq.quant_weight(w)
-    y_pair = fq.gemm(qa, sa, qw, sw, variant=fq.GEMM_PROMOTE_PAIR)
+    y_pair = fq.gemm(qa, sa, qw, sw, variant=pair_variant)
     y_one = fq.gemm(qa, sa, qw, sw, variant=fq.GEMM_PROMOTE)
     torch.cuda.synchronize()
     assert_gemm_close(bf16_to_f64(y_pair), bf16_to_f64(y_one), "pair vs one-SM")

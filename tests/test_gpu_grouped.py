@@ -15,7 +15,7 @@ import torch
 import fp8_block_scaled_fp8bq_b200 as fq
 import fp8bq_workloads as wl
 import oracle
-from helpers import assert_gemm_close, bf16_bits, bf16_to_f64, f32, need_gpu, u8
+from helpers import oracle_act, oracle_weight, assert_gemm_close, bf16_bits, bf16_to_f64, f32, need_gpu, u8
 
 pytestmark = pytest.mark.gpu
 
@@ -126,7 +126,9 @@ def test_moe_layer_full_size(which):
         if r1 > r0:
             rows.update({r0, r1 - 1, int(rng.integers(r0, r1))})
     rows = np.array(sorted(rows), dtype=np.int64)
-    ref = oracle.grouped_gemm(u8(qa), f32(sa)[:, :R], u8(qw), f32(sw), offn, rows=rows)
+    oqa, osa = oracle_act(x, mode)
+    oqw, osw = oracle_weight(w, mode)
+    ref = oracle.grouped_gemm(oqa, osa, oqw, osw, offn, rows=rows)
     got = bf16_to_f64(y[torch.from_numpy(rows).cuda()])
     assert_gemm_close(got, ref, "moe " + which)
 

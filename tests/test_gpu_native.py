@@ -13,7 +13,7 @@ import torch
 import fp8_block_scaled_fp8bq_b200 as fq
 import fp8bq_workloads as wl
 import oracle
-from helpers import assert_gemm_close, bf16_bits, bf16_to_f64, f32, need_gpu, u8
+from helpers import oracle_act, oracle_weight, assert_gemm_close, bf16_bits, bf16_to_f64, f32, need_gpu, u8
 
 pytestmark = pytest.mark.gpu
 NATIVE = fq.GEMM_NATIVE_POW2
@@ -68,6 +68,8 @@ def test_llama_shapes_against_oracle_and_promotion(name):
     yp = fq.gemm(qa, sa, qw, sw, fq.SCALE_POW2, variant=fq.GEMM_PROMOTE)
     torch.cuda.synchronize()
     rows = np.array([0, 1, 127, 128, 500, M - 1])
-    ref = oracle.gemm(u8(qa), f32(sa)[:, :M], u8(qw), f32(sw), rows=rows, blockint=True)
+    oqa, osa = oracle_act(x, fq.SCALE_POW2, rows)
+    oqw, osw = oracle_weight(w, fq.SCALE_POW2)
+    ref = oracle.gemm(oqa, osa, oqw, osw, blockint=True)
     assert_gemm_close(bf16_to_f64(yn[torch.from_numpy(rows).cuda()]), ref, "native " + name)
     assert_gemm_close(bf16_to_f64(yn), bf16_to_f64(yp), "native vs promotion " + name)
