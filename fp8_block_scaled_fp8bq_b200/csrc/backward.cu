@@ -27,53 +27,55 @@ using namespace qdev;
 // ---------------------------------------------------------------------------
 // Token-axis 1x128 quantization, transposed output
 // ---------------------------------------------------------------------------
-// Block (bx, by): tokens [128 by, +128) x columns [64 bx, +64) of X.  The
-// 128 x 64 bf16 tile is staged in shared memory (128-byte rows, 16-byte loads,
-// 8 lanes per row); warp w then owns tokens [16 w, 16 w + 16) and lane l the
-// column pair (2 l, 2 l + 1), reading one 4-byte word per token (a warp reads
-// one 128-byte row at a time: no bank conflicts).  Per column, the 8 warps'
-// partial amaxes meet in shared memory; each lane then writes 16 codes of each
-// of its two columns (16 contiguous tokens, 16 bytes) into X^T.
-constexpr int kTTok = 128, kTCol = 64;
+// Block (bx, by): tokens [128 by, +128) x columns [128 bx, +128) of X.  The
+// 128 x 128 bf16 tile is staged in shared memory (256-byte rows, 16-byte
+// loads, 16 lanes per row).  Warp w owns tokens [32 (w & 3), +32) of column
+// half w >> 2, and lane l the column pair (2 l, 2 l + 1) of that half: it reads
+// one 4-byte word per token (a warp reads 128 contiguous bytes of one row:
+// no bank conflicts).  The four token groups' partial amaxes meet in shared
+// memory; each lane then writes 32 token-contiguous codes of each of its two
+// columns into X^T, i.e. whole 32-byte sectors.
+constexpr int kTTok = 128, kTCol = 128;
 
 template <int MODE>
 __global__ void __launch_bounds__(256) quant_act_t_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
                                                           int64_t ldx, uint8_t *__restrict__ qt, int64_t ldqt,
                                                           float *__restrict__ st, int64_t ldst) {
   __shared__ __align__(16) uint32_t tile[kTTok][kTCol / 2];
-  __shared__ uint32_t part[8][kTCol / 2 + 1];  // [warp][column pair]: packed |bf16| maxima
+  __shared__ uint32_t part[4][kTCol / 2];  // [token group][column pair]: packed |bf16| maxima
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t m0 = (int64_t)blockIdx.y * kTTok, k0 = (int64_t)blockIdx.x * kTCol;
 
 #pragma unroll
-  for (int it = 0; it < 4; ++it) {  // 128 rows x 8 chunks of 16 bytes
+  for (int it = 0; it < 8; ++it) {  // 128 rows x 16 chunks of 16 bytes
     const int idx = it * 256 + threadIdx.x;
-    const int r = idx >> 3, c = idx & 7;
+    const int r = idx >> 4, c = idx & 15;
     const int64_t m = m0 + r, k = k0 + c * 8;
     const uint4 v = (m < M && k < K) ? ld_nc_v4(x + m * ldx + k) : make_uint4(0, 0, 0, 0);
     *reinterpret_cast<uint4 *>(&tile[r][c * 4]) = v;
   }
   __syncthreads();
 
-  uint32_t w[16];
+  const int tg = warp & 3, ch = warp >> 2;
+  const int pc = ch * 32 + lane;  // column pair within the tile
+  uint32_t w[32];
   uint32_t am = 0;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    w[i] = tile[warp * 16 + i][lane];
+  for (int i = 0; i < 32; ++i) {
+    w[i] = tile[tg * 32 + i][pc];
     am = __vmaxu2(am, w[i] & 0x7FFF7FFFu);
   }
-  part[warp][lane] = am;
+  part[tg][pc] = am;
   __syncthreads();
-#pragma unroll
-  for (int v = 0; v < 8; ++v) am = __vmaxu2(am, part[v][lane]);
+  am = __vmaxu2(__vmaxu2(part[0][pc], part[1][pc]), __vmaxu2(part[2][pc], part[3][pc]));
   const TileScale t0 = tile_scale<MODE>(bits_to_amax(am & 0xFFFFu));
   const TileScale t1 = tile_scale<MODE>(bits_to_amax(am >> 16));
 
-  const int64_t ka = k0 + 2 * lane, kb = ka + 1;
-  const int64_t mt = m0 + warp * 16;  // first token of this lane's 16
-  uint32_t ca[4], cb[4];              // 16 codes of column ka, 16 of column kb
+  const int64_t ka = k0 + 2 * pc, kb = ka + 1;
+  const int64_t mt = m0 + tg * 32;  // first token of this lane's 32
+  uint32_t ca[8], cb[8];            // 32 codes of column ka, 32 of column kb
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < 8; ++j) {
     const float2 qa0 = quotient2<MODE>(make_float2(bf16_lo(w[4 * j]), bf16_lo(w[4 * j + 1])), t0);
     const float2 qa1 = quotient2<MODE>(make_float2(bf16_lo(w[4 * j + 2]), bf16_lo(w[4 * j + 3])), t0);
     const float2 qb0 = quotient2<MODE>(make_float2(bf16_hi(w[4 * j]), bf16_hi(w[4 * j + 1])), t1);
@@ -82,21 +84,27 @@ __global__ void __launch_bounds__(256) quant_act_t_kernel(const uint16_t *__rest
     cb[j] = e4m3x2(qb0.x, qb0.y) | (e4m3x2(qb1.x, qb1.y) << 16);
   }
   if (mt < M) {
-    const bool whole = mt + 16 <= M;
+    const bool whole = mt + 32 <= M;
     if (ka < K) {
       uint8_t *d = qt + ka * ldqt + mt;
-      if (whole) *reinterpret_cast<uint4 *>(d) = make_uint4(ca[0], ca[1], ca[2], ca[3]);
-      else
-        for (int i = 0; i < 16 && mt + i < M; ++i) d[i] = (uint8_t)(ca[i >> 2] >> (8 * (i & 3)));
+      if (whole) {
+        *reinterpret_cast<uint4 *>(d) = make_uint4(ca[0], ca[1], ca[2], ca[3]);
+        *reinterpret_cast<uint4 *>(d + 16) = make_uint4(ca[4], ca[5], ca[6], ca[7]);
+      } else {
+        for (int i = 0; i < 32 && mt + i < M; ++i) d[i] = (uint8_t)(ca[i >> 2] >> (8 * (i & 3)));
+      }
     }
     if (kb < K) {
       uint8_t *d = qt + kb * ldqt + mt;
-      if (whole) *reinterpret_cast<uint4 *>(d) = make_uint4(cb[0], cb[1], cb[2], cb[3]);
-      else
-        for (int i = 0; i < 16 && mt + i < M; ++i) d[i] = (uint8_t)(cb[i >> 2] >> (8 * (i & 3)));
+      if (whole) {
+        *reinterpret_cast<uint4 *>(d) = make_uint4(cb[0], cb[1], cb[2], cb[3]);
+        *reinterpret_cast<uint4 *>(d + 16) = make_uint4(cb[4], cb[5], cb[6], cb[7]);
+      } else {
+        for (int i = 0; i < 32 && mt + i < M; ++i) d[i] = (uint8_t)(cb[i >> 2] >> (8 * (i & 3)));
+      }
     }
   }
-  if (warp == 0) {
+  if (tg == 0) {
     float *srow = st + (int64_t)blockIdx.y * ldst;
     if (ka < K) srow[ka] = t0.s;
     if (kb < K) srow[kb] = t1.s;
