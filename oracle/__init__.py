@@ -75,6 +75,8 @@ def lib():
         L.o_swiglu_bf16.argtypes = [P, P, I64, P]
         L.o_gemm_wgrad_rows.restype = None
         L.o_gemm_wgrad_rows.argtypes = [P, I64, P, I64, P, I64, P, I64, I64, I64, I64, P, I64, P]
+        L.o_decode_attention.restype = None
+        L.o_decode_attention.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, I64, ctypes.c_double, P]
         L.o_adamw_step.restype = None
         L.o_adamw_step.argtypes = [P, P, P, P, I64, ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                                    ctypes.c_float, I64]
@@ -357,3 +359,36 @@ def gemm_wgrad(qa, sa, qb, sb, rows=None):
     lib().o_gemm_wgrad_rows(_p(qa), M, _p(sa), sa.shape[1], _p(qb), M, _p(sb), sb.shape[1], N, K, M,
                             None if r is None else _p(r), R, _p(y))
     return y
+
+
+# --- decode attention over an FP8 KV cache --------------------------------------
+
+def quant_kv(x_bits, mode):
+    """E4M3 codes of a key or value cache [B, S, Hkv, D=128] (bf16 bits) with one
+    scale per head vector (one 1x128 tile): returns (codes [B, S, Hkv, D],
+    scales [B, S, Hkv])."""
+    x = np.asarray(x_bits, dtype=np.uint16)
+    B, S, H, D = x.shape
+    if D != 128:
+        raise ValueError("head dimension must be 128 (one 1x128 tile)")
+    q, s = quant_act(x.reshape(B * S * H, D), mode)
+    return q.reshape(B, S, H, D), s[0, :B * S * H].reshape(B, S, H)
+
+
+def decode_attention(q_bits, kq, ks, vq, vs, lens, scale):
+    """Attention of one query token per batch entry over its cached tokens
+    (see o_decode_attention); returns float64 [B, Hq, D]."""
+    q = _c(q_bits, np.uint16)
+    kq = _c(kq, np.uint8)
+    vq = _c(vq, np.uint8)
+    ks = _c(ks, np.float32)
+    vs = _c(vs, np.float32)
+    lens = _c(np.asarray(lens, dtype=np.int32), np.int32)
+    B, Hq, D = q.shape
+    _, S, Hkv, _ = kq.shape
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    out = np.empty((B, Hq, D), dtype=np.float64)
+    lib().o_decode_attention(_p(q), _p(kq), _p(ks), _p(vq), _p(vs), _p(lens), B, Hq, Hkv, S, D, float(scale),
+                             _p(out))
+    return out
