@@ -73,7 +73,7 @@ def load_peaks():
 
 def kernel_source_sha():
     h = hashlib.sha256()
-    for f in ("gemm.cu", "gemm_promote.cuh", "device.cuh", "api.cu"):
+    for f in ("gemm.cu", "gemm_promote.cuh", "device.cuh", "quant.cuh", "raster.cu"):
         h.update(open(os.path.join(ROOT, "fp8_block_scaled_fp8bq_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -424,7 +424,8 @@ def reference(args):
 CASES = (["gemm:" + n for n in NAMES] + ["decode:" + n for n in NAMES] + ["cublas:" + n for n in NAMES] +
          ["quant_act:4096", "quant_act:14336", "recalibrate:layer", "quant_weight:gate_up", "moe:up", "moe:down",
           "swiglu:gate_up", "moe_swiglu:up", "adamw_recal:layer", "quant_act_t:4096", "quant_act_t:14336",
-          "transpose_weight:gate_up"] + ["dgrad:" + n for n in NAMES] + ["wgrad:" + n for n in NAMES])
+          "transpose_weight:gate_up", "decode_attn:1x32768", "decode_attn:16x8192", "decode_attn:64x4096",
+          "decode_attn:256x2048"] + ["dgrad:" + n for n in NAMES] + ["wgrad:" + n for n in NAMES])
 
 
 def decode_bytes(M, N, K):
@@ -532,6 +533,26 @@ def run_case(args):
                 + 4 * R * (N // 256)) / 1e9
         unit = "GB/s"
         print(json.dumps({"case": args.case, "flops": 2.0 * R * N * K}))
+    elif kind == "decode_attn":
+        # Llama-3.1-8B attention (32 query heads, 8 key/value heads, D = 128):
+        # one query token per sequence over a full FP8 cache of the given length
+        B_, S_ = (int(v) for v in what.split("x"))
+        Hq, Hkv = 32, 8
+        g = torch.Generator(device=dev).manual_seed(5)
+        kq = torch.randint(0, 0x7E, (B_, S_, Hkv, 128), generator=g, device=dev, dtype=torch.uint8)
+        vq = torch.randint(0, 0x7E, (B_, S_, Hkv, 128), generator=g, device=dev, dtype=torch.uint8)
+        kq |= torch.randint(0, 2, kq.shape, generator=g, device=dev, dtype=torch.uint8) << 7
+        vq |= torch.randint(0, 2, vq.shape, generator=g, device=dev, dtype=torch.uint8) << 7
+        ks = torch.rand((B_, S_, Hkv), generator=g, device=dev) * 0.01 + 0.001
+        vs = torch.rand((B_, S_, Hkv), generator=g, device=dev) * 0.01 + 0.001
+        qv = torch.randn((B_, Hq, 128), generator=g, device=dev).to(torch.bfloat16)
+        lens = torch.full((B_,), S_, dtype=torch.int32, device=dev)
+        out = torch.empty((B_, Hq, 128), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(16, int(fq.lib().fp8bq_decode_attention_workspace_size(B_, Hq, Hkv, S_))),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda: fq.decode_attention(qv, kq, ks, vq, vs, lens, out=out, ws=ws)  # noqa: E731
+        work = (B_ * S_ * Hkv * (2 * 128 + 8) + 2 * B_ * Hq * 128 * 2) / 1e9
+        unit = "GB/s"
     elif kind == "quant_act_t":
         K = int(what)
         x = wl.activations(M, K, seed=1, device=dev)

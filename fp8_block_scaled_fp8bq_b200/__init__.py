@@ -78,6 +78,9 @@ SIGNATURES = {
     "fp8bq_quant_act_t": (I32, [P, I64, I64, I64, P, I64, P, I64, I32, P]),
     "fp8bq_transpose_weight": (I32, [P, I64, I64, I64, P, P, I64, P, P]),
     "fp8bq_gemm_wgrad": (I32, [P, I64, P, I64, P, I64, P, I64, P, I64, I64, I64, I64, I32, P]),
+    "fp8bq_kv_cache_append": (I32, [P, P, P, P, P, P, P, I64, I64, I64, I32, P]),
+    "fp8bq_decode_attention_workspace_size": (SZ, [I64, I64, I64, I64]),
+    "fp8bq_decode_attention": (I32, [P, P, P, P, P, P, I64, I64, I64, I64, ctypes.c_float, P, P, SZ, P]),
     "fp8bq_adamw_recalibrate": (I32, [ctypes.POINTER(AdamWDesc), I32, ctypes.POINTER(AdamWConfig), I32, P]),
     "fp8bq_gemm_swiglu_quant": (I32, [P, I64, P, I64, P, I64, P, P, I64, P, I64, P, I64, I64, I64, I64, I32, P]),
     "fp8bq_grouped_gemm_swiglu_quant": (I32, [P, I64, P, I64, P, P, P, I32, I64, I64, I64, P, I64, P, I64, P, I64,
@@ -214,6 +217,30 @@ def gemm_wgrad(qa, sa, qb, sb, M, mode=SCALE_FP32, out=None, stream=None):
     _check(lib().fp8bq_gemm_wgrad(_ptr(qa), _ld(qa), _ptr(sa), sa.stride(0), _ptr(qb), _ld(qb), _ptr(sb),
                                   sb.stride(0), _ptr(out), _ld(out), N, K, M, mode, _stream(stream)),
            "fp8bq_gemm_wgrad")
+    return out
+
+
+def kv_cache_append(k_new, v_new, positions, kq, ks, vq, vs, mode=SCALE_FP32, stream=None):
+    """Quantize one new token per sequence into the FP8 cache at positions[b]."""
+    B, S, Hkv, D = kq.shape
+    _check(lib().fp8bq_kv_cache_append(_ptr(k_new), _ptr(v_new), _ptr(positions), _ptr(kq), _ptr(ks), _ptr(vq),
+                                       _ptr(vs), B, Hkv, S, mode, _stream(stream)), "fp8bq_kv_cache_append")
+
+
+def decode_attention(q, kq, ks, vq, vs, seq_lens, softmax_scale=None, out=None, ws=None, stream=None):
+    """One query token per sequence over its FP8 KV cache; q bf16 [B, Hq, 128]."""
+    B, Hq, D = q.shape
+    _, S, Hkv, _ = kq.shape
+    if softmax_scale is None:
+        softmax_scale = 1.0 / float(D) ** 0.5
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    need = int(lib().fp8bq_decode_attention_workspace_size(B, Hq, Hkv, S))
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().fp8bq_decode_attention(_ptr(q), _ptr(kq), _ptr(ks), _ptr(vq), _ptr(vs), _ptr(seq_lens), B, Hq, Hkv,
+                                        S, softmax_scale, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "fp8bq_decode_attention")
     return out
 
 

@@ -46,27 +46,6 @@ int num_sms() {
   return g_sms[d];
 }
 
-void choose_raster(int64_t M, int64_t N, int64_t K, int bm, int bn, int32_t *band, int32_t *n_major) {
-  // Panels of one band must stay in L2 while the other operand and the output
-  // stream past them: a third of the 126 MB L2, with room left for the panels
-  // in flight and the output lines not yet written back.
-  constexpr int64_t kBandBytes = int64_t(40) << 20;
-  const int64_t num_m = (M + bm - 1) / bm, num_n = (N + bn - 1) / bn;
-  const int64_t a_panel = (int64_t)bm * K, w_panel = (int64_t)bn * K;
-  const int64_t band_m = std::max<int64_t>(1, std::min<int64_t>(num_m, kBandBytes / std::max<int64_t>(a_panel, 1)));
-  const int64_t band_n = std::max<int64_t>(1, std::min<int64_t>(num_n, kBandBytes / std::max<int64_t>(w_panel, 1)));
-  // M bands: A is read once, W once per band; N bands the other way round.
-  const int64_t bytes_m = M * K + N * K * ((num_m + band_m - 1) / band_m);
-  const int64_t bytes_n = N * K + M * K * ((num_n + band_n - 1) / band_n);
-  if (bytes_m <= bytes_n) {
-    *band = (int32_t)band_m;
-    *n_major = 0;
-  } else {
-    *band = (int32_t)band_n;
-    *n_major = 1;
-  }
-}
-
 fp8bq_status cuda_fail(cudaError_t e, const char *what) {
   snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", what, cudaGetErrorString(e));
   return FP8BQ_ERR_CUDA;
@@ -361,6 +340,45 @@ fp8bq_status fp8bq_gemm_wgrad(const uint8_t *qa, int64_t lda, const float *sa, i
   if (ldsa < N || ldsa % 4 != 0 || !aligned(sa, 16)) return FP8BQ_ERR_INVALID_ARG;
   if (ldsb < K || ldsb % 4 != 0 || !aligned(sb, 16)) return FP8BQ_ERR_INVALID_ARG;
   return launch_gemm_wgrad(qa, lda, sa, ldsa, qb, ldb, sb, ldsb, y, ldy, N, K, M, static_cast<cudaStream_t>(stream));
+}
+
+size_t fp8bq_decode_attention_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t S) {
+  return decode_attention_workspace_size(B, Hq, Hkv, S);
+}
+
+fp8bq_status fp8bq_decode_attention(const void *q, const uint8_t *kq, const float *ks, const uint8_t *vq,
+                                    const float *vs, const int32_t *seq_lens, int64_t B, int64_t Hq, int64_t Hkv,
+                                    int64_t S, float softmax_scale, void *o, void *ws, size_t ws_bytes,
+                                    void *stream) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || S < 0) return FP8BQ_ERR_INVALID_ARG;
+  if (B >= kMaxDim || Hq >= 65536 || Hkv >= 65536 || S >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
+  if (B == 0 || Hq == 0) return FP8BQ_OK;
+  if (Hkv == 0 || Hq % Hkv != 0) return FP8BQ_ERR_INVALID_ARG;
+  const int64_t G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return FP8BQ_ERR_UNSUPPORTED;
+  if (B * Hkv > 0x7fffffffLL) return FP8BQ_ERR_UNSUPPORTED;
+  if (!q || !o || !aligned(q, 2) || !aligned(o, 8)) return FP8BQ_ERR_INVALID_ARG;
+  if (S > 0) {
+    if (!kq || !ks || !vq || !vs || !seq_lens || !ws) return FP8BQ_ERR_INVALID_ARG;
+    if (!aligned(kq, 16) || !aligned(vq, 4) || !aligned(ks, 4) || !aligned(vs, 4) || !aligned(seq_lens, 4) ||
+        !aligned(ws, 16))
+      return FP8BQ_ERR_INVALID_ARG;
+  }
+  return launch_decode_attention(q, kq, ks, vq, vs, seq_lens, B, Hq, Hkv, S, softmax_scale, o, ws, ws_bytes,
+                                 static_cast<cudaStream_t>(stream));
+}
+
+fp8bq_status fp8bq_kv_cache_append(const void *k_new, const void *v_new, const int32_t *positions, uint8_t *kq,
+                                   float *ks, uint8_t *vq, float *vs, int64_t B, int64_t Hkv, int64_t S, int mode,
+                                   void *stream) {
+  if (B < 0 || Hkv < 0 || S < 0 || bad_mode(mode)) return FP8BQ_ERR_INVALID_ARG;
+  if (2 * B * Hkv >= kMaxDim || S >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
+  if (B == 0 || Hkv == 0 || S == 0) return FP8BQ_OK;
+  if (!k_new || !v_new || !positions || !kq || !ks || !vq || !vs) return FP8BQ_ERR_INVALID_ARG;
+  if (!aligned(k_new, 8) || !aligned(v_new, 8) || !aligned(positions, 4) || !aligned(kq, 4) || !aligned(vq, 4) ||
+      !aligned(ks, 4) || !aligned(vs, 4))
+    return FP8BQ_ERR_INVALID_ARG;
+  return launch_kv_append(k_new, v_new, positions, kq, ks, vq, vs, B, Hkv, S, mode, static_cast<cudaStream_t>(stream));
 }
 
 fp8bq_status fp8bq_adamw_recalibrate(const fp8bq_adamw_desc *descs, int n, const fp8bq_adamw_config *cfg, int mode,

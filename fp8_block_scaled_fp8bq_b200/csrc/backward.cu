@@ -76,12 +76,13 @@ __global__ void __launch_bounds__(256) quant_act_t_kernel(const uint16_t *__rest
   uint32_t ca[8], cb[8];            // 32 codes of column ka, 32 of column kb
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    const float2 qa0 = quotient2<MODE>(make_float2(bf16_lo(w[4 * j]), bf16_lo(w[4 * j + 1])), t0);
-    const float2 qa1 = quotient2<MODE>(make_float2(bf16_lo(w[4 * j + 2]), bf16_lo(w[4 * j + 3])), t0);
-    const float2 qb0 = quotient2<MODE>(make_float2(bf16_hi(w[4 * j]), bf16_hi(w[4 * j + 1])), t1);
-    const float2 qb1 = quotient2<MODE>(make_float2(bf16_hi(w[4 * j + 2]), bf16_hi(w[4 * j + 3])), t1);
-    ca[j] = e4m3x2(qa0.x, qa0.y) | (e4m3x2(qa1.x, qa1.y) << 16);
-    cb[j] = e4m3x2(qb0.x, qb0.y) | (e4m3x2(qb1.x, qb1.y) << 16);
+    // codes of -(x / s), sign bits flipped back (see neg_quotient2)
+    const float2 qa0 = neg_quotient2<MODE>(make_float2(bf16_lo(w[4 * j]), bf16_lo(w[4 * j + 1])), t0);
+    const float2 qa1 = neg_quotient2<MODE>(make_float2(bf16_lo(w[4 * j + 2]), bf16_lo(w[4 * j + 3])), t0);
+    const float2 qb0 = neg_quotient2<MODE>(make_float2(bf16_hi(w[4 * j]), bf16_hi(w[4 * j + 1])), t1);
+    const float2 qb1 = neg_quotient2<MODE>(make_float2(bf16_hi(w[4 * j + 2]), bf16_hi(w[4 * j + 3])), t1);
+    ca[j] = (e4m3x2(qa0.x, qa0.y) | (e4m3x2(qa1.x, qa1.y) << 16)) ^ 0x80808080u;
+    cb[j] = (e4m3x2(qb0.x, qb0.y) | (e4m3x2(qb1.x, qb1.y) << 16)) ^ 0x80808080u;
   }
   if (mt < M) {
     const bool whole = mt + 32 <= M;

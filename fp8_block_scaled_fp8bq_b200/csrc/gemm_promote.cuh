@@ -433,10 +433,10 @@ __device__ __forceinline__ bool swiglu_epilogue(const Smem &S, const GemmArgs &a
 #pragma unroll
     for (int c = 0; c < 4; ++c) {  // 16 codes per store
       uint4 pk;
-      pk.x = qdev::encode2<MODE>(hw[8 * c + 0], ts) | (qdev::encode2<MODE>(hw[8 * c + 1], ts) << 16);
-      pk.y = qdev::encode2<MODE>(hw[8 * c + 2], ts) | (qdev::encode2<MODE>(hw[8 * c + 3], ts) << 16);
-      pk.z = qdev::encode2<MODE>(hw[8 * c + 4], ts) | (qdev::encode2<MODE>(hw[8 * c + 5], ts) << 16);
-      pk.w = qdev::encode2<MODE>(hw[8 * c + 6], ts) | (qdev::encode2<MODE>(hw[8 * c + 7], ts) << 16);
+      pk.x = qdev::encode4<MODE>(hw[8 * c + 0], hw[8 * c + 1], ts);
+      pk.y = qdev::encode4<MODE>(hw[8 * c + 2], hw[8 * c + 3], ts);
+      pk.z = qdev::encode4<MODE>(hw[8 * c + 4], hw[8 * c + 5], ts);
+      pk.w = qdev::encode4<MODE>(hw[8 * c + 6], hw[8 * c + 7], ts);
       *reinterpret_cast<uint4 *>(q + 16 * c) = pk;
     }
     if (HALF == 0) a.sh[(int64_t)tl.nb * a.ldsh + m] = ts.s;

@@ -84,5 +84,12 @@ fp8bq_status launch_transpose_weight(const uint8_t *q, int64_t N, int64_t K, int
 fp8bq_status launch_gemm_wgrad(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qb,
                                int64_t ldb, const float *sb, int64_t ldsb, void *y, int64_t ldy, int64_t N, int64_t K,
                                int64_t M, cudaStream_t stream);
+size_t decode_attention_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t S);
+fp8bq_status launch_decode_attention(const void *q, const uint8_t *kq, const float *ks, const uint8_t *vq,
+                                     const float *vs, const int32_t *lens, int64_t B, int64_t Hq, int64_t Hkv,
+                                     int64_t S, float scale, void *o, void *ws, size_t ws_bytes, cudaStream_t stream);
+fp8bq_status launch_kv_append(const void *k_new, const void *v_new, const int32_t *pos, uint8_t *kq, float *ks,
+                              uint8_t *vq, float *vs, int64_t B, int64_t Hkv, int64_t S, int mode,
+                              cudaStream_t stream);
 
 }  // namespace fp8bq

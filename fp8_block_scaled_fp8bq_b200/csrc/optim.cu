@@ -135,7 +135,7 @@ __device__ __forceinline__ void adamw_tile(const OptTensor &T, const OptParams &
   for (int i = 0; i < 16; ++i) {
     const int64_t n = r0 + i;
     if (kin && n < T.N)
-      *reinterpret_cast<uint32_t *>(T.q + n * T.K + k) = encode2<MODE>(wb[i][0], ts) | (encode2<MODE>(wb[i][1], ts) << 16);
+      *reinterpret_cast<uint32_t *>(T.q + n * T.K + k) = encode4<MODE>(wb[i][0], wb[i][1], ts);
   }
   if (threadIdx.x == 0) T.s[nb * T.KB + kb] = ts.s;
   __syncthreads();  // red[] is reused by the next tile

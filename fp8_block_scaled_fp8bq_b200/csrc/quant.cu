@@ -107,17 +107,100 @@ __device__ __forceinline__ void quant_tile_scalar(const TileTensor &T, int64_t n
   __syncthreads();
 }
 
+// The tensor holding global tile `tile`: the last one whose first tile is <= tile.
+__device__ __forceinline__ int tensor_of(const RecalParams &p, int64_t tile) {
+  int lo = 0, hi = p.n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.t[mid].tile_begin <= tile) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Vector path, software pipelined through shared memory: every thread copies
+// its own eight 16-byte chunks of the next tile with cp.async while it encodes
+// the current one, so a block always has a tile's loads in flight.  A thread
+// reads back only the chunks it copied itself (no block barrier is needed for
+// the data; the one per tile is for the amax).
+__device__ __forceinline__ void issue_tile_copy(const TileTensor &T, int64_t nb, int64_t kb, uint4 *buf) {
+  const int t = threadIdx.x;
+  const int c = t & 15, r0 = t >> 4;
+  const int64_t k = kb * 128 + c * 8;
+  const bool kin = k < T.K;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t n = nb * 128 + r0 + 16 * i;
+    const bool in = kin && n < T.N;
+    cp_async_16(buf + i * 256 + t, in ? static_cast<const void *>(T.w + n * T.ldw + k) : static_cast<const void *>(T.w),
+                in ? 16u : 0u);
+  }
+}
+
 template <int MODE>
-__global__ void __launch_bounds__(256, 4) recalibrate_kernel(const __grid_constant__ RecalParams p) {
+__global__ void __launch_bounds__(256, 3) recalibrate_pipelined_kernel(const __grid_constant__ RecalParams p) {
+  __shared__ uint32_t red[8];
+  extern __shared__ uint4 stage_buf[];  // 2 x [8][256] 16-byte chunks (64 KB)
+  int64_t tile = blockIdx.x;
+  if (tile >= p.total) return;
+  int ti = tensor_of(p, tile);
+  int64_t local = tile - p.t[ti].tile_begin;
+  int64_t nb = local / p.t[ti].KB, kb = local - nb * p.t[ti].KB;
+  issue_tile_copy(p.t[ti], nb, kb, stage_buf);
+  cp_async_commit();
+  for (int it = 0;; ++it) {
+    uint4 *cur = stage_buf + (it & 1) * 2048;
+    const int64_t next = tile + gridDim.x;
+    int tn = ti;
+    int64_t nbn = 0, kbn = 0;
+    if (next < p.total) {
+      tn = tensor_of(p, next);
+      const int64_t ln = next - p.t[tn].tile_begin;
+      nbn = ln / p.t[tn].KB;
+      kbn = ln - nbn * p.t[tn].KB;
+      issue_tile_copy(p.t[tn], nbn, kbn, stage_buf + ((it + 1) & 1) * 2048);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();  // this thread's copies of the current tile have landed
+    uint4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = cur[i * 256 + threadIdx.x];
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = max(m, absmax_bits8(v[i]));
+    m = __reduce_max_sync(0xffffffffu, m);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) m = max(m, red[w]);
+    const TileScale ts = tile_scale<MODE>(bits_to_amax(m));
+    const TileTensor &T = p.t[ti];
+    const int c = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+    const int64_t k = kb * 128 + c * 8;
+    if (k < T.K) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int64_t n = nb * 128 + r0 + 16 * i;
+        if (n < T.N) *reinterpret_cast<uint2 *>(T.q + n * T.ldq + k) = encode8<MODE>(v[i], ts);
+      }
+    }
+    if (threadIdx.x == 0) T.s[nb * T.KB + kb] = ts.s;
+    __syncthreads();  // red[] is reused by the next tile
+    if (next >= p.total) break;
+    tile = next;
+    ti = tn;
+    nb = nbn;
+    kb = kbn;
+  }
+  cp_async_wait<0>();
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(256, 3) recalibrate_kernel(const __grid_constant__ RecalParams p) {
   __shared__ uint32_t red[8];
   for (int64_t tile = blockIdx.x; tile < p.total; tile += gridDim.x) {
-    int lo = 0, hi = p.n - 1;  // last tensor whose first tile is <= tile
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (p.t[mid].tile_begin <= tile) lo = mid;
-      else hi = mid - 1;
-    }
-    const TileTensor &T = p.t[lo];
+    const TileTensor &T = p.t[tensor_of(p, tile)];
     const int64_t local = tile - T.tile_begin;
     const int64_t nb = local / T.KB, kb = local - nb * T.KB;
     if (T.vec) quant_tile_vec<MODE>(T, nb, kb, red);
@@ -140,6 +223,25 @@ __global__ void __launch_bounds__(256) encode_kernel(const float *__restrict__ x
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 int g_recal_blocks_per_sm[2] = {0, 0};
+
+constexpr int kPipeSmem = 2 * 8 * 256 * 16;  // two stages of a 128x128 bf16 tile
+int g_pipe_blocks_per_sm = 0;
+
+fp8bq_status prepare_pipelined() {
+  if (g_pipe_blocks_per_sm > 0) return FP8BQ_OK;
+  cudaError_t e = cudaFuncSetAttribute(recalibrate_pipelined_kernel<FP8BQ_SCALE_FP32>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kPipeSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(recalibrate_pipelined_kernel<FP8BQ_SCALE_POW2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kPipeSmem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(recalibrate)");
+  int b = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, recalibrate_pipelined_kernel<FP8BQ_SCALE_FP32>, 256,
+                                                    kPipeSmem);
+  if (e != cudaSuccess) return cuda_fail(e, "occupancy(recalibrate)");
+  g_pipe_blocks_per_sm = std::max(1, b);
+  return FP8BQ_OK;
+}
 
 }  // namespace
 
@@ -205,11 +307,23 @@ fp8bq_status launch_recalibrate(const fp8bq_weight_desc *descs, int n, int mode,
       p.total += ((d.N + 127) / 128) * (int64_t)t.KB;
     }
     if (p.total == 0) continue;
-    const unsigned grid = (unsigned)std::min<int64_t>(p.total, resident);
-    if (mode == FP8BQ_SCALE_FP32)
-      recalibrate_kernel<FP8BQ_SCALE_FP32><<<grid, 256, 0, stream>>>(p);
-    else
-      recalibrate_kernel<FP8BQ_SCALE_POW2><<<grid, 256, 0, stream>>>(p);
+    bool all_vec = true;
+    for (int i = 0; i < p.n; ++i) all_vec = all_vec && p.t[i].vec;
+    if (all_vec) {
+      fp8bq_status st = prepare_pipelined();
+      if (st != FP8BQ_OK) return st;
+      const unsigned grid = (unsigned)std::min<int64_t>(p.total, (int64_t)num_sms() * g_pipe_blocks_per_sm);
+      if (mode == FP8BQ_SCALE_FP32)
+        recalibrate_pipelined_kernel<FP8BQ_SCALE_FP32><<<grid, 256, kPipeSmem, stream>>>(p);
+      else
+        recalibrate_pipelined_kernel<FP8BQ_SCALE_POW2><<<grid, 256, kPipeSmem, stream>>>(p);
+    } else {
+      const unsigned grid = (unsigned)std::min<int64_t>(p.total, resident);
+      if (mode == FP8BQ_SCALE_FP32)
+        recalibrate_kernel<FP8BQ_SCALE_FP32><<<grid, 256, 0, stream>>>(p);
+      else
+        recalibrate_kernel<FP8BQ_SCALE_POW2><<<grid, 256, 0, stream>>>(p);
+    }
     fp8bq_status st = check_launch("recalibrate");
     if (st != FP8BQ_OK) return st;
   }

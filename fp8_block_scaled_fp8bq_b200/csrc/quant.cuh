@@ -98,31 +98,51 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
 }
 
-// Two quotients at once with the packed FP32 instructions (the same IEEE
-// operations as quotient(), two lanes per instruction).
+// The negated quotient -(x / s), correctly rounded, two lanes per instruction.
+// Negating the per-tile constant r instead of per-element values leaves the
+// packed sequence with no sign flips:
+//   -q0 = RN(x * -r),  e = x - q0 s = fma(-q0, s, x) (exact),
+//   -q1 = RN(e * -r - q0) = fma(e, -r, -q0),
+// which is -(q0 + e r), Markstein's correction of q0, negated (round to
+// nearest is symmetric).  Zero keeps its sign: x = -0 gives +0 = -(-0) and
+// x = +0 gives -0.  The E4M3 code of x / s is then the code of -(x / s) with
+// its sign bit flipped (the conversion is sign-symmetric).
 template <int MODE>
-__device__ __forceinline__ float2 quotient2(float2 x, const TileScale &t) {
-  const float2 r2 = make_float2(t.r, t.r);
-  if (MODE == FP8BQ_SCALE_POW2) return __fmul2_rn(x, r2);
-  if (t.exact) return make_float2(__fdiv_rn(x.x, t.s), __fdiv_rn(x.y, t.s));
-  const float2 q0 = __fmul2_rn(x, r2);
-  const float2 res = __ffma2_rn(q0, make_float2(t.s, t.s), make_float2(-x.x, -x.y));
-  return __ffma2_rn(make_float2(-res.x, -res.y), r2, q0);
+__device__ __forceinline__ float2 neg_quotient2(float2 x, const TileScale &t) {
+  const float2 nr2 = make_float2(-t.r, -t.r);
+  if (MODE == FP8BQ_SCALE_POW2) return __fmul2_rn(x, nr2);
+  if (t.exact) return make_float2(-__fdiv_rn(x.x, t.s), -__fdiv_rn(x.y, t.s));
+  const float2 nq0 = __fmul2_rn(x, nr2);
+  const float2 e = __ffma2_rn(nq0, make_float2(t.s, t.s), x);
+  return __ffma2_rn(e, nr2, nq0);
 }
 
-// Two bf16 packed in a 32-bit word (lower address in the low half) -> E4M3x2.
+// Codes of -(x / s) for two bf16 packed in a 32-bit word (lower address in the
+// low half): the codes of x / s with both sign bits flipped.
+template <int MODE>
+__device__ __forceinline__ uint32_t encode2_neg(uint32_t w, const TileScale &t) {
+  const float2 nq = neg_quotient2<MODE>(make_float2(bf16_lo(w), bf16_hi(w)), t);
+  return e4m3x2(nq.x, nq.y);
+}
+
+// Four bf16 (two packed words) -> four E4M3 codes.
+template <int MODE>
+__device__ __forceinline__ uint32_t encode4(uint32_t w01, uint32_t w23, const TileScale &t) {
+  return (encode2_neg<MODE>(w01, t) | (encode2_neg<MODE>(w23, t) << 16)) ^ 0x80808080u;
+}
+
+// Two bf16 packed in a 32-bit word -> E4M3x2.
 template <int MODE>
 __device__ __forceinline__ uint32_t encode2(uint32_t w, const TileScale &t) {
-  const float2 q = quotient2<MODE>(make_float2(bf16_lo(w), bf16_hi(w)), t);
-  return e4m3x2(q.x, q.y);
+  return encode2_neg<MODE>(w, t) ^ 0x8080u;
 }
 
 // 8 bf16 (one 16-byte vector) -> 8 E4M3 codes (8 bytes).
 template <int MODE>
 __device__ __forceinline__ uint2 encode8(uint4 v, const TileScale &t) {
   uint2 r;
-  r.x = encode2<MODE>(v.x, t) | (encode2<MODE>(v.y, t) << 16);
-  r.y = encode2<MODE>(v.z, t) | (encode2<MODE>(v.w, t) << 16);
+  r.x = encode4<MODE>(v.x, v.y, t);
+  r.y = encode4<MODE>(v.z, v.w, t);
   return r;
 }
 
