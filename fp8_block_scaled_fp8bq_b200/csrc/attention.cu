@@ -63,7 +63,7 @@ struct AttnArgs {
 };
 
 template <int G>
-__global__ void __launch_bounds__(kAttnWarps * 32) decode_attn_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(kAttnWarps * 32, G >= 8 ? 2 : 4) decode_attn_kernel(const AttnArgs a) {
   __shared__ __align__(16) float qs[G][kD];
   __shared__ __align__(16) float ps[kAttnWarps][kTokPerIter][G];
   __shared__ float red_m[kAttnWarps][G], red_l[kAttnWarps][G];
