@@ -12,15 +12,18 @@
 // Split over the sequence (flash decoding): block (b, g, split) handles one
 // key/value head g of batch entry b over one chunk of tokens, for all G query
 // heads that share g (grouped-query attention), so each cached vector is read
-// once.  Per warp and 32 tokens:
-//   scores   lane l takes token l: its 128-byte key row in eight 16-byte loads,
-//            converted pairwise (e4m3x2 -> f16x2 -> f32), dotted with the G
-//            queries (shared memory, broadcast reads) with packed FP32 fma;
+// once.  Every warp streams its 32-token steps through two shared-memory
+// stages with cp.async (16-byte pieces, each key and value row read as whole
+// 128-byte lines), so the next step's bytes are in flight while the current
+// one is computed.  Per warp and step:
+//   scores   lane l takes token l: its key row from the stage, converted
+//            pairwise (e4m3x2 -> f16x2 -> f32), dotted with the G queries
+//            (shared memory, broadcast reads) with packed FP32 fma;
 //   softmax  running max and sum per head across the warp (online softmax);
 //   values   the probabilities go to shared memory; lane l then owns head
-//            dimensions 4l .. 4l+3 and reads each token's 4 value bytes
-//            (128 contiguous bytes per warp) and the token's G probabilities
-//            (one broadcast load) and accumulates with packed fma.
+//            dimensions 4l .. 4l+3 and reads each token's 4 value bytes from
+//            the stage and the token's G probabilities (one broadcast load)
+//            and accumulates with packed fma.
 // The four warps' partial (max, sum, output) meet in shared memory and the
 // block writes one partial per query head; a second kernel merges the splits.
 #include <cuda_bf16.h>
@@ -44,6 +47,12 @@ constexpr int kTokPerIter = 32;   // tokens per warp iteration
 constexpr int kChunkQuantum = kAttnWarps * kTokPerIter;
 constexpr int kPart = kD + 4;     // floats per split partial: output [D], max, sum, 2 pad (16-byte rows)
 
+// 4-byte asynchronous copy global -> shared (src_bytes = 0: zero-fill, nothing read).
+__device__ __forceinline__ void cp_async_4(void *smem_dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_addr(smem_dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
 // Two E4M3 codes (low byte first) -> two floats, exactly.
 __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t c) {
   __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)c, __NV_E4M3);
@@ -62,12 +71,46 @@ struct AttnArgs {
   float scale;
 };
 
+// Per-warp staging of one 32-token step in shared memory (two such stages per
+// warp, double-buffered): key rows padded to 144 bytes so that each lane's
+// eight 16-byte reads of its own row are conflict-free, value rows of 128
+// bytes, and the 32 tokens' key and value scales.
+constexpr int kKPitch = 144;
+struct StepStage {
+  uint8_t k[kTokPerIter][kKPitch];
+  uint8_t v[kTokPerIter][kD];
+  float ks[kTokPerIter];
+  float vs[kTokPerIter];
+};
+
+// Issue the asynchronous copies of the step at token `base` (this lane's
+// share: four 16-byte key pieces, four value pieces, one key and one value
+// scale).  Tokens at or past t_end are zero-filled.
+__device__ __forceinline__ void issue_step(StepStage &st, const uint8_t *kbase, const uint8_t *vbase,
+                                           const float *ksb, const float *vsb, int64_t row_stride, int64_t Hkv,
+                                           int base, int t_end, int lane) {
+  const int c = lane & 7, r = lane >> 3;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int u = 4 * i + r;
+    const bool in = base + u < t_end;
+    const int64_t off = (int64_t)(in ? base + u : 0) * row_stride + 16 * c;
+    cp_async_16(&st.k[u][16 * c], kbase + off, in ? 16u : 0u);
+    cp_async_16(&st.v[u][16 * c], vbase + off, in ? 16u : 0u);
+  }
+  const bool in = base + lane < t_end;
+  const int64_t so = (int64_t)(in ? base + lane : 0) * Hkv;
+  cp_async_4(&st.ks[lane], ksb + so, in ? 4u : 0u);
+  cp_async_4(&st.vs[lane], vsb + so, in ? 4u : 0u);
+}
+
 template <int G>
-__global__ void __launch_bounds__(kAttnWarps * 32, G >= 8 ? 2 : 4) decode_attn_kernel(const AttnArgs a) {
-  __shared__ __align__(16) float qs[G][kD];
-  __shared__ __align__(16) float ps[kAttnWarps][kTokPerIter][G];
+__global__ void __launch_bounds__(kAttnWarps * 32) decode_attn_kernel(const AttnArgs a) {
+  extern __shared__ __align__(16) uint8_t attn_smem[];
+  StepStage *stages = reinterpret_cast<StepStage *>(attn_smem);  // [kAttnWarps][2]
+  float(*qs)[kD] = reinterpret_cast<float(*)[kD]>(attn_smem + sizeof(StepStage) * 2 * kAttnWarps);
+  float(*ps)[kTokPerIter][G] = reinterpret_cast<float(*)[kTokPerIter][G]>(qs + G);
   __shared__ float red_m[kAttnWarps][G], red_l[kAttnWarps][G];
-  __shared__ __align__(16) float red_o[kAttnWarps][G][kD];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bg = blockIdx.x, split = blockIdx.y;
   const int b = bg / a.Hkv, g = bg - b * a.Hkv;
@@ -94,49 +137,41 @@ __global__ void __launch_bounds__(kAttnWarps * 32, G >= 8 ? 2 : 4) decode_attn_k
   const uint8_t *vbase = a.vq + ((int64_t)b * a.S * a.Hkv + g) * kD;
   const float *ksb = a.ks + (int64_t)b * a.S * a.Hkv + g;
   const float *vsb = a.vs + (int64_t)b * a.S * a.Hkv + g;
+  StepStage *my = stages + 2 * warp;
 
-  for (int base = t_begin + warp * kTokPerIter; base < t_end; base += kAttnWarps * kTokPerIter) {
+  int base = t_begin + warp * kTokPerIter;
+  if (base < t_end) issue_step(my[0], kbase, vbase, ksb, vsb, row_stride, a.Hkv, base, t_end, lane);
+  cp_async_commit();
+  for (int it = 0; base < t_end; ++it, base += kAttnWarps * kTokPerIter) {
+    StepStage &st = my[it & 1];
+    const int next = base + kAttnWarps * kTokPerIter;
+    if (next < t_end) issue_step(my[(it + 1) & 1], kbase, vbase, ksb, vsb, row_stride, a.Hkv, next, t_end, lane);
+    cp_async_commit();
+    cp_async_wait<1>();  // this lane's copies of the current step have landed
+    __syncwarp();        // ... and every other lane's
     // ---- scores: lane = token
-    const int t = base + lane;
-    const bool valid = t < t_end;
+    const bool valid = base + lane < t_end;
     float2 acc[G];
 #pragma unroll
     for (int j = 0; j < G; ++j) acc[j] = make_float2(0.f, 0.f);
-    float kscale = 0.f, vscale = 0.f;
-    // the value bytes of the warp's 32 tokens are requested before the key
-    // math, so their latency overlaps it
-    const int n = min(kTokPerIter, t_end - base);
-    uint32_t vw[kTokPerIter];
 #pragma unroll
-    for (int u = 0; u < kTokPerIter; ++u)
-      vw[u] = u < n ? __ldg(reinterpret_cast<const uint32_t *>(vbase + (int64_t)(base + u) * row_stride) + lane) : 0u;
-    if (valid) {
-      const uint4 *krow = reinterpret_cast<const uint4 *>(kbase + (int64_t)t * row_stride);
-      kscale = __ldg(ksb + (int64_t)t * a.Hkv);
-      vscale = __ldg(vsb + (int64_t)t * a.Hkv);
-      // L1-allocating loads: a lane reads its 128-byte key row in eight 16-byte
-      // pieces, so the second half of every 32-byte sector is an L1 hit
-      uint4 kr[8];
+    for (int c = 0; c < 8; ++c) {
+      const uint4 kv = *reinterpret_cast<const uint4 *>(&st.k[lane][16 * c]);
+      const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-      for (int c = 0; c < 8; ++c) kr[c] = __ldg(krow + c);
+      for (int i = 0; i < 4; ++i) {
+        const float2 k01 = e4m3x2_to_float2((uint16_t)(w4[i] & 0xFFFFu));
+        const float2 k23 = e4m3x2_to_float2((uint16_t)(w4[i] >> 16));
+        const int d = c * 16 + i * 4;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 kv = kr[c];
-        const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 k01 = e4m3x2_to_float2((uint16_t)(w4[i] & 0xFFFFu));
-          const float2 k23 = e4m3x2_to_float2((uint16_t)(w4[i] >> 16));
-          const int d = c * 16 + i * 4;
-#pragma unroll
-          for (int j = 0; j < G; ++j) {
-            const float4 qv = *reinterpret_cast<const float4 *>(&qs[j][d]);
-            acc[j] = __ffma2_rn(k01, make_float2(qv.x, qv.y), acc[j]);
-            acc[j] = __ffma2_rn(k23, make_float2(qv.z, qv.w), acc[j]);
-          }
+        for (int j = 0; j < G; ++j) {
+          const float4 qv = *reinterpret_cast<const float4 *>(&qs[j][d]);
+          acc[j] = __ffma2_rn(k01, make_float2(qv.x, qv.y), acc[j]);
+          acc[j] = __ffma2_rn(k23, make_float2(qv.z, qv.w), acc[j]);
         }
       }
     }
+    const float kscale = st.ks[lane], vscale = st.vs[lane];
     // ---- online softmax across the warp's 32 tokens
     float p[G];
 #pragma unroll
@@ -145,7 +180,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, G >= 8 ? 2 : 4) decode_attn_k
       float mt = s;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
-      const float mn = fmaxf(m[j], mt);  // finite: base < t_end, so lane 0's token is valid
+      const float mn = fmaxf(m[j], mt);  // finite: token base (lane 0) is valid
       const float alpha = expf(m[j] - mn);
       const float e = valid ? expf(s - mn) : 0.f;
       float sum = e;
@@ -161,10 +196,11 @@ __global__ void __launch_bounds__(kAttnWarps * 32, G >= 8 ? 2 : 4) decode_attn_k
     for (int j = 0; j < G; ++j) ps[warp][lane][j] = p[j];
     __syncwarp();
     // ---- values: lane = 4 head dimensions
-#pragma unroll
-    for (int u = 0; u < kTokPerIter; ++u) {
-      const float2 v01 = e4m3x2_to_float2((uint16_t)(vw[u] & 0xFFFFu));
-      const float2 v23 = e4m3x2_to_float2((uint16_t)(vw[u] >> 16));
+    const int n = min(kTokPerIter, t_end - base);
+    for (int u = 0; u < n; ++u) {
+      const uint32_t vw = *reinterpret_cast<const uint32_t *>(&st.v[u][4 * lane]);
+      const float2 v01 = e4m3x2_to_float2((uint16_t)(vw & 0xFFFFu));
+      const float2 v23 = e4m3x2_to_float2((uint16_t)(vw >> 16));
 #pragma unroll
       for (int j = 0; j < G; ++j) {
         const float pj = ps[warp][u][j];
@@ -172,10 +208,14 @@ __global__ void __launch_bounds__(kAttnWarps * 32, G >= 8 ? 2 : 4) decode_attn_k
         o[j][1] = __ffma2_rn(v23, make_float2(pj, pj), o[j][1]);
       }
     }
-    __syncwarp();  // ps is rewritten by the next iteration
+    __syncwarp();  // the stage and ps are rewritten by later steps
   }
+  cp_async_wait<0>();
 
-  // ---- merge the four warps, write this split's partial per query head
+  // ---- merge the four warps (the stage buffers are free now: reuse them for
+  // the partial outputs), write this split's partial per query head
+  __syncthreads();
+  float(*red_o)[G][kD] = reinterpret_cast<float(*)[G][kD]>(attn_smem);
 #pragma unroll
   for (int j = 0; j < G; ++j) {
     if (lane == 0) {
@@ -207,27 +247,48 @@ __global__ void __launch_bounds__(kAttnWarps * 32, G >= 8 ? 2 : 4) decode_attn_k
   }
 }
 
-// One warp per (b, query head): merge the splits and round to bf16.
+template <int G>
+constexpr int attn_smem_bytes() {
+  return (int)(sizeof(StepStage) * 2 * kAttnWarps + sizeof(float) * G * kD + sizeof(float) * kAttnWarps * kTokPerIter * G);
+}
+static_assert(sizeof(StepStage) * 2 * kAttnWarps >= sizeof(float) * kAttnWarps * 8 * kD, "partial outputs fit the stages");
+
+// One warp per (b, query head): merge the splits and round to bf16.  The
+// split maxima are read by the lanes in parallel; the weighted sum over the
+// splits keeps eight 16-byte loads in flight per lane.
 __global__ void __launch_bounds__(128) decode_attn_combine_kernel(const float *__restrict__ ws, int32_t BH,
                                                                   int32_t nsplit, uint16_t *__restrict__ out) {
   const int bh = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (bh >= BH) return;
   const float *p = ws + (int64_t)bh * nsplit * kPart;
   float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, p[s * kPart + kD]);
+  for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, p[s * kPart + kD]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.f;
   if (M != -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      const float ms = p[s * kPart + kD];
-      if (ms == -INFINITY) continue;
-      const float w = expf(ms - M);
-      const float4 v = *reinterpret_cast<const float4 *>(p + s * kPart + 4 * lane);
-      acc.x += w * v.x;
-      acc.y += w * v.y;
-      acc.z += w * v.z;
-      acc.w += w * v.w;
-      den += w * p[s * kPart + kD + 1];
+    for (int s0 = 0; s0 < nsplit; s0 += 8) {
+      float4 v[8];
+      float ms[8], ls[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int s = s0 + k;
+        const bool in = s < nsplit;
+        v[k] = in ? *reinterpret_cast<const float4 *>(p + s * kPart + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+        ms[k] = in ? p[s * kPart + kD] : -INFINITY;
+        ls[k] = in ? p[s * kPart + kD + 1] : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (ms[k] == -INFINITY) continue;
+        const float w = expf(ms[k] - M);
+        acc.x += w * v[k].x;
+        acc.y += w * v[k].y;
+        acc.z += w * v[k].z;
+        acc.w += w * v[k].w;
+        den += w * ls[k];
+      }
     }
   }
   const float r = den > 0.f ? 1.f / den : 0.f;
@@ -265,10 +326,29 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const uint16_t *__restri
   if (lane == 0) (which ? vs : ks)[slot] = ts.s;
 }
 
-// Splits of the sequence: about eight blocks per SM in all (two waves of the
-// three or four resident blocks), never chunks shorter than one block's pass.
+int g_attn_ready = 0;
+
+// The stages need more than the default 48 KB of dynamic shared memory.
+fp8bq_status prepare_attention() {
+  if (g_attn_ready) return FP8BQ_OK;
+  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       attn_smem_bytes<1>());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(decode_attn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<2>());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(decode_attn_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<4>());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(decode_attn_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<8>());
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_attention)");
+  g_attn_ready = 1;
+  return FP8BQ_OK;
+}
+
+// Splits of the sequence: about eight blocks per SM in all, never chunks
+// shorter than four passes of a block (a block's fixed costs -- the queries,
+// the pipeline fill, the merge -- stay small against its streaming).
 int attn_splits(int64_t B, int64_t Hkv, int64_t S) {
-  const int64_t max_splits = std::max<int64_t>(1, (S + kChunkQuantum - 1) / kChunkQuantum);
+  const int64_t max_splits = std::max<int64_t>(1, (S + 4 * kChunkQuantum - 1) / (4 * kChunkQuantum));
   const int64_t want = std::max<int64_t>(1, (8 * (int64_t)num_sms() + B * Hkv - 1) / std::max<int64_t>(B * Hkv, 1));
   return (int)std::min(max_splits, want);
 }
@@ -306,14 +386,16 @@ fp8bq_status launch_decode_attention(const void *q, const uint8_t *kq, const flo
   a.chunk = (int32_t)((chunk + kChunkQuantum - 1) / kChunkQuantum * kChunkQuantum);
   a.scale = scale;
   const dim3 grid((unsigned)(B * Hkv), (unsigned)a.nsplit);
+  fp8bq_status st = prepare_attention();
+  if (st != FP8BQ_OK) return st;
   switch (Hq / Hkv) {
-    case 1: decode_attn_kernel<1><<<grid, kAttnWarps * 32, 0, stream>>>(a); break;
-    case 2: decode_attn_kernel<2><<<grid, kAttnWarps * 32, 0, stream>>>(a); break;
-    case 4: decode_attn_kernel<4><<<grid, kAttnWarps * 32, 0, stream>>>(a); break;
-    case 8: decode_attn_kernel<8><<<grid, kAttnWarps * 32, 0, stream>>>(a); break;
+    case 1: decode_attn_kernel<1><<<grid, kAttnWarps * 32, attn_smem_bytes<1>(), stream>>>(a); break;
+    case 2: decode_attn_kernel<2><<<grid, kAttnWarps * 32, attn_smem_bytes<2>(), stream>>>(a); break;
+    case 4: decode_attn_kernel<4><<<grid, kAttnWarps * 32, attn_smem_bytes<4>(), stream>>>(a); break;
+    case 8: decode_attn_kernel<8><<<grid, kAttnWarps * 32, attn_smem_bytes<8>(), stream>>>(a); break;
     default: return FP8BQ_ERR_UNSUPPORTED;
   }
-  fp8bq_status st = check_launch("decode_attention");
+  st = check_launch("decode_attention");
   if (st != FP8BQ_OK) return st;
   const int32_t BH = (int32_t)(B * Hq);
   decode_attn_combine_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, stream>>>(a.ws, BH, a.nsplit,
