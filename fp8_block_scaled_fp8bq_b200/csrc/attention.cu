@@ -104,6 +104,30 @@ __device__ __forceinline__ void issue_step(StepStage &st, const uint8_t *kbase, 
   cp_async_4(&st.vs[lane], vsb + so, in ? 4u : 0u);
 }
 
+// Sum over the 8 lanes of a lane group (lanes 8k .. 8k+7) of v[0..7],
+// reduce-scatter style: afterwards lane l holds the group sum of v[l & 7].
+// Seven shuffles instead of the 24 of eight separate reductions.
+__device__ __forceinline__ float group8_reduce_scatter(const float (&v)[8], int lane) {
+  const bool b2 = lane & 4, b1 = lane & 2, b0 = lane & 1;
+  float w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float send = b2 ? v[k] : v[k + 4];
+    const float keep = b2 ? v[k + 4] : v[k];
+    w[k] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+  float x[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const float send = b1 ? w[k] : w[k + 2];
+    const float keep = b1 ? w[k + 2] : w[k];
+    x[k] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  const float send = b0 ? x[0] : x[1];
+  const float keep = b0 ? x[1] : x[0];
+  return keep + __shfl_xor_sync(0xffffffffu, send, 1);
+}
+
 template <int G>
 __global__ void __launch_bounds__(kAttnWarps * 32) decode_attn_kernel(const AttnArgs a) {
   extern __shared__ __align__(16) uint8_t attn_smem[];
@@ -123,6 +147,27 @@ __global__ void __launch_bounds__(kAttnWarps * 32) decode_attn_kernel(const Attn
     qs[j][d] = __uint_as_float((uint32_t)a.q[((int64_t)b * a.Hq + h0 + j) * kD + d] << 16);
   }
   __syncthreads();
+
+  // G <= 4: lane (grp = lane >> 3, dg = lane & 7) scores token 4 i + grp of
+  // step i = 0..7 over head dimensions [16 dg, +16), with its 16 query
+  // dimensions of each head held in registers; a reduce-scatter across each
+  // 8-lane group then leaves lane l the score of token 4 (l & 7) + (l >> 3).
+  // G = 8: lane l scores token l over all 128 dimensions, queries read from
+  // shared memory.
+  constexpr bool kQReg = G <= 4;
+  const int dg = lane & 7, grp = lane >> 3;
+  float2 qr[kQReg ? G : 1][8];
+  if constexpr (kQReg) {
+#pragma unroll
+    for (int j = 0; j < G; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float4 qv = *reinterpret_cast<const float4 *>(&qs[j][dg * 16 + 4 * e]);
+        qr[j][2 * e] = make_float2(qv.x, qv.y);
+        qr[j][2 * e + 1] = make_float2(qv.z, qv.w);
+      }
+  }
+  const int my_u = kQReg ? 4 * dg + grp : lane;  // the token whose score this lane ends up with
 
   float m[G], l[G];
   float2 o[G][2];  // dimensions 4 lane .. 4 lane + 3
@@ -149,38 +194,65 @@ __global__ void __launch_bounds__(kAttnWarps * 32) decode_attn_kernel(const Attn
     cp_async_commit();
     cp_async_wait<1>();  // this lane's copies of the current step have landed
     __syncwarp();        // ... and every other lane's
-    // ---- scores: lane = token
-    const bool valid = base + lane < t_end;
-    float2 acc[G];
+    // ---- scores
+    const bool valid = base + my_u < t_end;
+    float sc[G];
+    if constexpr (kQReg) {
+      float part[G][8];
 #pragma unroll
-    for (int j = 0; j < G; ++j) acc[j] = make_float2(0.f, 0.f);
+      for (int i = 0; i < 8; ++i) {
+        const uint4 kv = *reinterpret_cast<const uint4 *>(&st.k[4 * i + grp][16 * dg]);
+        const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
+        float2 kf[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint4 kv = *reinterpret_cast<const uint4 *>(&st.k[lane][16 * c]);
-      const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 k01 = e4m3x2_to_float2((uint16_t)(w4[i] & 0xFFFFu));
-        const float2 k23 = e4m3x2_to_float2((uint16_t)(w4[i] >> 16));
-        const int d = c * 16 + i * 4;
+        for (int c = 0; c < 4; ++c) {
+          kf[2 * c] = e4m3x2_to_float2((uint16_t)(w4[c] & 0xFFFFu));
+          kf[2 * c + 1] = e4m3x2_to_float2((uint16_t)(w4[c] >> 16));
+        }
 #pragma unroll
         for (int j = 0; j < G; ++j) {
-          const float4 qv = *reinterpret_cast<const float4 *>(&qs[j][d]);
-          acc[j] = __ffma2_rn(k01, make_float2(qv.x, qv.y), acc[j]);
-          acc[j] = __ffma2_rn(k23, make_float2(qv.z, qv.w), acc[j]);
+          float2 acc = __fmul2_rn(kf[0], qr[j][0]);
+#pragma unroll
+          for (int e = 1; e < 8; ++e) acc = __ffma2_rn(kf[e], qr[j][e], acc);
+          part[j][i] = acc.x + acc.y;
         }
       }
+#pragma unroll
+      for (int j = 0; j < G; ++j) sc[j] = group8_reduce_scatter(part[j], lane);
+    } else {
+      float2 acc[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) acc[j] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 kv = *reinterpret_cast<const uint4 *>(&st.k[lane][16 * c]);
+        const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 k01 = e4m3x2_to_float2((uint16_t)(w4[i] & 0xFFFFu));
+          const float2 k23 = e4m3x2_to_float2((uint16_t)(w4[i] >> 16));
+          const int d = c * 16 + i * 4;
+#pragma unroll
+          for (int j = 0; j < G; ++j) {
+            const float4 qv = *reinterpret_cast<const float4 *>(&qs[j][d]);
+            acc[j] = __ffma2_rn(k01, make_float2(qv.x, qv.y), acc[j]);
+            acc[j] = __ffma2_rn(k23, make_float2(qv.z, qv.w), acc[j]);
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < G; ++j) sc[j] = acc[j].x + acc[j].y;
     }
-    const float kscale = st.ks[lane], vscale = st.vs[lane];
+    const float kscale = st.ks[my_u], vscale = st.vs[my_u];
     // ---- online softmax across the warp's 32 tokens
     float p[G];
 #pragma unroll
     for (int j = 0; j < G; ++j) {
-      const float s = valid ? (acc[j].x + acc[j].y) * kscale * a.scale : -INFINITY;
+      const float s = valid ? sc[j] * kscale * a.scale : -INFINITY;
       float mt = s;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
-      const float mn = fmaxf(m[j], mt);  // finite: token base (lane 0) is valid
+      const float mn = fmaxf(m[j], mt);  // finite: token base is valid
       const float alpha = expf(m[j] - mn);
       const float e = valid ? expf(s - mn) : 0.f;
       float sum = e;
@@ -193,7 +265,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) decode_attn_kernel(const Attn
       p[j] = e * vscale;  // the value scale rides with the probability
     }
 #pragma unroll
-    for (int j = 0; j < G; ++j) ps[warp][lane][j] = p[j];
+    for (int j = 0; j < G; ++j) ps[warp][my_u][j] = p[j];
     __syncwarp();
     // ---- values: lane = 4 head dimensions
     const int n = min(kTokPerIter, t_end - base);
