@@ -63,11 +63,12 @@ fp8bq_status launch_grouped_gemm(const uint8_t *qa, int64_t lda, const float *sa
     return e == cudaSuccess ? FP8BQ_OK : cuda_fail(e, "memset(y)");
   }
   CUtensorMap tA, tB, tY;
-  memset(&tY, 0, sizeof(tY));
   if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qa, (uint64_t)K, (uint64_t)rows, (uint64_t)lda, BK, BM,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_3d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, (uint64_t)K, (uint64_t)N, (uint64_t)E, (uint64_t)K,
-                    (uint64_t)N * (uint64_t)K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+                    (uint64_t)N * (uint64_t)K, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)rows, (uint64_t)ldy * 2, 32, 32,
+                    CU_TENSOR_MAP_SWIZZLE_64B))
     return FP8BQ_ERR_INVALID_ARG;
   fp8bq_status st = prepare_kernel<true, kEpiBf16>();
   if (st != FP8BQ_OK) return st;

@@ -89,8 +89,9 @@ template <int EPI>
 constexpr bool tma_store_epi() { return EPI == kEpiBf16 || EPI == kEpiBf16RowB; }
 
 // Per-warp bf16 staging: dense = 32 rows x 64 columns in the TMA 128-byte
-// swizzle; grouped = 32 rows x 32 columns (64-byte rows, 16-byte chunks XOR
-// ((row >> 1) & 3), conflict-free for both the row writes and the copy-out).
+// swizzle; grouped = 32 rows x 32 columns in the TMA 64-byte swizzle (64-byte
+// rows, 16-byte chunks XOR ((row >> 1) & 3), conflict-free for both the row
+// writes and the warp's masked copy-out).
 template <bool G>
 struct Cfg {
   static constexpr int kEpiBufBytes = G ? 32 * 64 : 32 * 128;
@@ -601,12 +602,15 @@ __device__ __forceinline__ void run_epilogue(const Smem &S, uint32_t tmem_base, 
         }
       }
     } else {
-      // bf16 out, rows masked to the expert: four 32-column chunks; each lane
-      // writes its row into the staging buffer, then the warp copies 8 rows x
-      // 64 bytes per instruction to global memory.
+      // bf16 out in four 32-column chunks through the staging buffer, whose
+      // layout is the TMA's 64-byte swizzle.  A tile wholly inside its expert
+      // leaves with TMA stores; a tile that runs past its expert's last row
+      // is copied by the warp, 8 rows x 64 bytes per instruction, rows masked.
       const int rbase = tl.row0 + quarter * 32;
+      const bool whole = tl.row0 + BM <= tl.row_end;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
+        if (lane == 0) bulk_wait_group_read0();  // an earlier TMA store has left the buffer
         __syncwarp();
         uint8_t *rowp = ebuf + lane * 64;
 #pragma unroll
@@ -619,22 +623,31 @@ __device__ __forceinline__ void run_epilogue(const Smem &S, uint32_t tmem_base, 
           pk.w = pack_bf16x2(a[3].x, a[3].y);
           *reinterpret_cast<uint4 *>(rowp + ((j ^ ((lane >> 1) & 3)) << 4)) = pk;
         }
-        __syncwarp();
         const int n0 = tl.nb * BN + half * 128 + c * 32;
+        if (whole) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && n0 < args.N) {
+            tma_store_2d(tmY, ebuf, n0, rbase);
+            bulk_commit_group();
+          }
+        } else {
+          __syncwarp();
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          const int r = it * 8 + (lane >> 2);
-          const int p = lane & 3;
-          const uint4 v = *reinterpret_cast<const uint4 *>(ebuf + r * 64 + ((p ^ ((r >> 1) & 3)) << 4));
-          const int gr = rbase + r;
-          const int gc = n0 + p * 8;
-          if (gr < tl.row_end && gc < args.N)
-            *reinterpret_cast<uint4 *>(args.y + (int64_t)gr * args.ldy + gc) = v;
+          for (int it = 0; it < 4; ++it) {
+            const int r = it * 8 + (lane >> 2);
+            const int p = lane & 3;
+            const uint4 v = *reinterpret_cast<const uint4 *>(ebuf + r * 64 + ((p ^ ((r >> 1) & 3)) << 4));
+            const int gr = rbase + r;
+            const int gc = n0 + p * 8;
+            if (gr < tl.row_end && gc < args.N)
+              *reinterpret_cast<uint4 *>(args.y + (int64_t)gr * args.ldy + gc) = v;
+          }
         }
       }
     }
   }
-  if constexpr (!G && tma_store_epi<EPI>()) {
+  if constexpr (tma_store_epi<EPI>()) {
     if (lane == 0) bulk_wait_group0();
   }
   __syncwarp();
@@ -665,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
-    if constexpr (!G && tma_store_epi<EPI>()) prefetch_tensormap(&tmY);
+    if constexpr (tma_store_epi<EPI>()) prefetch_tensormap(&tmY);
   }
   if constexpr (G) {
     if (warp == 2) build_schedule(S, args, lane);
