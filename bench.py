@@ -323,6 +323,23 @@ def cpu_baseline_oracle(budget_s=15.0):
             "sample_seconds": round(t_weight + t_rows, 2)}
 
 
+def max_over_ranks(value, device):
+    """The maximum of a per-rank float over all ranks (identity for one rank):
+    the job's time is its slowest replica's."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(work_per_step, steps, world, secs):
+    """Whole-job rate: every replica processes work_per_step per step; secs is
+    the slowest replica's time for `steps` steps."""
+    return world * work_per_step * steps / secs
+
+
 def ours(args):
     import torch.distributed as dist
     import fp8_block_scaled_fp8bq_b200 as fq
@@ -343,13 +360,10 @@ def ours(args):
     step = LayerStep(fq, device)
     with ClockSampler(local) as clk:
         secs, events = timed_steps(step, args.steps, args.warmup, rank_sync)
-    if world > 1:
-        t = torch.tensor([secs], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        secs = float(t.item())
+    secs = max_over_ranks(secs, device)
     K = args.steps
     flops = gemm_flops_step()
-    value = world * flops * K / secs / 1e12
+    value = job_throughput(flops, K, world, secs) / 1e12
 
     # per-row figures from the per-launch events
     def avg_ms(key):
@@ -386,11 +400,8 @@ def ours(args):
     # end to end: host buffers, copies inside the timed region
     Ke = max(1, min(K, 10))
     e2e_s, h2d, d2h = e2e_steps(fq, step, Ke, rank_sync)
-    if world > 1:
-        t = torch.tensor([e2e_s], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
-    e2e = {"value": round(world * flops * Ke / e2e_s / 1e12, 2), "unit": "TFLOP/s",
+    e2e_s = max_over_ranks(e2e_s, device)
+    e2e = {"value": round(job_throughput(flops, Ke, world, e2e_s) / 1e12, 2), "unit": "TFLOP/s",
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": Ke}
 
     if rank == 0:
