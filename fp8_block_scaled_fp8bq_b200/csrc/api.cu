@@ -356,11 +356,11 @@ fp8bq_status fp8bq_decode_attention(const void *q, const uint8_t *kq, const floa
   if (Hkv == 0 || Hq % Hkv != 0) return FP8BQ_ERR_INVALID_ARG;
   const int64_t G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return FP8BQ_ERR_UNSUPPORTED;
-  if (B * Hkv > 0x7fffffffLL) return FP8BQ_ERR_UNSUPPORTED;
+  if (B * Hq > 0x7fffffffLL) return FP8BQ_ERR_UNSUPPORTED;
   if (!q || !o || !aligned(q, 2) || !aligned(o, 8)) return FP8BQ_ERR_INVALID_ARG;
   if (S > 0) {
     if (!kq || !ks || !vq || !vs || !seq_lens || !ws) return FP8BQ_ERR_INVALID_ARG;
-    if (!aligned(kq, 16) || !aligned(vq, 4) || !aligned(ks, 4) || !aligned(vs, 4) || !aligned(seq_lens, 4) ||
+    if (!aligned(kq, 16) || !aligned(vq, 16) || !aligned(ks, 4) || !aligned(vs, 4) || !aligned(seq_lens, 4) ||
         !aligned(ws, 16))
       return FP8BQ_ERR_INVALID_ARG;
   }

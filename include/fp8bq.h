@@ -394,13 +394,19 @@ FP8BQ_API fp8bq_status fp8bq_kv_cache_append(const void *k_new, const void *v_ne
  * query head h reads key/value head h / (Hq / Hkv).
  *   s_t = softmax_scale * sum_d q[b][h][d] dec(kq[b][t][g][d]) ks[b][t][g]
  *   o[b][h][d] = sum_t softmax(s)_t dec(vq[b][t][g][d]) vs[b][t][g]
- * FP32 arithmetic, bf16 out; a sequence with no cached token gives 0.
+ * Both sums run on the tensor cores with FP32 accumulation: the cached codes
+ * enter exactly (as f16), the query scaled per head by a power of two so its
+ * largest |q| lies in [2^14, 2^15) (exact to 2^-28 of that largest element),
+ * and the probabilities times the value scales (relative to the largest value
+ * scale so far) as the sum of two f16 values, a relative rounding of about
+ * 2^-22 per term; the softmax itself is FP32.  bf16 out; a sequence with no
+ * cached token gives 0.
  *   q  bf16 [B][Hq][128];  o  bf16 [B][Hq][128]
  *   ws device workspace of fp8bq_decode_attention_workspace_size(B, Hq, Hkv, S)
  *      bytes (per-split partial results), 16-byte aligned.
- * Requirements: Hq % Hkv == 0 with Hq / Hkv in {1, 2, 4, 8}; kq 16-byte
- * aligned; vq, ks, vs, seq_lens 4 bytes; o 8 bytes.  FP8BQ_ERR_WORKSPACE if ws
- * is too small.
+ * Requirements: Hq % Hkv == 0 with Hq / Hkv in {1, 2, 4, 8}; kq and vq
+ * 16-byte aligned; ks, vs, seq_lens 4 bytes; o 8 bytes.  FP8BQ_ERR_WORKSPACE
+ * if ws is too small.
  */
 FP8BQ_API size_t fp8bq_decode_attention_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t S);
 FP8BQ_API fp8bq_status fp8bq_decode_attention(const void *q, const uint8_t *kq, const float *ks,

@@ -146,6 +146,23 @@ def test_swiglu_validation(L):
     assert gcall(rows=0) == 0
 
 
+def test_decode_attention_validation(L):
+    f = L.fp8bq_decode_attention
+
+    def call(B=2, Hq=8, Hkv=2, S=64, q=FAKE, kq=FAKE, vq=FAKE, ws=FAKE, o=FAKE):
+        return f(q, kq, FAKE, vq, FAKE, FAKE, B, Hq, Hkv, S, 0.1, o, ws, 1 << 20, None)
+    assert call(Hq=6, Hkv=4) == INVALID                                  # Hq % Hkv
+    assert call(Hq=6, Hkv=2) == UNSUPPORTED                              # 3 query heads per key/value head
+    assert call(Hq=32, Hkv=2) == UNSUPPORTED                             # 16 per key/value head
+    assert call(kq=ctypes.c_void_p(0x10004)) == INVALID                  # kq 16-byte alignment
+    assert call(vq=ctypes.c_void_p(0x10004)) == INVALID                  # vq 16-byte alignment
+    assert call(ws=ctypes.c_void_p(0x10008)) == INVALID
+    assert call(o=ctypes.c_void_p(0x10004)) == INVALID
+    assert call(vq=None) == INVALID
+    assert call(B=-1) == INVALID
+    assert call(B=0) == 0 and call(Hq=0) == 0
+
+
 def test_interleave_gate_up_layout():
     """Host-side layout helper of the fused gate+up call: 128-row blocks
     alternate gate block j, up block j (values exact in bf16)."""

@@ -82,6 +82,36 @@ def test_peaked_scores_pick_one_token():
     assert_gemm_close(got, ref, "one-hot")
 
 
+def test_value_scales_spanning_decades():
+    # value vectors whose magnitudes grow and shrink over 2^-12 .. 2^12 along
+    # the sequence: the largest value scale seen so far changes many times
+    B, Hkv, Hq, S = 2, 2, 8, 700
+    k = _bf16((B, S, Hkv, 128), seed=31)
+    v = _bf16((B, S, Hkv, 128), seed=32).float()
+    t = torch.arange(S, dtype=torch.float32)
+    mag = torch.exp2(12.0 * torch.sin(t / 37.0))[None, :, None, None]
+    v = (v * mag).to(torch.bfloat16)
+    kq, ks = oracle.quant_kv(bf16_bits(k), fq.SCALE_FP32)
+    vq, vs = oracle.quant_kv(bf16_bits(v), fq.SCALE_FP32)
+    q = _bf16((B, Hq, 128), seed=33, scale=0.3)
+    got = _run(q, kq, ks, vq, vs, [S, 517], 0.125)
+    ref = oracle.decode_attention(bf16_bits(q), kq, ks, vq, vs, [S, 517], 0.125)
+    assert_gemm_close(got, ref, "value scales over decades")
+
+
+@pytest.mark.parametrize("qscale", [0.0, 1e-30, 1e-6, 1e3, 1e20])
+def test_query_magnitudes(qscale):
+    # the per-head power-of-two scaling of the query keeps tiny and huge
+    # queries exact; a zero query averages the values
+    B, Hkv, Hq, S = 2, 2, 4, 200
+    kq, ks, vq, vs = _cache(B, S, Hkv, seed=41)
+    q = (_bf16((B, Hq, 128), seed=42).float() * qscale).to(torch.bfloat16)
+    q[1, 3] = _bf16((128,), seed=43)  # one head of ordinary size beside them
+    got = _run(q, kq, ks, vq, vs, [S, 150], 0.09)
+    ref = oracle.decode_attention(bf16_bits(q), kq, ks, vq, vs, [S, 150], 0.09)
+    assert_gemm_close(got, ref, "query scale %g" % qscale)
+
+
 @pytest.mark.parametrize("mode", [fq.SCALE_FP32, fq.SCALE_POW2])
 def test_kv_append_bit_exact(mode):
     B, Hkv, S = 4, 8, 40
@@ -125,6 +155,20 @@ def test_llama8b_decode_batch16_context8192():
         ref = oracle.decode_attention(bf16_bits(q[b:b + 1]), kq[b:b + 1], ks[b:b + 1], vq[b:b + 1], vs[b:b + 1],
                                       [lens[b]], scale)
         assert_gemm_close(got[b:b + 1], ref, "llama decode b=%d" % b)
+
+
+@pytest.mark.parametrize("B,Hkv,Hq,S", [(1, 1, 8, 20000),     # one head: many splits of one sequence
+                                         (40, 4, 16, 900)])     # more heads than SMs: whole or few splits
+def test_split_regimes(B, Hkv, Hq, S):
+    kq, ks, vq, vs = _cache(B, S, Hkv, seed=51)
+    q = _bf16((B, Hq, 128), seed=52)
+    lens = [S - (97 * b) % S for b in range(B)]
+    scale = 1.0 / math.sqrt(128.0)
+    got = _run(q, kq, ks, vq, vs, lens, scale)
+    for b in sorted({0, B // 2, B - 1}):
+        ref = oracle.decode_attention(bf16_bits(q[b:b + 1]), kq[b:b + 1], ks[b:b + 1], vq[b:b + 1], vs[b:b + 1],
+                                      [lens[b]], scale)
+        assert_gemm_close(got[b:b + 1], ref, "b=%d" % b)
 
 
 def test_workspace_too_small():
