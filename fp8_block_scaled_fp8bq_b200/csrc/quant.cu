@@ -18,6 +18,8 @@
 
 #include "device.cuh"
 #include "internal.h"
+#include <cuda_bf16.h>
+
 #include "quant.cuh"
 
 namespace fp8bq {
@@ -137,6 +139,18 @@ __device__ __forceinline__ void issue_tile_copy(const TileTensor &T, int64_t nb,
   }
 }
 
+// max |x| of 8 bf16 as a bf16 bit pattern, by packed bf16 maxima of the
+// absolute values (exact for finite values).
+__device__ __forceinline__ uint32_t absmax_bits8_bf16(uint4 v) {
+  auto pair = [](uint32_t a, uint32_t b) {
+    const __nv_bfloat162 m = __hmax2(__habs2(*reinterpret_cast<const __nv_bfloat162 *>(&a)),
+                                     __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&b)));
+    return *reinterpret_cast<const uint32_t *>(&m);
+  };
+  const uint32_t m = pair(pair(v.x, v.y), pair(v.z, v.w));
+  return max(m & 0xFFFFu, m >> 16);
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(256, 3) recalibrate_pipelined_kernel(const __grid_constant__ RecalParams p) {
   __shared__ uint32_t red[8];
@@ -167,7 +181,7 @@ __global__ void __launch_bounds__(256, 3) recalibrate_pipelined_kernel(const __g
     for (int i = 0; i < 8; ++i) v[i] = cur[i * 256 + threadIdx.x];
     uint32_t m = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m = max(m, absmax_bits8(v[i]));
+    for (int i = 0; i < 8; ++i) m = max(m, absmax_bits8_bf16(v[i]));
     m = __reduce_max_sync(0xffffffffu, m);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
     __syncthreads();
