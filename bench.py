@@ -473,7 +473,8 @@ CASES = (["gemm:" + n for n in NAMES] + ["decode:" + n for n in NAMES] + ["cubla
          ["quant_act:4096", "quant_act:14336", "recalibrate:layer", "quant_weight:gate_up", "moe:up", "moe:down",
           "swiglu:gate_up", "moe_swiglu:up", "adamw_recal:layer", "quant_act_t:4096", "quant_act_t:14336",
           "transpose_weight:gate_up", "decode_attn:1x32768", "decode_attn:16x8192", "decode_attn:64x4096",
-          "decode_attn:256x2048"] + ["dgrad:" + n for n in NAMES] + ["wgrad:" + n for n in NAMES])
+          "decode_attn:256x2048", "recalibrate:model"] + ["dgrad:" + n for n in NAMES] +
+         ["wgrad:" + n for n in NAMES])
 
 
 def decode_bytes(M, N, K):
@@ -666,6 +667,17 @@ def run_case(args):
         sw = torch.empty((fq.ceil_div(N, 128), fq.ceil_div(K, 128)), dtype=torch.float32, device=dev)
         fn = lambda: fq.quant_weight(w, mode, q=q, sw=sw)  # noqa: E731
         work, unit = recal_bytes(N, K) / 1e9, "GB/s"
+    elif what == "model":
+        # the whole model's recalibration: 32 layers x 4 weights after one
+        # synthetic update, one call (128 tensors)
+        tensors = []
+        for _, _, w in wl.model_weights_after_step(device=dev):
+            N, K = w.shape
+            tensors.append((w, torch.empty((N, K), dtype=torch.uint8, device=dev),
+                            torch.empty((fq.ceil_div(N, 128), fq.ceil_div(K, 128)), dtype=torch.float32,
+                                        device=dev)))
+        fn = lambda: fq.recalibrate(tensors, mode)  # noqa: E731
+        work, unit = sum(recal_bytes(*w.shape) for w, _, _ in tensors) / 1e9, "GB/s"
     else:
         step = LayerStep(fq, dev, mode=mode)
         fn = lambda: fq.recalibrate(step.recal_list, mode)  # noqa: E731

@@ -107,6 +107,15 @@ def layer_weight_seed(layer, name, seed=0):
     return seed + 1000 * (layer + 1) + 10 * i
 
 
+def model_weights_after_step(layers=LLAMA8B_LAYERS, device="cpu"):
+    """The recalibration workload: every layer's four Llama-8B-shaped weights,
+    each after one synthetic update step.  Yields (layer, name, W bf16 [N, K])."""
+    for layer in range(layers):
+        for name, (N, K) in LLAMA8B_SHAPES.items():
+            seed = layer_weight_seed(layer, name)
+            yield layer, name, weight_step(weights(N, K, seed, device=device), seed + 1)
+
+
 def zipf_probs(E=MOE_EXPERTS, s=MOE_ZIPF_S):
     r = torch.arange(1, E + 1, dtype=torch.float64)
     p = r.pow(-s)

@@ -169,6 +169,44 @@ def test_recalibrate_layer_equals_oracle(mode):
         assert np.array_equal(f32(s).view(np.uint32), osw.view(np.uint32))
 
 
+def test_recalibrate_whole_model_full_size():
+    """The recalibration step at full size: 32 layers x the four Llama-8B-shaped
+    weights (6,979,321,856 parameters) after one synthetic update, requantized
+    in one call with power-of-2 scales.  Every tile is checked for the scale
+    rule (an exact power of two, the smallest with amax <= 448 s) and every
+    element for the encode's error bound; the first, the last and two seeded
+    tiles of every tensor are compared with the oracle bit for bit."""
+    tensors = []
+    for layer, name, w in wl.model_weights_after_step(device="cuda"):
+        N, K = w.shape
+        tensors.append((w, torch.empty((N, K), dtype=torch.uint8, device="cuda"),
+                        torch.empty((N // 128, K // 128), dtype=torch.float32, device="cuda")))
+    assert sum(w.numel() for w, _, _ in tensors) == 6_979_321_856
+    fq.recalibrate(tensors, fq.SCALE_POW2)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(2024)
+    for w, q, s in tensors:
+        N, K = w.shape
+        NB, KB = N // 128, K // 128
+        # every tile: s = 2^e with amax <= 448 s < 2 amax (smallest such e; amax > 0 here)
+        amax = w.float().abs().reshape(NB, 128, KB, 128).amax(dim=(1, 3))
+        mant = s.view(torch.int32) & 0x7FFFFF
+        assert bool((mant == 0).all()) and bool((amax <= 448.0 * s).all()) and bool((448.0 * s < 2 * amax).all())
+        # every element: |dec(q) s - w| <= max(2^-4 |w|, 2^-10 s) (half an E4M3 step, normal or subnormal)
+        for r0 in range(0, N, 4096):
+            rows = slice(r0, min(N, r0 + 4096))
+            se = s[r0 // 128:(rows.stop + 127) // 128].repeat_interleave(128, 0).repeat_interleave(128, 1)
+            dec = q[rows].view(torch.float8_e4m3fn).float() * se
+            wf = w[rows].float()
+            assert bool(((dec - wf).abs() <= torch.maximum(wf.abs() / 16, se / 1024)).all())
+        picks = {(0, 0), (NB - 1, KB - 1)} | {(int(rng.integers(NB)), int(rng.integers(KB))) for _ in range(2)}
+        for nb, kb in sorted(picks):
+            tile = (slice(nb * 128, nb * 128 + 128), slice(kb * 128, kb * 128 + 128))
+            oq, osw = oracle.quant_weight(bf16_bits(w[tile]), fq.SCALE_POW2)
+            assert np.array_equal(u8(q[tile]), oq)
+            assert f32(s[nb, kb]).view(np.uint32) == osw.reshape(-1)[0].view(np.uint32)
+
+
 def test_recalibrate_many_tensors_crosses_launch_chunks():
     tensors = []
     for i in range(300):                                  # > 128 descriptors: several launches
