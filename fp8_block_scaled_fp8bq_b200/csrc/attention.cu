@@ -41,9 +41,9 @@
 //            [0, 1]; the accumulator is rescaled when that largest scale
 //            grows, together with the softmax rescale).  Each weight is split
 //            into two f16 values (high part + rounded remainder) and the MMA
-//            runs on both, so the weights keep about 22 bits.  A thread's value A
-//            fragments pair two tokens' codes at one head dimension (byte
-//            permutes of its two rows' 16-byte pieces).
+//            runs on both, so the weights keep about 22 bits.  A thread's
+//            value A fragments pair two tokens' codes at one head dimension
+//            (byte permutes of its two rows' 16-byte pieces).
 // The four warps' partial (max, sum, output) meet in shared memory and the
 // block writes one partial per query head; a second kernel merges the splits.
 #include <cuda_bf16.h>
