@@ -491,7 +491,8 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const uint16_t *__restri
   const TileScale ts = tile_scale<MODE>(bits_to_amax(am));
   const int64_t slot = ((int64_t)b * S + t) * Hkv + g;
   uint8_t *dst = (which ? vq : kq) + slot * kD;
-  *reinterpret_cast<uint32_t *>(dst + 4 * lane) = encode4<MODE>(x.x, x.y, ts);
+  *reinterpret_cast<uint32_t *>(dst + 4 * lane) =
+      fast_tile<MODE>(ts) ? encode4<MODE, true>(x.x, x.y, ts) : encode4<MODE>(x.x, x.y, ts);
   if (lane == 0) (which ? vs : ks)[slot] = ts.s;
 }
 

@@ -37,6 +37,22 @@ using namespace qdev;
 // columns into X^T, i.e. whole 32-byte sectors.
 constexpr int kTTok = 128, kTCol = 128;
 
+// The 32 tokens of two columns (low and high bf16 halves of w[]) -> codes.
+template <int MODE, bool FAST>
+__device__ __forceinline__ void encode_columns(const uint32_t (&w)[32], const TileScale &t0, const TileScale &t1,
+                                               uint32_t (&ca)[8], uint32_t (&cb)[8]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    // codes of -(x / s), sign bits flipped back (see neg_quotient2)
+    const float2 qa0 = neg_quotient2<MODE, FAST>(make_float2(bf16_lo(w[4 * j]), bf16_lo(w[4 * j + 1])), t0);
+    const float2 qa1 = neg_quotient2<MODE, FAST>(make_float2(bf16_lo(w[4 * j + 2]), bf16_lo(w[4 * j + 3])), t0);
+    const float2 qb0 = neg_quotient2<MODE, FAST>(make_float2(bf16_hi(w[4 * j]), bf16_hi(w[4 * j + 1])), t1);
+    const float2 qb1 = neg_quotient2<MODE, FAST>(make_float2(bf16_hi(w[4 * j + 2]), bf16_hi(w[4 * j + 3])), t1);
+    ca[j] = (e4m3x2(qa0.x, qa0.y) | (e4m3x2(qa1.x, qa1.y) << 16)) ^ 0x80808080u;
+    cb[j] = (e4m3x2(qb0.x, qb0.y) | (e4m3x2(qb1.x, qb1.y) << 16)) ^ 0x80808080u;
+  }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(256) quant_act_t_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
                                                           int64_t ldx, uint8_t *__restrict__ qt, int64_t ldqt,
@@ -74,16 +90,8 @@ __global__ void __launch_bounds__(256) quant_act_t_kernel(const uint16_t *__rest
   const int64_t ka = k0 + 2 * pc, kb = ka + 1;
   const int64_t mt = m0 + tg * 32;  // first token of this lane's 32
   uint32_t ca[8], cb[8];            // 32 codes of column ka, 32 of column kb
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    // codes of -(x / s), sign bits flipped back (see neg_quotient2)
-    const float2 qa0 = neg_quotient2<MODE>(make_float2(bf16_lo(w[4 * j]), bf16_lo(w[4 * j + 1])), t0);
-    const float2 qa1 = neg_quotient2<MODE>(make_float2(bf16_lo(w[4 * j + 2]), bf16_lo(w[4 * j + 3])), t0);
-    const float2 qb0 = neg_quotient2<MODE>(make_float2(bf16_hi(w[4 * j]), bf16_hi(w[4 * j + 1])), t1);
-    const float2 qb1 = neg_quotient2<MODE>(make_float2(bf16_hi(w[4 * j + 2]), bf16_hi(w[4 * j + 3])), t1);
-    ca[j] = (e4m3x2(qa0.x, qa0.y) | (e4m3x2(qa1.x, qa1.y) << 16)) ^ 0x80808080u;
-    cb[j] = (e4m3x2(qb0.x, qb0.y) | (e4m3x2(qb1.x, qb1.y) << 16)) ^ 0x80808080u;
-  }
+  if (fast_tile<MODE>(t0) && fast_tile<MODE>(t1)) encode_columns<MODE, true>(w, t0, t1, ca, cb);
+  else encode_columns<MODE, false>(w, t0, t1, ca, cb);
   if (mt < M) {
     const bool whole = mt + 32 <= M;
     if (ka < K) {

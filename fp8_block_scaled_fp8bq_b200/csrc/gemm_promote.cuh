@@ -431,14 +431,26 @@ __device__ __forceinline__ bool swiglu_epilogue(const Smem &S, const GemmArgs &a
   if (m < tl.row_end) {
     const int64_t col0 = (int64_t)tl.nb * 128 + KEEP;
     uint8_t *q = a.qh + (int64_t)m * a.ldqh + col0;
+    if (qdev::fast_tile<MODE>(ts)) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {  // 16 codes per store
-      uint4 pk;
-      pk.x = qdev::encode4<MODE>(hw[8 * c + 0], hw[8 * c + 1], ts);
-      pk.y = qdev::encode4<MODE>(hw[8 * c + 2], hw[8 * c + 3], ts);
-      pk.z = qdev::encode4<MODE>(hw[8 * c + 4], hw[8 * c + 5], ts);
-      pk.w = qdev::encode4<MODE>(hw[8 * c + 6], hw[8 * c + 7], ts);
-      *reinterpret_cast<uint4 *>(q + 16 * c) = pk;
+      for (int c = 0; c < 4; ++c) {  // 16 codes per store
+        uint4 pk;
+        pk.x = qdev::encode4<MODE, true>(hw[8 * c + 0], hw[8 * c + 1], ts);
+        pk.y = qdev::encode4<MODE, true>(hw[8 * c + 2], hw[8 * c + 3], ts);
+        pk.z = qdev::encode4<MODE, true>(hw[8 * c + 4], hw[8 * c + 5], ts);
+        pk.w = qdev::encode4<MODE, true>(hw[8 * c + 6], hw[8 * c + 7], ts);
+        *reinterpret_cast<uint4 *>(q + 16 * c) = pk;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint4 pk;
+        pk.x = qdev::encode4<MODE>(hw[8 * c + 0], hw[8 * c + 1], ts);
+        pk.y = qdev::encode4<MODE>(hw[8 * c + 2], hw[8 * c + 3], ts);
+        pk.z = qdev::encode4<MODE>(hw[8 * c + 4], hw[8 * c + 5], ts);
+        pk.w = qdev::encode4<MODE>(hw[8 * c + 6], hw[8 * c + 7], ts);
+        *reinterpret_cast<uint4 *>(q + 16 * c) = pk;
+      }
     }
     if (HALF == 0) a.sh[(int64_t)tl.nb * a.ldsh + m] = ts.s;
     if (a.h != nullptr) {

@@ -131,11 +131,20 @@ __device__ __forceinline__ void adamw_tile(const OptTensor &T, const OptParams &
 #pragma unroll
   for (int w = 1; w < 8; ++w) amax = max(amax, red[w]);
   const TileScale ts = tile_scale<MODE>(bits_to_amax(amax));
+  if (fast_tile<MODE>(ts)) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int64_t n = r0 + i;
-    if (kin && n < T.N)
-      *reinterpret_cast<uint32_t *>(T.q + n * T.K + k) = encode4<MODE>(wb[i][0], wb[i][1], ts);
+    for (int i = 0; i < 16; ++i) {
+      const int64_t n = r0 + i;
+      if (kin && n < T.N)
+        *reinterpret_cast<uint32_t *>(T.q + n * T.K + k) = encode4<MODE, true>(wb[i][0], wb[i][1], ts);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int64_t n = r0 + i;
+      if (kin && n < T.N)
+        *reinterpret_cast<uint32_t *>(T.q + n * T.K + k) = encode4<MODE>(wb[i][0], wb[i][1], ts);
+    }
   }
   if (threadIdx.x == 0) T.s[nb * T.KB + kb] = ts.s;
   __syncthreads();  // red[] is reused by the next tile

@@ -73,10 +73,18 @@ __device__ __forceinline__ void quant_tile_vec(const TileTensor &T, int64_t nb, 
 #pragma unroll
   for (int w = 1; w < 8; ++w) m = max(m, red[w]);
   const TileScale ts = tile_scale<MODE>(bits_to_amax(m));
+  if (fast_tile<MODE>(ts)) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int64_t n = nb * 128 + r0 + 16 * i;
-    if (kin && n < T.N) *reinterpret_cast<uint2 *>(T.q + n * T.ldq + k) = encode8<MODE>(v[i], ts);
+    for (int i = 0; i < 8; ++i) {
+      const int64_t n = nb * 128 + r0 + 16 * i;
+      if (kin && n < T.N) *reinterpret_cast<uint2 *>(T.q + n * T.ldq + k) = encode8<MODE, true>(v[i], ts);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t n = nb * 128 + r0 + 16 * i;
+      if (kin && n < T.N) *reinterpret_cast<uint2 *>(T.q + n * T.ldq + k) = encode8<MODE>(v[i], ts);
+    }
   }
   if (t == 0) T.s[nb * T.KB + kb] = ts.s;
   __syncthreads();  // red[] is reused by the next tile
@@ -193,10 +201,18 @@ __global__ void __launch_bounds__(256, 3) recalibrate_pipelined_kernel(const __g
     const int c = threadIdx.x & 15, r0 = threadIdx.x >> 4;
     const int64_t k = kb * 128 + c * 8;
     if (k < T.K) {
+      if (fast_tile<MODE>(ts)) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int64_t n = nb * 128 + r0 + 16 * i;
-        if (n < T.N) *reinterpret_cast<uint2 *>(T.q + n * T.ldq + k) = encode8<MODE>(v[i], ts);
+        for (int i = 0; i < 8; ++i) {
+          const int64_t n = nb * 128 + r0 + 16 * i;
+          if (n < T.N) *reinterpret_cast<uint2 *>(T.q + n * T.ldq + k) = encode8<MODE, true>(v[i], ts);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int64_t n = nb * 128 + r0 + 16 * i;
+          if (n < T.N) *reinterpret_cast<uint2 *>(T.q + n * T.ldq + k) = encode8<MODE>(v[i], ts);
+        }
       }
     }
     if (threadIdx.x == 0) T.s[nb * T.KB + kb] = ts.s;
