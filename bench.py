@@ -71,10 +71,36 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def _strip_comments(src):
+    """C/C++ source without its comments (string and character literals kept),
+    so that a comment-only edit leaves the fingerprint of the code unchanged."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out)
+
+
 def kernel_source_sha():
+    """Fingerprint of the GEMM kernel's code (its sources without comments)."""
     h = hashlib.sha256()
     for f in ("gemm.cu", "gemm_promote.cuh", "device.cuh", "quant.cuh", "raster.cu"):
-        h.update(open(os.path.join(ROOT, "fp8_block_scaled_fp8bq_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "fp8_block_scaled_fp8bq_b200", "csrc", f), encoding="utf-8").read()
+        h.update(_strip_comments(src).encode("utf-8"))
     return h.hexdigest()[:16]
 
 

@@ -2,7 +2,7 @@
 // (cp.async.bulk.tensor) loads and stores, and the tcgen05 tensor-core / TMEM
 // instructions.  Written from the PTX ISA's instruction descriptions.
 //
-// No TMA load here uses .multicast::cluster: every CTA fetches its own tiles.
+// Every CTA fetches its own tiles: no TMA load here is shared across a cluster.
 #pragma once
 
 #include <cuda.h>
