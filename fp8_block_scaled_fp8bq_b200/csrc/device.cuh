@@ -354,7 +354,7 @@ __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_add
 
 // TMA tile load into this CTA's shared memory whose completion is counted on
 // an mbarrier that may live in the peer CTA of the pair (shared::cluster
-// address).  No multicast: each CTA fetches its own tiles.
+// address).  Each CTA fetches its own tiles.
 __device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const CUtensorMap *map, uint32_t bar_cluster_addr,
                                                  int32_t x, int32_t y) {
   asm volatile(

@@ -17,7 +17,7 @@
 // instead of 12 KB, and a stage is 32 KB instead of 48 KB, so the ring is six
 // stages deep.
 //
-// Synchronization (no TMA multicast; each CTA fetches its own tiles):
+// Synchronization (each CTA fetches its own tiles):
 //   full[s]   in CTA 0: CTA 0's producer arms it with both CTAs' bytes; both
 //             CTAs' TMA loads complete on it.
 //   empty[s]  in both CTAs: the MMA's commit arrives on both (multicast).
