@@ -72,9 +72,14 @@ def load_peaks():
 
 
 def _strip_comments(src):
-    """C/C++ source without its comments (string and character literals kept),
-    so that a comment-only edit leaves the fingerprint of the code unchanged."""
+    """C/C++ source without its comments and with every run of whitespace
+    outside string and character literals folded to one space, so that an
+    edit of comments or layout leaves the fingerprint of the code unchanged."""
     out, i, n = [], 0, len(src)
+
+    def space():
+        if out and out[-1] != " ":
+            out.append(" ")
     while i < n:
         c = src[i]
         if c in "\"'":
@@ -86,13 +91,18 @@ def _strip_comments(src):
         elif src.startswith("//", i):
             j = src.find("\n", i)
             i = n if j < 0 else j
+            space()
         elif src.startswith("/*", i):
             j = src.find("*/", i + 2)
             i = n if j < 0 else j + 2
+            space()
+        elif c.isspace():
+            space()
+            i += 1
         else:
             out.append(c)
             i += 1
-    return "".join(out)
+    return "".join(out).strip()
 
 
 def kernel_source_sha():
