@@ -55,9 +55,12 @@ extern "C" {
 fp8bq_status fp8bq_gemm_decode_noalloc(const void *x, int64_t ldx, const uint8_t *qw, int64_t ldw, const float *sw,
                                        void *y, int64_t ldy, int64_t M, int64_t N, int64_t K, int mode,
                                        void *stream) {
-  // The shapes whose workspace would not fit in the fixed scratch are refused
-  // before anything runs.
-  if (M > 0 && N > 0 && K > 0 && fp8bq_gemm_decode_workspace_size(M, N, K) > kNoAllocScratchBytes)
+  // Arguments that need no device are checked before the scratch is looked
+  // up; the shapes whose workspace would not fit in the fixed scratch are
+  // refused before anything runs.
+  if (M < 0 || N < 0 || K < 0 || (mode != FP8BQ_SCALE_FP32 && mode != FP8BQ_SCALE_POW2)) return FP8BQ_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return FP8BQ_OK;
+  if (K > 0 && fp8bq_gemm_decode_workspace_size(M, N, K) > kNoAllocScratchBytes)
     return FP8BQ_ERR_WORKSPACE;
   void *scratch = nullptr;
   fp8bq_status st = scratch_for_current_device(&scratch);

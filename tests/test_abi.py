@@ -163,6 +163,81 @@ def test_decode_attention_validation(L):
     assert call(B=0) == 0 and call(Hq=0) == 0
 
 
+def test_decode_gemm_validation(L):
+    f = L.fp8bq_gemm_decode
+
+    def call(M=16, N=256, K=256, ldx=256, ldw=256, ldy=256, mode=0, x=FAKE, qw=FAKE, y=FAKE):
+        return f(x, ldx, qw, ldw, FAKE, y, ldy, M, N, K, mode, FAKE, 1 << 20, None)
+    assert call(M=-1) == INVALID
+    assert call(mode=3) == INVALID
+    assert call(M=0) == 0 and call(N=0) == 0
+    assert call(y=ctypes.c_void_p(0x10008)) == INVALID                 # y 16-byte alignment
+    assert call(ldy=200) == INVALID                                    # ldy < N
+    assert call(K=200, ldx=200, ldw=208) == UNSUPPORTED                # K % 128
+    assert call(M=257) == UNSUPPORTED                                  # beyond the decode sizes
+    assert call(x=None) == INVALID
+    assert call(ldx=128) == INVALID                                    # ldx < K
+    assert call(qw=ctypes.c_void_p(0x10004)) == INVALID
+    g = L.fp8bq_gemm_decode_noalloc
+    assert g(FAKE, 256, FAKE, 256, FAKE, FAKE, 256, -1, 256, 256, 0, None) == INVALID
+    assert g(FAKE, 256, FAKE, 256, FAKE, FAKE, 256, 0, 256, 256, 0, None) == 0
+
+
+def test_backward_validation(L):
+    qt = L.fp8bq_quant_act_t
+
+    def call_qt(M=256, K=256, ldx=256, ldqt=256, ldst=256, st=FAKE):
+        return qt(FAKE, M, K, ldx, FAKE, ldqt, st, ldst, 0, None)
+    assert call_qt(K=260, ldx=264, ldst=264) == UNSUPPORTED              # K % 8
+    assert call_qt(ldqt=264) == INVALID                                 # ldqt % 16
+    assert call_qt(ldx=128) == INVALID                                  # ldx < K
+    assert call_qt(st=ctypes.c_void_p(0x10004)) == INVALID              # st 16-byte alignment
+    assert call_qt(M=0) == 0 and call_qt(M=-1) == INVALID
+    tw = L.fp8bq_transpose_weight
+
+    def call_tw(N=256, K=256, ldq=256, ldqt=256):
+        return tw(FAKE, N, K, ldq, FAKE, FAKE, ldqt, FAKE, None)
+    assert call_tw(N=200) == UNSUPPORTED                                # N % 16
+    assert call_tw(K=200, ldq=208) == UNSUPPORTED                       # K % 16
+    assert call_tw(ldq=264) == INVALID and call_tw(ldqt=128) == INVALID
+    assert call_tw(N=0) == 0
+    wg = L.fp8bq_gemm_wgrad
+
+    def call_wg(N=256, K=256, M=256, lda=256, ldb=256, ldsa=256, ldsb=256, ldy=256, y=FAKE):
+        return wg(FAKE, lda, FAKE, ldsa, FAKE, ldb, FAKE, ldsb, y, ldy, N, K, M, 0, None)
+    assert call_wg(M=200, lda=208, ldb=208) == UNSUPPORTED              # M % 128
+    assert call_wg(ldy=260) == INVALID                                  # ldy % 8
+    assert call_wg(lda=128) == INVALID                                  # lda < M
+    assert call_wg(ldsb=200) == INVALID                                 # ldsb < K
+    assert call_wg(y=None) == INVALID
+    assert call_wg(N=0) == 0
+
+
+def test_kv_append_and_adamw_validation(L):
+    kv = L.fp8bq_kv_cache_append
+
+    def call_kv(B=2, Hkv=2, S=16, mode=0, k=FAKE):
+        return kv(k, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, B, Hkv, S, mode, None)
+    assert call_kv(mode=5) == INVALID
+    assert call_kv(k=ctypes.c_void_p(0x10004)) == INVALID              # k_new 8-byte alignment
+    assert call_kv(B=-1) == INVALID
+    assert call_kv(B=0) == 0 and call_kv(S=0) == 0
+    ad = L.fp8bq_adamw_recalibrate
+
+    def desc(K=256, grad=FAKE):
+        return fq.AdamWDesc(FAKE, grad, FAKE, FAKE, None, FAKE, FAKE, 128, K)
+
+    def cfg(beta1=0.9, step=1):
+        return fq.AdamWConfig(1e-3, beta1, 0.999, 1e-8, 0.0, step)
+    one = (fq.AdamWDesc * 1)(desc())
+    assert ad(one, 1, ctypes.byref(cfg(beta1=1.0)), 0, None) == INVALID
+    assert ad(one, 1, ctypes.byref(cfg(step=0)), 0, None) == INVALID
+    assert ad(one, 1, None, 0, None) == INVALID
+    assert ad((fq.AdamWDesc * 1)(desc(K=258)), 1, ctypes.byref(cfg()), 0, None) == UNSUPPORTED   # K % 4
+    assert ad((fq.AdamWDesc * 1)(desc(grad=None)), 1, ctypes.byref(cfg()), 0, None) == INVALID
+    assert ad(one, 0, ctypes.byref(cfg()), 0, None) == 0
+
+
 def test_interleave_gate_up_layout():
     """Host-side layout helper of the fused gate+up call: 128-row blocks
     alternate gate block j, up block j (values exact in bf16)."""
