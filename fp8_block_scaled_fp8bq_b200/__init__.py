@@ -64,6 +64,9 @@ SIGNATURES = {
     "fp8bq_version": (ctypes.c_int, []),
     "fp8bq_status_string": (ctypes.c_char_p, [I32]),
     "fp8bq_last_cuda_error": (ctypes.c_char_p, []),
+    "fp8bq_get_last_cuda_error": (I32, [ctypes.POINTER(ctypes.c_int)]),
+    "fp8bq_recalibrate_workspace_size": (SZ, [I32]),
+    "fp8bq_grouped_gemm_workspace_size": (SZ, [I32, I64, I64, I64]),
     "fp8bq_get_device_error": (I32, [ctypes.POINTER(ctypes.c_uint64)]),
     "fp8bq_e4m3_encode": (I32, [P, I64, P, P]),
     "fp8bq_quant_act": (I32, [P, I64, I64, I64, P, I64, P, I64, I32, P]),

@@ -14,8 +14,7 @@ namespace fp8bq {
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-int g_sms[kMaxDevices] = {0};
+std::atomic<int> g_sms[kMaxDevices] = {};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -24,6 +23,24 @@ EncodeTiledFn g_encode = nullptr;
 std::once_flag g_encode_once;
 
 thread_local char g_last_cuda_error[256] = {0};
+thread_local int g_last_cuda_code = 0;  // cudaError_t of this thread's last failing call, 0 once read
+
+TensorMapCache g_maps;
+
+TensorMapKey map_key(int rank, CUtensorMapDataType dtype, const void *base, const uint64_t *dims,
+                     const uint64_t *strides, uint32_t box0, uint32_t box1, CUtensorMapSwizzle swizzle) {
+  TensorMapKey k;
+  memset(&k, 0, sizeof(k));
+  k.base = base;
+  for (int i = 0; i < rank; ++i) k.dims[i] = dims[i];
+  for (int i = 0; i + 1 < rank; ++i) k.strides[i] = strides[i];
+  k.box[0] = box0;
+  k.box[1] = box1;
+  k.rank = rank;
+  k.dtype = (int32_t)dtype;
+  k.swizzle = (int32_t)swizzle;
+  return k;
+}
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -36,18 +53,23 @@ int current_device() {
 }  // namespace
 
 int num_sms() {
-  int d = current_device();
-  if (d < 0 || d >= kMaxDevices) d = 0;
-  if (g_sms[d] == 0) {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) {  // not cached: ask the runtime every time
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0) n = 148;
-    g_sms[d] = n;
+    return n;
   }
-  return g_sms[d];
+  int n = g_sms[d].load(std::memory_order_relaxed);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0) n = 148;
+    g_sms[d].store(n, std::memory_order_relaxed);  // every thread computes the same value
+  }
+  return n;
 }
 
 fp8bq_status cuda_fail(cudaError_t e, const char *what) {
   snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", what, cudaGetErrorString(e));
+  g_last_cuda_code = (int)e;
   return FP8BQ_ERR_CUDA;
 }
 
@@ -68,27 +90,51 @@ bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
   if (g_encode == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_stride_bytes};
+  const TensorMapKey key = map_key(2, dtype, base, dims, strides, box_inner, box_outer, swizzle);
+  if (g_maps.find(key, map)) return true;
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estride[2] = {1, 1};
   CUresult r = g_encode(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estride,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (r != CUDA_SUCCESS) return false;
+  g_maps.insert(key, *map);
+  return true;
 }
 
 bool make_tmap_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
                   CUtensorMapSwizzle swizzle) {
-  CUtensorMap probe;
-  if (!make_tmap_2d(&probe, dtype, base, d0, d1, stride1_bytes, box0, box1, swizzle)) return false;  // loads g_encode
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const TensorMapKey key = map_key(3, dtype, base, dims, strides, box0, box1, swizzle);
+  if (g_maps.find(key, map)) return true;
+  CUtensorMap probe;
+  if (!make_tmap_2d(&probe, dtype, base, d0, d1, stride1_bytes, box0, box1, swizzle)) return false;  // loads g_encode
   cuuint32_t box[3] = {box0, box1, 1};
   cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = g_encode(map, dtype, 3, const_cast<void *>(base), dims, strides, box, estride,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (r != CUDA_SUCCESS) return false;
+  g_maps.insert(key, *map);
+  return true;
+}
+
+fp8bq_status check_decode_args(const void *x, int64_t ldx, const uint8_t *qw, int64_t ldw, const float *sw,
+                               const void *y, int64_t ldy, int64_t M, int64_t N, int64_t K, int mode, bool *work) {
+  *work = false;
+  if (M < 0 || N < 0 || K < 0 || (mode != FP8BQ_SCALE_FP32 && mode != FP8BQ_SCALE_POW2)) return FP8BQ_ERR_INVALID_ARG;
+  if (M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31)) return FP8BQ_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return FP8BQ_OK;
+  if (y == nullptr || ldy < N || !aligned(y, 16) || ldy % 8 != 0) return FP8BQ_ERR_INVALID_ARG;
+  if (K != 0) {
+    if (K % 128 != 0 || M > 256) return FP8BQ_ERR_UNSUPPORTED;
+    if (!x || !qw || !sw || ldx < K || ldw < K) return FP8BQ_ERR_INVALID_ARG;
+    if (!aligned(x, 2) || !aligned(qw, 16) || ldw % 16 != 0 || !aligned(sw, 4)) return FP8BQ_ERR_INVALID_ARG;
+  }
+  *work = true;
+  return FP8BQ_OK;
 }
 
 }  // namespace fp8bq
@@ -159,6 +205,26 @@ const char *fp8bq_status_string(fp8bq_status s) {
 }
 
 const char *fp8bq_last_cuda_error(void) { return g_last_cuda_error; }
+
+fp8bq_status fp8bq_get_last_cuda_error(int *cuda_code) {
+  const int c = g_last_cuda_code;
+  g_last_cuda_code = 0;
+  if (cuda_code) *cuda_code = c;
+  return c != 0 ? FP8BQ_ERR_CUDA : FP8BQ_OK;
+}
+
+size_t fp8bq_recalibrate_workspace_size(int n) {
+  (void)n;
+  return 0;
+}
+
+size_t fp8bq_grouped_gemm_workspace_size(int E, int64_t max_rows, int64_t N, int64_t K) {
+  (void)E;
+  (void)max_rows;
+  (void)N;
+  (void)K;
+  return 0;
+}
 
 fp8bq_status fp8bq_get_device_error(uint64_t *code) {
   unsigned long long v = 0, w = 0;
@@ -246,17 +312,13 @@ size_t fp8bq_gemm_decode_workspace_size(int64_t M, int64_t N, int64_t K) { retur
 fp8bq_status fp8bq_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, int64_t ldw, const float *sw, void *y,
                                int64_t ldy, int64_t M, int64_t N, int64_t K, int mode, void *ws, size_t ws_bytes,
                                void *stream) {
-  if (M < 0 || N < 0 || K < 0 || bad_mode(mode)) return FP8BQ_ERR_INVALID_ARG;
-  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
-  if (M == 0 || N == 0) return FP8BQ_OK;
-  if (y == nullptr || ldy < N || !aligned(y, 16) || ldy % 8 != 0) return FP8BQ_ERR_INVALID_ARG;
+  bool work = false;
+  const fp8bq_status st = check_decode_args(x, ldx, qw, ldw, sw, y, ldy, M, N, K, mode, &work);
+  if (st != FP8BQ_OK || !work) return st;
   if (K == 0) {
     cudaError_t e = cudaMemset2DAsync(y, (size_t)ldy * 2, 0, (size_t)N * 2, (size_t)M, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FP8BQ_OK : cuda_fail(e, "memset(y)");
   }
-  if (K % 128 != 0 || M > 256) return FP8BQ_ERR_UNSUPPORTED;
-  if (!x || !qw || !sw || ldx < K || ldw < K) return FP8BQ_ERR_INVALID_ARG;
-  if (!aligned(x, 2) || !aligned(qw, 16) || ldw % 16 != 0 || !aligned(sw, 4)) return FP8BQ_ERR_INVALID_ARG;
   return launch_gemm_decode(x, ldx, qw, ldw, sw, y, ldy, M, N, K, mode, ws, ws_bytes,
                             static_cast<cudaStream_t>(stream));
 }

@@ -360,29 +360,20 @@ Plan make_plan(int64_t M, int64_t N, int64_t K) {
   return p;
 }
 
-int g_dready[3][64] = {{0}};
-
 template <int NT>
 fp8bq_status launch_decode_nt(const CUtensorMap &tW, const CUtensorMap &tX, const CUtensorMap &tS,
-                              const DecodeArgs &a, cudaStream_t stream, int slot) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 64) dev = 0;
-  int &ready = g_dready[slot][dev];
-  if (ready == -1) return FP8BQ_ERR_UNSUPPORTED;
-  if (ready == 0) {
+                              const DecodeArgs &a, cudaStream_t stream) {
+  static DeviceOnce once;  // one per instantiation
+  const fp8bq_status ready = once.get([](int) {
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, decode_kernel<NT>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, decode_kernel<NT>);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(decode)");
-    if (fa.numRegs != kDLaunchRegs) {
-      ready = -1;
-      return FP8BQ_ERR_UNSUPPORTED;
-    }
+    if (fa.numRegs != kDLaunchRegs) return FP8BQ_ERR_UNSUPPORTED;
     e = cudaFuncSetAttribute(decode_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, DCfg<NT>::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
-    ready = 1;
-  }
+    return FP8BQ_OK;
+  });
+  if (ready != FP8BQ_OK) return ready;
   decode_kernel<NT><<<a.G, kDThreads, DCfg<NT>::kSmemBytes, stream>>>(tW, tX, tS, a);
   fp8bq_status st = check_launch("gemm_decode");
   if (st != FP8BQ_OK) return st;
@@ -454,9 +445,9 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
   a.y = static_cast<uint16_t *>(y);
   a.ldy = ldy;
   switch (p.NT) {
-    case 16: return launch_decode_nt<16>(tW, tX, tS, a, stream, 0);
-    case 32: return launch_decode_nt<32>(tW, tX, tS, a, stream, 1);
-    default: return launch_decode_nt<64>(tW, tX, tS, a, stream, 2);
+    case 16: return launch_decode_nt<16>(tW, tX, tS, a, stream);
+    case 32: return launch_decode_nt<32>(tW, tX, tS, a, stream);
+    default: return launch_decode_nt<64>(tW, tX, tS, a, stream);
   }
 }
 

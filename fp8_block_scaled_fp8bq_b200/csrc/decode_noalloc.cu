@@ -25,7 +25,6 @@ static __device__ __align__(256) uint8_t g_decode_scratch[kNoAllocScratchBytes];
 // Device address of g_decode_scratch per device.  In host code the array's
 // name only stands in for the symbol, so the address comes from
 // cudaGetSymbolAddress, once per device, with that device current.
-constexpr int kMaxDevices = 64;
 void *g_scratch_addr[kMaxDevices] = {nullptr};
 std::mutex g_scratch_mutex;
 
@@ -55,15 +54,17 @@ extern "C" {
 fp8bq_status fp8bq_gemm_decode_noalloc(const void *x, int64_t ldx, const uint8_t *qw, int64_t ldw, const float *sw,
                                        void *y, int64_t ldy, int64_t M, int64_t N, int64_t K, int mode,
                                        void *stream) {
-  // Arguments that need no device are checked before the scratch is looked
-  // up; the shapes whose workspace would not fit in the fixed scratch are
-  // refused before anything runs.
-  if (M < 0 || N < 0 || K < 0 || (mode != FP8BQ_SCALE_FP32 && mode != FP8BQ_SCALE_POW2)) return FP8BQ_ERR_INVALID_ARG;
-  if (M == 0 || N == 0) return FP8BQ_OK;
+  // Every argument check of fp8bq_gemm_decode comes first (so a bad pointer
+  // or an unsupported size is reported as such), then the shapes whose
+  // workspace would not fit in the fixed scratch are refused; nothing runs
+  // before these checks pass.
+  bool work = false;
+  fp8bq_status st = check_decode_args(x, ldx, qw, ldw, sw, y, ldy, M, N, K, mode, &work);
+  if (st != FP8BQ_OK || !work) return st;
   if (K > 0 && fp8bq_gemm_decode_workspace_size(M, N, K) > kNoAllocScratchBytes)
     return FP8BQ_ERR_WORKSPACE;
   void *scratch = nullptr;
-  fp8bq_status st = scratch_for_current_device(&scratch);
+  st = scratch_for_current_device(&scratch);
   if (st != FP8BQ_OK) return st;
   return fp8bq_gemm_decode(x, ldx, qw, ldw, sw, y, ldy, M, N, K, mode, scratch, kNoAllocScratchBytes, stream);
 }

@@ -307,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-int g_nready[64] = {0};
+DeviceOnce g_native_once;
 
 }  // namespace
 
@@ -324,23 +324,16 @@ fp8bq_status launch_gemm_native(const uint8_t *qa, int64_t lda, const float *sa,
       !make_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M, (uint64_t)ldy * 2, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_64B))
     return FP8BQ_ERR_INVALID_ARG;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (g_nready[dev] == -1) return FP8BQ_ERR_UNSUPPORTED;
-  if (g_nready[dev] == 0) {
+  const fp8bq_status ready = g_native_once.get([](int) {
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, gemm_native_kernel);
+    cudaError_t e = cudaFuncGetAttributes(&fa, gemm_native_kernel);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(gemm_native)");
-    if (fa.numRegs != kLaunchRegs) {
-      g_nready[dev] = -1;
-      return FP8BQ_ERR_UNSUPPORTED;
-    }
+    if (fa.numRegs != kLaunchRegs) return FP8BQ_ERR_UNSUPPORTED;
     e = cudaFuncSetAttribute(gemm_native_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm_native)");
-    g_nready[dev] = 1;
-  }
+    return FP8BQ_OK;
+  });
+  if (ready != FP8BQ_OK) return ready;
   NativeArgs a;
   a.sa = sa;
   a.sw = sw;

@@ -327,19 +327,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-int g_pready[2][64] = {};         // [tile shape][device]: 0 unknown, 1 ready, -1 refused
-int g_pmax_clusters[2][64] = {};
+std::atomic<int> g_pmax_clusters[2][kMaxDevices] = {};  // [tile shape][device], set once the kernel is ready
 
+// Per-device set-up of the pair kernel: register count, shared-memory opt-in
+// and the number of clusters of two that fit at once.
 template <int PBN>
-bool pair_ready(int dev) {
-  constexpr int si = PBN == 256 ? 0 : 1;
-  if (g_pready[si][dev] == 0) {
+fp8bq_status pair_ready() {
+  static DeviceOnce once;  // one per instantiation
+  return once.get([](int dev) {
+    constexpr int si = PBN == 256 ? 0 : 1;
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, gemm_pair_kernel<PBN>) != cudaSuccess || fa.numRegs != kLaunchRegs ||
         cudaFuncSetAttribute(gemm_pair_kernel<PBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              PairCfg<PBN>::kSmemBytes) != cudaSuccess) {
-      g_pready[si][dev] = -1;
-      return false;
+      cudaGetLastError();
+      return FP8BQ_ERR_UNSUPPORTED;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 128);
@@ -355,22 +357,22 @@ bool pair_ready(int dev) {
     int nclusters = 0;
     if (cudaOccupancyMaxActiveClusters(&nclusters, gemm_pair_kernel<PBN>, &cfg) != cudaSuccess || nclusters < 1) {
       cudaGetLastError();
-      g_pready[si][dev] = -1;
-      return false;
+      return FP8BQ_ERR_UNSUPPORTED;
     }
-    g_pmax_clusters[si][dev] = nclusters;
-    g_pready[si][dev] = 1;
-  }
-  return g_pready[si][dev] == 1;
+    g_pmax_clusters[si][dev].store(nclusters, std::memory_order_relaxed);
+    return FP8BQ_OK;
+  });
 }
 
 template <int PBN>
 fp8bq_status launch_pair(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
                          int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                          cudaStream_t stream) {
+  const fp8bq_status ready = pair_ready<PBN>();
+  if (ready != FP8BQ_OK) return ready;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || !pair_ready<PBN>(dev))
-    return FP8BQ_ERR_UNSUPPORTED;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   CUtensorMap tA, tB, tY;
   if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qa, (uint64_t)K, (uint64_t)M, (uint64_t)lda, BK, CBM,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -392,7 +394,8 @@ fp8bq_status launch_pair(const uint8_t *qa, int64_t lda, const float *sa, int64_
   choose_raster(M, N, K, PBM, PBN, &a.band, &a.n_major);
   const int64_t tiles = (int64_t)a.num_m * a.num_n;
   const int si = PBN == 256 ? 0 : 1;
-  const int pairs = (int)std::min<int64_t>(tiles, std::min(g_pmax_clusters[si][dev], num_sms() / 2));
+  const int pairs = (int)std::min<int64_t>(
+      tiles, std::min(g_pmax_clusters[si][dev].load(std::memory_order_relaxed), num_sms() / 2));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
   cfg.blockDim = dim3(kThreads);
@@ -405,18 +408,14 @@ fp8bq_status launch_pair(const uint8_t *qa, int64_t lda, const float *sa, int64_
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<PBN>, tA, tB, tY, a);
+  e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<PBN>, tA, tB, tY, a);
   if (e != cudaSuccess) return cuda_fail(e, "gemm_pair launch");
   return check_launch("gemm_pair");
 }
 
 }  // namespace
 
-bool pair_gemm_available() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  return pair_ready<256>(dev) && pair_ready<128>(dev);
-}
+bool pair_gemm_available() { return pair_ready<256>() == FP8BQ_OK && pair_ready<128>() == FP8BQ_OK; }
 
 cudaError_t take_device_error_pair(unsigned long long *v) { return take_tu_device_error(v); }
 

@@ -726,31 +726,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Per-device one-time setup: opt in to the large shared-memory carve-up and
 // confirm that the kernel was built with the register count the setmaxnreg
 // split assumes (a smaller count would make setmaxnreg.inc wait forever).
-int g_ready[2][4][64] = {};  // [grouped][epilogue][device]: 0 unknown, 1 ready, -1 refused
-
 template <bool G, int EPI>
 fp8bq_status prepare_kernel() {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 64) dev = 0;
-  int &ready = g_ready[G ? 1 : 0][EPI][dev];
-  if (ready == 1) return FP8BQ_OK;
-  if (ready == -1) return FP8BQ_ERR_UNSUPPORTED;
-  cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, gemm_promote_kernel<G, EPI>);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(gemm)");
-  if (fa.numRegs != kLaunchRegs) {
-    ready = -1;
-    return FP8BQ_ERR_UNSUPPORTED;
-  }
-  e = cudaFuncSetAttribute(gemm_promote_kernel<G, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Cfg<G>::kSmemBytes);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
-  ready = 1;
-  return FP8BQ_OK;
+  static DeviceOnce once;  // one per instantiation
+  return once.get([](int) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, gemm_promote_kernel<G, EPI>);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(gemm)");
+    if (fa.numRegs != kLaunchRegs) return FP8BQ_ERR_UNSUPPORTED;
+    e = cudaFuncSetAttribute(gemm_promote_kernel<G, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg<G>::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
+    return FP8BQ_OK;
+  });
 }
-
 
 }  // namespace
 }  // namespace fp8bq

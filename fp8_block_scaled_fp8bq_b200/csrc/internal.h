@@ -5,6 +5,12 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <unordered_map>
+
 #include "../../include/fp8bq.h"
 
 namespace fp8bq {
@@ -13,11 +19,99 @@ namespace fp8bq {
 // offsets and the tile prefix of all experts in shared memory).
 constexpr int kMaxExperts = 1024;
 
+// Highest device ordinal + 1 for which the library keeps per-device state.
+constexpr int kMaxDevices = 64;
+
 // Number of SMs of the current device (cached per device).
 int num_sms();
 
 // Record the failing CUDA call for diagnostics and map it to FP8BQ_ERR_CUDA.
 fp8bq_status cuda_fail(cudaError_t e, const char *what);
+
+// The result of a per-device one-time set-up (a kernel attribute opt-in, a
+// register-count check, a symbol lookup), safe to call from several host
+// threads: the first caller on a device runs `setup(dev)` under a mutex,
+// later callers read the cached status without locking.  Definite answers
+// (FP8BQ_OK, FP8BQ_ERR_UNSUPPORTED) are cached; a failing CUDA call is not, so
+// the next call tries again.  A device ordinal outside [0, kMaxDevices) is
+// FP8BQ_ERR_UNSUPPORTED.
+class DeviceOnce {
+ public:
+  // For the current device.
+  template <class F>
+  fp8bq_status get(F &&setup) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    return get_for(dev, setup);
+  }
+
+  template <class F>
+  fp8bq_status get_for(int dev, F &&setup) {
+    if (dev < 0 || dev >= kMaxDevices) return FP8BQ_ERR_UNSUPPORTED;
+    int v = state_[dev].load(std::memory_order_acquire);
+    if (v != 0) return static_cast<fp8bq_status>(v - 1);
+    std::lock_guard<std::mutex> lock(mutex_);
+    v = state_[dev].load(std::memory_order_relaxed);
+    if (v != 0) return static_cast<fp8bq_status>(v - 1);
+    const fp8bq_status st = setup(dev);
+    if (st == FP8BQ_OK || st == FP8BQ_ERR_UNSUPPORTED) state_[dev].store(st + 1, std::memory_order_release);
+    return st;
+  }
+
+ private:
+  std::atomic<int> state_[kMaxDevices] = {};  // 0: not yet; else status + 1
+  std::mutex mutex_;
+};
+
+// Encoded TMA descriptors, keyed by everything that goes into one.  A
+// descriptor holds nothing beyond its arguments, so an entry stays valid for
+// as long as a caller passes the same pointer and shape.  Guarded by a mutex;
+// emptied when it holds kCapacity entries.
+struct TensorMapKey {
+  const void *base;
+  uint64_t dims[3], strides[2];
+  uint32_t box[2];
+  int32_t rank, dtype, swizzle, pad;  // no implicit padding: compared and hashed as bytes
+};
+static_assert(sizeof(TensorMapKey) == 72, "TensorMapKey has no padding");
+
+class TensorMapCache {
+ public:
+  static constexpr size_t kCapacity = 4096;
+  bool find(const TensorMapKey &k, CUtensorMap *out) {
+    std::lock_guard<std::mutex> lock(mutex_);
+    auto it = maps_.find(Bytes(k));
+    if (it == maps_.end()) return false;
+    *out = it->second;
+    return true;
+  }
+  void insert(const TensorMapKey &k, const CUtensorMap &m) {
+    std::lock_guard<std::mutex> lock(mutex_);
+    if (maps_.size() >= kCapacity) maps_.clear();
+    maps_[Bytes(k)] = m;
+  }
+  size_t size() {
+    std::lock_guard<std::mutex> lock(mutex_);
+    return maps_.size();
+  }
+
+ private:
+  struct Bytes {
+    unsigned char b[sizeof(TensorMapKey)];
+    explicit Bytes(const TensorMapKey &k) { memcpy(b, &k, sizeof(b)); }
+    bool operator==(const Bytes &o) const { return memcmp(b, o.b, sizeof(b)) == 0; }
+  };
+  struct Hash {
+    size_t operator()(const Bytes &k) const {
+      uint64_t h = 1469598103934665603ull;  // FNV-1a
+      for (unsigned char c : k.b) h = (h ^ c) * 1099511628211ull;
+      return (size_t)h;
+    }
+  };
+  std::unordered_map<Bytes, CUtensorMap, Hash> maps_;
+  std::mutex mutex_;
+};
 
 // Check the last launch.
 fp8bq_status check_launch(const char *what);
@@ -62,6 +156,10 @@ fp8bq_status launch_gemm_native(const uint8_t *qa, int64_t lda, const float *sa,
                                 int64_t ldw, const float *sw, void *y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                                 cudaStream_t stream);
 size_t decode_workspace_size(int64_t M, int64_t N, int64_t K);
+// Argument checks of fp8bq_gemm_decode (no device access).  *work is false for
+// the no-op sizes (M == 0 or N == 0) and for any error.
+fp8bq_status check_decode_args(const void *x, int64_t ldx, const uint8_t *qw, int64_t ldw, const float *sw,
+                               const void *y, int64_t ldy, int64_t M, int64_t N, int64_t K, int mode, bool *work);
 fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, int64_t ldw, const float *sw, void *y,
                                 int64_t ldy, int64_t M, int64_t N, int64_t K, int mode, void *ws, size_t ws_bytes,
                                 cudaStream_t stream);

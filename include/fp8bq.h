@@ -35,7 +35,9 @@
  *     The library allocates no device memory.
  *   - Every call is asynchronous and ordered on `stream` (a cudaStream_t; NULL is
  *     the legacy default stream).  No call synchronizes the host, except
- *     fp8bq_get_device_error.  Calls are safe from several host threads.
+ *     fp8bq_get_device_error.  Calls are safe from several host threads: the
+ *     library's host state (per-device set-up results, SM counts, encoded TMA
+ *     descriptors) is guarded by mutexes or atomics.
  *   - Leading dimensions (ld*) count elements, not bytes.
  *   - Status: FP8BQ_OK means the work was launched.  Arguments are checked
  *     before anything is launched; a failed check launches nothing.
@@ -89,6 +91,14 @@ FP8BQ_API const char *fp8bq_status_string(fp8bq_status status);
  * library ("" if none); valid until the thread's next failing call.
  */
 FP8BQ_API const char *fp8bq_last_cuda_error(void);
+
+/*
+ * Status of this host thread's last failing CUDA call inside the library:
+ * FP8BQ_ERR_CUDA if one failed since the previous call of this function
+ * (*cuda_code, if not NULL, receives its cudaError_t value), FP8BQ_OK (and 0)
+ * otherwise.  Reading clears it; fp8bq_last_cuda_error keeps the text.
+ */
+FP8BQ_API fp8bq_status fp8bq_get_last_cuda_error(int *cuda_code);
 
 /*
  * Reads and clears the device error word of the current device (this call
@@ -152,6 +162,14 @@ typedef struct {
  * fp8bq_quant_weight on each tensor.  Tensors must not overlap.
  */
 FP8BQ_API fp8bq_status fp8bq_recalibrate(const fp8bq_weight_desc *descs, int n, int mode, void *stream);
+
+/*
+ * Device workspace fp8bq_recalibrate needs for n tensors: always 0.  The
+ * descriptors travel inside the launch parameters (up to 128 tensors per
+ * launch), so the call takes no workspace argument; this query exists so that
+ * callers written against a workspace-taking interface can size theirs.
+ */
+FP8BQ_API size_t fp8bq_recalibrate_workspace_size(int n);
 
 /*
  * Block-scaled FP8 GEMM, Y = X W^T ("Technical breakthrough": linear layers in
@@ -260,6 +278,13 @@ FP8BQ_API fp8bq_status fp8bq_grouped_gemm(const uint8_t *qa, int64_t lda, const 
                                 const int32_t *offsets, int E, int64_t total_rows,
                                 int64_t N, int64_t K, void *y, int64_t ldy,
                                 int mode, void *stream);
+
+/*
+ * Device workspace fp8bq_grouped_gemm needs: always 0.  The tile scheduler
+ * builds its per-expert tables in each CTA's shared memory from `offsets`, so
+ * the call takes no workspace argument.
+ */
+FP8BQ_API size_t fp8bq_grouped_gemm_workspace_size(int E, int64_t max_rows, int64_t N, int64_t K);
 
 /*
  * Gate+up projection of a gated (SwiGLU) feed-forward block with the

@@ -29,9 +29,23 @@ def L():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for n in ("fp8bq_quant_act", "fp8bq_quant_weight", "fp8bq_recalibrate", "fp8bq_gemm",
-              "fp8bq_grouped_gemm", "fp8bq_gemm_decode"):
+    # the hot path's entry points and their size queries and diagnostics
+    for n in ("fp8bq_quant_act", "fp8bq_quant_weight", "fp8bq_recalibrate", "fp8bq_recalibrate_workspace_size",
+              "fp8bq_gemm", "fp8bq_gemm_decode", "fp8bq_gemm_decode_workspace_size", "fp8bq_grouped_gemm",
+              "fp8bq_grouped_gemm_workspace_size", "fp8bq_status_string", "fp8bq_get_last_cuda_error"):
         assert n in names
+
+
+def test_workspace_queries_and_last_error(L):
+    # recalibration and the grouped GEMM keep their tables in launch parameters
+    # and shared memory: no workspace
+    assert L.fp8bq_recalibrate_workspace_size(128) == 0
+    assert L.fp8bq_grouped_gemm_workspace_size(128, 32768, 1536, 2048) == 0
+    code = ctypes.c_int(-1)
+    assert L.fp8bq_get_last_cuda_error(ctypes.byref(code)) in (0, 3)
+    # reading clears it
+    assert L.fp8bq_get_last_cuda_error(ctypes.byref(code)) == 0 and code.value == 0
+    assert L.fp8bq_get_last_cuda_error(None) == 0
 
 
 def test_every_declared_symbol_is_exported(L):
