@@ -77,6 +77,8 @@ def lib():
         L.o_gemm_wgrad_rows.argtypes = [P, I64, P, I64, P, I64, P, I64, I64, I64, I64, P, I64, P]
         L.o_decode_attention.restype = None
         L.o_decode_attention.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, I64, ctypes.c_double, P]
+        L.o_prefill_attention.restype = None
+        L.o_prefill_attention.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64, I64, ctypes.c_double, P, I64, P, P]
         L.o_adamw_step.restype = None
         L.o_adamw_step.argtypes = [P, P, P, P, I64, ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                                    ctypes.c_float, I64]
@@ -392,3 +394,33 @@ def decode_attention(q_bits, kq, ks, vq, vs, lens, scale):
     lib().o_decode_attention(_p(q), _p(kq), _p(ks), _p(vq), _p(vs), _p(lens), B, Hq, Hkv, S, D, float(scale),
                              _p(out))
     return out
+
+
+def prefill_attention(qq, qs, kq, ks, vq, vs, lens, scale, rows=None, want_mag=False):
+    """Causal attention of FP8 queries over FP8 keys/values of the same
+    sequences (see o_prefill_attention).  qq [B, S, Hq, D] codes, qs [B, S, Hq];
+    kq, vq [B, S, Hkv, D], ks, vs [B, S, Hkv]; lens [B].  rows: optional flat
+    query indices b * S + i.  Returns float64 [R, Hq, D] (and the term
+    magnitudes sum_j p_j |v_j| if want_mag)."""
+    qq = _c(qq, np.uint8)
+    kq = _c(kq, np.uint8)
+    vq = _c(vq, np.uint8)
+    qs = _c(qs, np.float32)
+    ks = _c(ks, np.float32)
+    vs = _c(vs, np.float32)
+    lens = _c(np.asarray(lens, dtype=np.int32), np.int32)
+    B, S, Hq, D = qq.shape
+    Hkv = kq.shape[2]
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    if rows is None:
+        r, R = None, B * S
+    else:
+        r = _c(np.asarray(rows, dtype=np.int64), np.int64)
+        R = r.size
+    out = np.empty((R, Hq, D), dtype=np.float64)
+    mag = np.empty((R, Hq, D), dtype=np.float64) if want_mag else None
+    lib().o_prefill_attention(_p(qq), _p(qs), _p(kq), _p(ks), _p(vq), _p(vs), _p(lens), B, S, Hq, Hkv, D,
+                              float(scale), None if r is None else _p(r), R, _p(out),
+                              None if mag is None else _p(mag))
+    return (out, mag) if want_mag else out

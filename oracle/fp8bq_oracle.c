@@ -539,6 +539,68 @@ O_API void o_decode_attention(const uint16_t *q, const uint8_t *kq, const float 
 }
 
 /*
+ * Causal (prefill) attention over FP8 queries, keys and values: the "FP8 KV
+ * cache and attention" of section "Real-world performance gains", for the
+ * many-query case.  Every query, key and value head vector (D = 128) is one
+ * 1x128 tile of section "Technical breakthrough": E4M3 codes and one scale.
+ * Query row i of sequence b (i < lens[b]) attends the keys j <= i of its own
+ * sequence; query head h reads key/value head h / (Hq / Hkv):
+ *   s_j   = scale * qs[b,i,h] * ks[b,j,g] * sum_d dec(qq[b,i,h,d]) dec(kq[b,j,g,d])
+ *   p_j   = exp(s_j - max_j s) / sum_j exp(s_j - max_j s)
+ *   o[d]  = sum_j p_j * vs[b,j,g] * dec(vq[b,j,g,d])
+ * everything in double.  Rows i >= lens[b] are 0.  When `mag` is not NULL it
+ * also receives sum_j p_j |vs[b,j,g] dec(vq[b,j,g,d])|, the size of the terms
+ * of o[d] (an error bound of a kernel that rounds the weights p_j is
+ * proportional to it).
+ * rows: the query rows to compute (indices b * S + i), or NULL for all; out
+ * (and mag) are [R][Hq][D] for R = nrows (or B * S).
+ */
+O_API void o_prefill_attention(const uint8_t *qq, const float *qs, const uint8_t *kq, const float *ks,
+                               const uint8_t *vq, const float *vs, const int32_t *lens, int64_t B, int64_t S,
+                               int64_t Hq, int64_t Hkv, int64_t D, double scale, const int64_t *rows, int64_t nrows,
+                               double *out, double *mag)
+{
+    const int64_t R = rows ? nrows : B * S;
+    int64_t rh;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (rh = 0; rh < R * Hq; ++rh) {
+        const int64_t r = rh / Hq, h = rh % Hq, g = h / (Hq / Hkv);
+        const int64_t bi = rows ? rows[r] : r;
+        const int64_t b = bi / S, i = bi % S;
+        int64_t L = lens[b] < S ? lens[b] : S, j, d;
+        double mx = -HUGE_VAL, den = 0.0;
+        double *o = out + rh * D;
+        double *m = mag ? mag + rh * D : NULL;
+        double *sc;
+        for (d = 0; d < D; ++d) {
+            o[d] = 0.0;
+            if (m) m[d] = 0.0;
+        }
+        if (i >= L) continue;
+        sc = (double *)malloc(sizeof(double) * (size_t)(i + 1));
+        for (j = 0; j <= i; ++j) {
+            const uint8_t *qv = qq + ((b * S + i) * Hq + h) * D;
+            const uint8_t *kv = kq + ((b * S + j) * Hkv + g) * D;
+            double dot = 0.0;
+            for (d = 0; d < D; ++d) dot += o_e4m3_decode(qv[d]) * o_e4m3_decode(kv[d]);
+            sc[j] = scale * (double)qs[(b * S + i) * Hq + h] * (double)ks[(b * S + j) * Hkv + g] * dot;
+            if (sc[j] > mx) mx = sc[j];
+        }
+        for (j = 0; j <= i; ++j) den += exp(sc[j] - mx);
+        for (j = 0; j <= i; ++j) {
+            const uint8_t *vv = vq + ((b * S + j) * Hkv + g) * D;
+            const double p = exp(sc[j] - mx) / den, sv = (double)vs[(b * S + j) * Hkv + g];
+            for (d = 0; d < D; ++d) {
+                const double t = p * sv * o_e4m3_decode(vv[d]);
+                o[d] += t;
+                if (m) m[d] += fabs(t);
+            }
+        }
+        free(sc);
+    }
+}
+
+/*
  * One optimizer step of an FP32 master weight, the step after which the
  * scales are recalibrated (section "Real-world performance gains": the policy
  * weights change every training step).  The pages do not name the optimizer;

@@ -131,3 +131,103 @@ def test_brute_force_against_scipy_softmax():
             vv = _dec(vq[b, :L, g]) * vs[b, :L, g, None]
             p = softmax(scale * (kk @ qd[b, h]))
             assert np.allclose(o[b, h], p @ vv, rtol=1e-12, atol=1e-14)
+
+
+# --- causal (prefill) attention over FP8 queries, keys and values -------------
+
+def _qkv(rng, B, S, Hq, Hkv, mode=oracle.SCALE_FP32):
+    q = rng.standard_normal((B, S, Hq, 128)).astype(np.float32)
+    qq, qs = oracle.quant_kv(_bits(q), mode)
+    kq, ks, vq, vs = _cache(rng, B, S, Hkv, mode=mode)
+    return qq, qs, kq, ks, vq, vs
+
+
+def test_prefill_brute_force_against_scipy_softmax():
+    # the definition evaluated independently: torch's E4M3 decode, numpy
+    # products, a causal mask and scipy's softmax, row by row
+    rng = np.random.default_rng(10)
+    B, S, Hq, Hkv = 2, 45, 4, 2
+    qq, qs, kq, ks, vq, vs = _qkv(rng, B, S, Hq, Hkv)
+    lens = [45, 17]
+    scale = 1.0 / np.sqrt(128.0)
+    o, mag = oracle.prefill_attention(qq, qs, kq, ks, vq, vs, lens, scale, want_mag=True)
+    o = o.reshape(B, S, Hq, 128)
+    mag = mag.reshape(B, S, Hq, 128)
+    for b in range(B):
+        L = lens[b]
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            qd = _dec(qq[b, :L, h]) * qs[b, :L, h, None]
+            kd = _dec(kq[b, :L, g]) * ks[b, :L, g, None]
+            vd = _dec(vq[b, :L, g]) * vs[b, :L, g, None]
+            s = scale * (qd @ kd.T)
+            s[np.triu_indices(L, 1)] = -np.inf
+            p = softmax(s, axis=1)
+            assert np.allclose(o[b, :L, h], p @ vd, rtol=1e-12, atol=1e-14)
+            assert np.allclose(mag[b, :L, h], p @ np.abs(vd), rtol=1e-12, atol=1e-14)
+        assert not o[b, L:].any() and not mag[b, L:].any()
+
+
+def test_prefill_first_row_is_its_own_value_and_future_keys_do_not_matter():
+    rng = np.random.default_rng(11)
+    B, S, Hq, Hkv = 1, 30, 4, 1
+    qq, qs, kq, ks, vq, vs = _qkv(rng, B, S, Hq, Hkv)
+    a = oracle.prefill_attention(qq, qs, kq, ks, vq, vs, [S], 0.1).reshape(B, S, Hq, 128)
+    for h in range(Hq):
+        assert np.array_equal(a[0, 0, h], _dec(vq[0, 0, 0]) * np.float64(vs[0, 0, 0]))
+    # rewriting keys and values at positions > 12 leaves rows 0..12 unchanged
+    kq2, vq2, ks2, vs2 = kq.copy(), vq.copy(), ks.copy(), vs.copy()
+    kq2[0, 13:] = 0x7E
+    vq2[0, 13:] = 0xFE
+    ks2[0, 13:] = 3.0
+    b = oracle.prefill_attention(qq, qs, kq2, ks2, vq2, vs2, [S], 0.1).reshape(B, S, Hq, 128)
+    assert np.array_equal(a[0, :13], b[0, :13])
+    assert not np.allclose(a[0, 13:], b[0, 13:])
+
+
+def test_prefill_zero_query_averages_the_visible_values():
+    rng = np.random.default_rng(12)
+    B, S, Hq, Hkv = 1, 21, 2, 2
+    qq, qs, kq, ks, vq, vs = _qkv(rng, B, S, Hq, Hkv)
+    qq[:] = 0
+    o = oracle.prefill_attention(qq, qs, kq, ks, vq, vs, [S], 0.3).reshape(B, S, Hq, 128)
+    for i in range(S):
+        for h in range(Hq):
+            mean = np.mean(_dec(vq[0, :i + 1, h]) * vs[0, :i + 1, h, None], axis=0)
+            assert np.allclose(o[0, i, h], mean, rtol=1e-12, atol=1e-15)
+
+
+def test_prefill_last_row_equals_decode_attention():
+    # with power-of-two scales a dequantized query is exactly a bf16 vector, so
+    # the last prefill row must equal the (separately pinned) decode attention
+    # of that query over the same cache
+    rng = np.random.default_rng(13)
+    B, S, Hq, Hkv = 2, 40, 8, 2
+    qq, qs, kq, ks, vq, vs = _qkv(rng, B, S, Hq, Hkv, mode=oracle.SCALE_POW2)
+    lens = [40, 23]
+    o = oracle.prefill_attention(qq, qs, kq, ks, vq, vs, lens, 0.088).reshape(B, S, Hq, 128)
+    qlast = np.stack([_dec(qq[b, lens[b] - 1]) * qs[b, lens[b] - 1, :, None] for b in range(B)])
+    qb = _bits(qlast)
+    assert np.array_equal(torch.from_numpy(qb.view(np.int16)).view(torch.bfloat16).double().numpy(), qlast)
+    d = oracle.decode_attention(qb, kq, ks, vq, vs, lens, 0.088)
+    for b in range(B):
+        assert np.allclose(o[b, lens[b] - 1], d[b], rtol=1e-12, atol=1e-15)
+
+
+def test_prefill_row_subset_and_grouped_heads():
+    rng = np.random.default_rng(14)
+    B, S, Hq, Hkv = 2, 19, 8, 4
+    qq, qs, kq, ks, vq, vs = _qkv(rng, B, S, Hq, Hkv)
+    full = oracle.prefill_attention(qq, qs, kq, ks, vq, vs, [19, 19], 0.1)
+    rows = np.array([0, 5, 18, 19, 37])
+    sub = oracle.prefill_attention(qq, qs, kq, ks, vq, vs, [19, 19], 0.1, rows=rows)
+    assert np.array_equal(full[rows], sub)
+    # value vectors of key/value head g all equal g + 1 (exact): every query head
+    # of group g returns g + 1
+    v = np.zeros((B, S, Hkv, 128), np.float32)
+    for g in range(Hkv):
+        v[:, :, g, :] = g + 1
+    vq2, vs2 = oracle.quant_kv(_bits(v), oracle.SCALE_POW2)
+    o = oracle.prefill_attention(qq, qs, kq, ks, vq2, vs2, [19, 19], 0.1).reshape(B, S, Hq, 128)
+    for h in range(Hq):
+        assert np.allclose(o[:, :, h], h // (Hq // Hkv) + 1, rtol=1e-14, atol=0)
