@@ -359,6 +359,185 @@ def cpu_baseline_oracle(budget_s=15.0):
             "sample_seconds": round(t_weight + t_rows, 2)}
 
 
+L2_BYTES = 126 * 2 ** 20
+
+
+def rotations(nbytes):
+    """Copies of a call's inputs to cycle through so that no call finds its
+    operands in L2 left there by the previous one (at least 4x L2 in total)."""
+    return max(1, -(-4 * L2_BYTES // max(1, nbytes)))
+
+
+def graph_ms(calls, reps=3):
+    """Per-call device time of `calls` (a list of no-argument launch functions),
+    replayed as one CUDA graph so the host does not pace the GPU; the median
+    of `reps` replays after one warm replay."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for fn in calls:
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        g.replay()
+        t1.record()
+        torch.cuda.synchronize()
+        times.append(t0.elapsed_time(t1) / len(calls))
+    del g
+    return statistics.median(times)
+
+
+def oracle_row(work, secs, unit_scale, unit, sample, extrapolated_from=None):
+    """The oracle's rate on a bounded sample, in the row's own unit."""
+    import oracle
+    d = {"value": work / secs / unit_scale, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+         "sample": sample, "sample_seconds": round(secs if extrapolated_from is None else extrapolated_from, 3)}
+    return d
+
+
+def bits(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def config_rows(fq, dev, peaks, gemm_ms_step):
+    """Every configuration of the workload besides the step itself: the single
+    linear, the whole-model power-of-2 recalibration, the 16 decode-shaped
+    linears (whole call, quantization included) and the two MoE expert GEMMs;
+    each timed on the device and, beside it, the oracle on a bounded sample of
+    the same work on the host cores.  Also the recalibration-overhead proxy."""
+    import oracle
+    rows = {}
+    hbm = peaks["hbm_gbs"]
+    fp8 = 2.0 * peaks["bf16_tflops"]
+
+    # --- single block-scaled linear: quantize X and W, FP8 GEMM (3 launches)
+    x, w = wl.single_linear(seed=0)
+    M, K = x.shape
+    N = w.shape[0]
+    n = rotations(M * K * 2 + N * K * 2)
+    xs = [x.to(dev) for _ in range(n)]
+    ws_ = [w.to(dev) for _ in range(n)]
+    qa = torch.empty((M, K), dtype=torch.uint8, device=dev)
+    sa = torch.empty(fq.act_scale_shape(M, K), dtype=torch.float32, device=dev)
+    qw = torch.empty((N, K), dtype=torch.uint8, device=dev)
+    sw = torch.empty((N // 128, K // 128), dtype=torch.float32, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+    def lin(i):
+        def f():
+            fq.quant_act(xs[i], fq.SCALE_FP32, q=qa, sa=sa)
+            fq.quant_weight(ws_[i], fq.SCALE_FP32, q=qw, sw=sw)
+            fq.gemm(qa, sa, qw, sw, fq.SCALE_FP32, out=y)
+        return f
+    ms = graph_ms([lin(i) for i in range(n)])
+    fl = 2.0 * M * N * K
+    t0 = time.perf_counter()
+    oqa, osa = oracle.quant_act(bits(x), 0)
+    oqw, osw = oracle.quant_weight(bits(w), 0)
+    oracle.gemm(oqa, osa, oqw, osw)
+    ot = time.perf_counter() - t0
+    rows["single_linear:256x512x512"] = {
+        "us_per_call": round(ms * 1e3, 2), "tflops": round(fl / (ms / 1e3) / 1e12, 3), "launches": 3,
+        "note": "latency-bound (0.13 GFLOP); quant_act + quant_weight + gemm in a CUDA graph",
+        "cpu_oracle": oracle_row(fl, ot, 1e12, "TFLOP/s", "the whole single linear")}
+    del xs, ws_
+
+    # --- decode-shaped linears: weights pre-quantized 128x128, X quantized inside the call
+    for name, (N, K) in wl.LLAMA8B_SHAPES.items():
+        wbf = wl.weights(N, K, seed=2)
+        wq, wsc = fq.quant_weight(wbf.to(dev), fq.SCALE_FP32)
+        oqw, osw = oracle.quant_weight(bits(wbf), 0)     # the oracle's own pre-quantized weight
+        # oracle: one row (act quant + FP64 GEMM against the whole weight); the
+        # time of M rows is M times that (rows are independent)
+        xb = bits(wl.activations(1, K, seed=1))
+        t0 = time.perf_counter()
+        oqa, osa = oracle.quant_act(xb, 0)
+        oracle.gemm(oqa, osa, oqw, osw)
+        t_row = time.perf_counter() - t0
+        for M in wl.DECODE_TOKENS:
+            nbytes = decode_bytes(M, N, K)
+            n = rotations(N * K)
+            qws = [wq] + [wq.clone() for _ in range(n - 1)]
+            x = wl.activations(M, K, seed=1, device=dev)
+            out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            wsp = torch.zeros(max(256, fq.gemm_decode_workspace_size(M, N, K)), dtype=torch.uint8, device=dev)
+            calls = [(lambda q=q: fq.gemm_decode(x, q, wsc, fq.SCALE_FP32, out=out, ws=wsp)) for q in qws]
+            ms = graph_ms(calls * max(1, 64 // n))
+            gbs = nbytes / (ms / 1e3) / 1e9
+            ot = t_row * M
+            rows["decode:%s:M%d" % (name, M)] = {
+                "us_per_call": round(ms * 1e3, 2), "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
+                "bytes": nbytes, "tflops": round(2.0 * M * N * K / (ms / 1e3) / 1e12, 1),
+                "cpu_oracle": oracle_row(nbytes, ot, 1e9, "GB/s",
+                                         "one row (act quant + FP64 GEMM against the whole weight), "
+                                         "time scaled to %d rows" % M)}
+            del qws
+        del wq, wsc, oqw, osw
+
+    # --- MoE expert GEMMs (Qwen3-30B-A3B-shaped, Zipf top-8 routing)
+    moe = wl.moe_layer(seed=0, device=dev)
+    off = moe["offsets"].to(torch.int32).to(dev)
+    offs = moe["offsets"].numpy()
+    for what in ("up", "down"):
+        x, w = moe["x_" + what], moe["w_" + what]
+        E, N, K = w.shape
+        R = x.shape[0]
+        qa, sa = fq.quant_act(x, fq.SCALE_FP32)
+        qw, sw = fq.quant_weight(w.reshape(E * N, K), fq.SCALE_FP32)
+        qw, sw = qw.view(E, N, K), sw.view(E, N // 128, K // 128)
+        y = torch.empty((R, N), dtype=torch.bfloat16, device=dev)
+        ms = graph_ms([lambda: fq.grouped_gemm(qa, sa, qw, sw, off, fq.SCALE_FP32, out=y)] * 10)
+        nbytes = moe_bytes(R, E, N, K)
+        fl = 2.0 * R * N * K
+        gbs = nbytes / (ms / 1e3) / 1e9
+        sample = np.unique(np.concatenate([np.arange(offs[e], min(offs[e + 1], offs[e] + 1)) for e in range(E)]))
+        oqa, osa = oracle.quant_act(bits(x), 0)
+        oqw, osw = oracle.quant_weight(bits(w.reshape(E * N, K)), 0)
+        oqw, osw = oqw.reshape(E, N, K), osw.reshape(E, N // 128, K // 128)
+        t0 = time.perf_counter()
+        oracle.grouped_gemm(oqa, osa, oqw, osw, offs, rows=sample)
+        ot = (time.perf_counter() - t0) * R / len(sample)
+        rows["moe:%s" % ("gate_up" if what == "up" else "down")] = {
+            "us_per_call": round(ms * 1e3, 2), "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
+            "tflops": round(fl / (ms / 1e3) / 1e12, 1), "frac_fp8_peak": round(fl / (ms / 1e3) / 1e12 / fp8, 3),
+            "bound": "hbm (roofline max(%.1f us flops, %.1f us bytes))" % (fl / fp8 / 1e6, nbytes / hbm / 1e3),
+            "cpu_oracle": oracle_row(nbytes, ot, 1e9, "GB/s",
+                                     "the first row of every non-empty expert (%d rows), time scaled to %d rows"
+                                     % (len(sample), R))}
+    del moe, qa, sa, qw, sw, y
+
+    # --- whole-model recalibration (32 layers x 4 weights, power-of-2 scales, one call)
+    tensors = []
+    for _, _, w in wl.model_weights_after_step(device=dev):
+        N, K = w.shape
+        tensors.append((w, torch.empty((N, K), dtype=torch.uint8, device=dev),
+                        torch.empty((N // 128, K // 128), dtype=torch.float32, device=dev)))
+    nbytes = sum(recal_bytes(*w.shape) for w, _, _ in tensors)
+    ms = graph_ms([lambda: fq.recalibrate(tensors, fq.SCALE_POW2)] * 3)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    ow = bits(tensors[1][0])           # one O-projection weight, 4096 x 4096
+    t0 = time.perf_counter()
+    oracle.quant_weight(ow, 1)
+    ot = (time.perf_counter() - t0) * nbytes / recal_bytes(*ow.shape)
+    rows["recalibrate:model_pow2"] = {
+        "ms": round(ms, 3), "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3), "tensors": len(tensors),
+        "params": int(sum(w.numel() for w, _, _ in tensors)),
+        "cpu_oracle": oracle_row(nbytes, ot, 1e9, "GB/s",
+                                 "one 4096x4096 weight, time scaled to the whole model's bytes")}
+    # per-step overhead proxy: the model's recalibration against 3 x 32 layers of
+    # the step's forward GEMMs (forward + the two backward GEMMs of a training step)
+    rows["recal_overhead"] = {
+        "value": round(ms / (3 * wl.LLAMA8B_LAYERS * gemm_ms_step), 4),
+        "definition": "recalibrate:model_pow2 ms / (3 x 32 x the benchmark step's four GEMM ms)",
+        "context": "the pages report about 2-3% recalibration overhead per training step on H100"}
+    del tensors
+    torch.cuda.empty_cache()
+    return rows
+
+
 def max_over_ranks(value, device):
     """The maximum of a per-rank float over all ranks (identity for one rank):
     the job's time is its slowest replica's."""
@@ -455,6 +634,8 @@ def ours(args):
         }
         if world == 1:
             line["cpu_baseline"] = cpu_baseline_oracle()
+            if not args.step_only:
+                rows.update(config_rows(fq, device, peaks, gemm_ms_total))
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -508,9 +689,30 @@ def reference(args):
 CASES = (["gemm:" + n for n in NAMES] + ["decode:" + n for n in NAMES] + ["cublas:" + n for n in NAMES] +
          ["quant_act:4096", "quant_act:14336", "recalibrate:layer", "quant_weight:gate_up", "moe:up", "moe:down",
           "swiglu:gate_up", "moe_swiglu:up", "adamw_recal:layer", "quant_act_t:4096", "quant_act_t:14336",
-          "transpose_weight:gate_up", "decode_attn:1x32768", "decode_attn:16x8192", "decode_attn:64x4096",
+          "transpose_weight:gate_up", "prefill_attn:4x2048", "prefill_attn:1x8192", "decode_attn:1x32768", "decode_attn:16x8192", "decode_attn:64x4096",
           "decode_attn:256x2048", "recalibrate:model"] + ["dgrad:" + n for n in NAMES] +
          ["wgrad:" + n for n in NAMES])
+
+
+def prefill_attn_flops(B, S, Hq, D=128):
+    """Causal attention: 2 x 2 x D FLOPs per (query, visible key, head)."""
+    return 4.0 * D * (S * (S + 1) // 2) * Hq * B
+
+
+def prefill_attn_inputs(fq, B, S, dev, Hq=32, Hkv=8):
+    """Seeded bf16 Q, K, V ~ N(0, 1) quantized 1x128 per head vector on the GPU."""
+    g = torch.Generator(device=dev).manual_seed(17)
+    q = torch.randn((B * S * Hq, 128), generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn((B * S * Hkv, 128), generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn((B * S * Hkv, 128), generator=g, device=dev).to(torch.bfloat16)
+    qq, qs = fq.quant_act(q)
+    kq, ks = fq.quant_act(k)
+    vq, vs = fq.quant_act(v)
+    shape_q, shape_kv = (B, S, Hq), (B, S, Hkv)
+    lens = torch.full((B,), S, dtype=torch.int32, device=dev)
+    return ((qq.view(*shape_q, 128), qs[0, :B * S * Hq].contiguous().view(shape_q)),
+            kq.view(*shape_kv, 128), ks[0, :B * S * Hkv].contiguous().view(shape_kv),
+            vq.view(*shape_kv, 128), vs[0, :B * S * Hkv].contiguous().view(shape_kv), lens)
 
 
 def decode_bytes(M, N, K):
@@ -573,7 +775,7 @@ def run_case(args):
         w = wl.weights(N, K, seed=2, device=dev)
         qw, sw = fq.quant_weight(w, mode)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(max(256, fq.gemm_decode_workspace_size(M, N, K)), dtype=torch.uint8, device=dev)
+        ws = torch.zeros(max(256, fq.gemm_decode_workspace_size(M, N, K)), dtype=torch.uint8, device=dev)
         fn = lambda: fq.gemm_decode(x, qw, sw, mode, out=y, ws=ws)  # noqa: E731
         work, unit = decode_bytes(M, N, K) / 1e9, "GB/s"
     elif kind == "moe":
@@ -638,6 +840,14 @@ def run_case(args):
         fn = lambda: fq.decode_attention(qv, kq, ks, vq, vs, lens, out=out, ws=ws)  # noqa: E731
         work = (B_ * S_ * Hkv * (2 * 128 + 8) + 2 * B_ * Hq * 128 * 2) / 1e9
         unit = "GB/s"
+    elif kind == "prefill_attn":
+        # Llama-3.1-8B attention (32 query heads, 8 key/value heads, D = 128),
+        # causal over B sequences of S tokens, FP8 queries, keys and values
+        B_, S_ = (int(v) for v in what.split("x"))
+        q, kq, ks, vq, vs, lens = prefill_attn_inputs(fq, B_, S_, dev)
+        out = torch.empty((B_, S_, 32, 128), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.prefill_attention(*q, kq, ks, vq, vs, lens, out=out)  # noqa: E731
+        work, unit = prefill_attn_flops(B_, S_, 32) / 1e12, "TFLOP/s"
     elif kind == "quant_act_t":
         K = int(what)
         x = wl.activations(M, K, seed=1, device=dev)
@@ -757,6 +967,8 @@ def main():
     ap.add_argument("--pair", action="store_true", help="--case gemm: the CTA-pair promotion kernel")
     ap.add_argument("--pair128", action="store_true",
                     help="--case gemm: the CTA-pair promotion kernel with 256x128 tiles")
+    ap.add_argument("--step-only", action="store_true",
+                    help="only the benchmark step (no rows for the other workload configurations)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)

@@ -85,7 +85,7 @@ def test_wgrad_within_tolerance(mode):
 @pytest.mark.parametrize("name", ["qkv", "down"])
 def test_wgrad_llama_full_size_sampled_rows(name):
     """dW of a Llama-8B-shaped projection at M = 8192 tokens; the oracle
-    quantizes dY and X itself and computes 8 sampled rows of dW."""
+    quantizes dY and X itself and computes one row of dW in every 128-row tile."""
     N, K = wl.LLAMA8B_SHAPES[name]
     M = wl.PREFILL_TOKENS
     dy = wl.activations(M, N, seed=51, device="cuda")
@@ -94,7 +94,8 @@ def test_wgrad_llama_full_size_sampled_rows(name):
     qb, sb = fq.quant_act_t(x)
     y = fq.gemm_wgrad(qa, sa, qb, sb, M)
     torch.cuda.synchronize()
-    rows = np.array([0, 1, 127, 128, 1000, N // 2, N - 2, N - 1])
+    rng = np.random.default_rng(N)
+    rows = np.array(sorted({0, N - 1} | {int(rng.integers(t, min(t + 128, N))) for t in range(0, N, 128)}))
     oa, osa = oracle.quant_act_t(bf16_bits(dy[:, torch.from_numpy(rows).cuda()]), fq.SCALE_FP32)
     ob, osb = oracle.quant_act_t(bf16_bits(x), fq.SCALE_FP32)
     ref = oracle.gemm_wgrad(oa, osa, ob, osb)
@@ -127,7 +128,8 @@ def test_dgrad_llama_down_full_size_sampled_rows():
     qwt, swt = fq.transpose_weight(qw, sw)
     dx = fq.gemm_dgrad(q_dy, s_dy, qwt, swt)
     torch.cuda.synchronize()
-    rows = np.array([0, 5, 4095, 4096, M - 1])
+    rng = np.random.default_rng(M)
+    rows = np.array(sorted({0, M - 1} | {int(rng.integers(t, t + 128)) for t in range(0, M, 128)}))
     oq, os_ = oracle.quant_act(bf16_bits(dy[torch.from_numpy(rows).cuda()]), fq.SCALE_FP32)
     oqw, osw = oracle_weight(w, fq.SCALE_FP32)
     ref = oracle.gemm_dgrad(oq, os_, oqw, osw)

@@ -34,6 +34,16 @@ def int_codes(rng, shape, vmax):
     return torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
 
 
+def tile_rows(M, seed, per_tile=1):
+    """`per_tile` seeded rows of every 128-row tile (the first and last rows of
+    the matrix always among them), so every persistent CTA's tiles are checked."""
+    rng = np.random.default_rng(seed)
+    rows = {0, M - 1}
+    for t in range(0, M, 128):
+        rows.update(int(r) for r in rng.integers(t, min(t + 128, M), size=per_tile))
+    return np.array(sorted(rows))
+
+
 def run_gemm(qa, sa, qw, sw, mode=fq.SCALE_FP32, variant=fq.GEMM_PROMOTE):
     """numpy operands -> GPU bf16 output as numpy uint16 bits and float64 values."""
     M, K = qa.shape
@@ -87,8 +97,8 @@ def test_single_linear_within_tolerance(mode):
 @pytest.mark.parametrize("name", list(wl.LLAMA8B_SHAPES))
 def test_llama_prefill_full_size_sampled_rows(mode, name):
     """The bench's launch configuration (M = 8192) end to end on the GPU: quantize
-    X and W, GEMM; the oracle quantizes the same bf16 inputs itself (16 sampled
-    rows of X, all of W) and computes those rows."""
+    X and W, GEMM; the oracle quantizes the same bf16 inputs itself (one row of
+    every 128-row tile of X, all of W) and computes those rows, every column."""
     N, K = wl.LLAMA8B_SHAPES[name]
     M = wl.PREFILL_TOKENS
     x = wl.activations(M, K, seed=N, device="cuda")
@@ -97,8 +107,7 @@ def test_llama_prefill_full_size_sampled_rows(mode, name):
     qw, sw = fq.quant_weight(w, mode)
     y = fq.gemm(qa, sa, qw, sw, mode)
     torch.cuda.synchronize()
-    rows = np.sort(np.random.default_rng(N).choice(M, 16, replace=False))
-    rows[0], rows[-1] = 0, M - 1
+    rows = tile_rows(M, seed=N)
     oqa, osa = oracle_act(x, mode, rows)
     oqw, osw = oracle_weight(w, mode)
     ref = oracle.gemm(oqa, osa, oqw, osw, blockint=True)
@@ -156,3 +165,25 @@ def test_pair_kernel_equals_one_sm_kernel(pair_variant):
     torch.cuda.synchronize()
     assert_gemm_close(bf16_to_f64(y_pair), bf16_to_f64(y_one), "pair vs one-SM")
     assert torch.equal(y_pair.view(torch.int16), y_one.view(torch.int16))
+
+
+@pytest.mark.parametrize("variant", VARIANTS + [fq.GEMM_NATIVE_POW2])
+def test_distinct_pow2_scales_more_tiles_than_sms_bit_exact(variant):
+    """Integer codes with distinct power-of-two scales per (row, K-block) and
+    (N-block, K-block) at M = 2048, N = 28672 (the gate+up shape's N): 1792
+    tiles of 128x256, about 12 per persistent CTA, so every CTA carries its
+    TMEM phase and its tile order across many tiles.  The FP32 sums are exact,
+    so the bf16 result equals the oracle's bit for bit; one row of every
+    128-row tile, every column, is compared."""
+    rng = np.random.default_rng(29)
+    M, N, K = 2048, 28672, 512
+    KB, NB = K // 128, N // 128
+    qa = int_codes(rng, (M, K), 4)
+    qw = int_codes(rng, (N, K), 4)
+    sa = (2.0 ** (((np.arange(M)[None, :] * 7 + np.arange(KB)[:, None]) % 5) - 2)).astype(np.float32)
+    sw = (2.0 ** (((np.arange(NB)[:, None] * 3 + np.arange(KB)[None, :]) % 7) - 3)).astype(np.float32)
+    bits, _ = run_gemm(qa, sa, qw, sw, fq.SCALE_POW2, variant)
+    rows = tile_rows(M, seed=5, per_tile=1)
+    ref = oracle.f64_to_bf16(oracle.gemm(qa, sa, qw, sw, rows=rows))
+    got = bits[rows]
+    assert np.array_equal(got, ref), np.argwhere(got != ref)[:5]

@@ -67,7 +67,8 @@ def test_llama_shapes_against_oracle_and_promotion(name):
     yn = fq.gemm(qa, sa, qw, sw, fq.SCALE_POW2, variant=NATIVE)
     yp = fq.gemm(qa, sa, qw, sw, fq.SCALE_POW2, variant=fq.GEMM_PROMOTE)
     torch.cuda.synchronize()
-    rows = np.array([0, 1, 127, 128, 500, M - 1])
+    rng = np.random.default_rng(N)
+    rows = np.array(sorted({0, 1, 127, 128, M - 1} | {int(rng.integers(t, t + 128)) for t in range(0, M, 128)}))
     oqa, osa = oracle_act(x, fq.SCALE_POW2, rows)
     oqw, osw = oracle_weight(w, fq.SCALE_POW2)
     ref = oracle.gemm(oqa, osa, oqw, osw, blockint=True)

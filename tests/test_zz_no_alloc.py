@@ -4,10 +4,12 @@ It is for callers that cannot allocate device memory when they call (a C or
 Fortran host program without a framework's memory pool, a serving loop with a
 fixed memory budget): the scratch lives in a fixed device array inside the
 library.  This test calls it through the C ABI and checks its output against
-fp8bq_gemm_decode with a caller workspace, within the GEMM tolerance of the
-other tests, on two calls in a row (the array keeps the previous call's
-contents, which must not leak into the next result).  It sits in its own file,
-collected last, and passes both alone in a fresh process and after the others.
+fp8bq_gemm_decode with a caller workspace and against the oracle (its own
+quantization of the same bf16 activations and weights, FP64 sums; every row up
+to M = 64, one row of every 16 above), within the GEMM tolerance of the other
+tests, on two calls in a row (the array keeps the previous call's contents,
+which must not leak into the next result).  It sits in its own file, collected
+last, and passes both alone in a fresh process and after the others.
 """
 import ctypes
 
@@ -17,7 +19,8 @@ import torch
 
 import fp8_block_scaled_fp8bq_b200 as fq
 import fp8bq_workloads as wl
-from helpers import assert_gemm_close, bf16_to_f64, need_gpu
+import oracle
+from helpers import assert_gemm_close, bf16_to_f64, need_gpu, oracle_act, oracle_weight
 
 pytestmark = pytest.mark.gpu
 
@@ -40,6 +43,8 @@ def test_noalloc_matches_workspace_entry_point(name, M, mode):
     N, K = wl.LLAMA8B_SHAPES[name]
     w = wl.weights(N, K, seed=N + K, device="cuda")
     qw, sw = fq.quant_weight(w, mode)
+    oqw, osw = oracle_weight(w, mode)
+    rows = np.arange(M) if M <= 64 else np.arange(0, M, 16)
     for call in range(2):                      # two calls in a row, different inputs
         x = wl.activations(M, K, seed=1000 * call + M, device="cuda")
         ref = fq.gemm_decode(x, qw, sw, mode)
@@ -48,6 +53,10 @@ def test_noalloc_matches_workspace_entry_point(name, M, mode):
         assert st == 0, "status %d" % st
         torch.cuda.synchronize()
         assert_gemm_close(bf16_to_f64(y), bf16_to_f64(ref), "%s M=%d call %d" % (name, M, call))
+        oqa, osa = oracle_act(x, mode, rows)
+        y64 = oracle.gemm(oqa, osa, oqw, osw, blockint=True)
+        got = bf16_to_f64(y[torch.from_numpy(rows).cuda()])
+        assert_gemm_close(got, y64, "%s M=%d call %d vs oracle" % (name, M, call))
     st, word = fq.device_error()
     assert st == 0 and word == 0
 
