@@ -12,6 +12,7 @@ performance gains" (per-step scale recalibration; mixture-of-experts) and
 section "Why this matters for AI economics" (power-of-2 scales).
 """
 import ctypes
+import math
 import os
 
 import torch
@@ -84,6 +85,7 @@ SIGNATURES = {
     "fp8bq_kv_cache_append": (I32, [P, P, P, P, P, P, P, I64, I64, I64, I32, P]),
     "fp8bq_decode_attention_workspace_size": (SZ, [I64, I64, I64, I64]),
     "fp8bq_decode_attention": (I32, [P, P, P, P, P, P, I64, I64, I64, I64, ctypes.c_float, P, P, SZ, P]),
+    "fp8bq_prefill_attention": (I32, [P, P, P, P, P, P, P, I64, I64, I64, I64, ctypes.c_float, P, P]),
     "fp8bq_adamw_recalibrate": (I32, [ctypes.POINTER(AdamWDesc), I32, ctypes.POINTER(AdamWConfig), I32, P]),
     "fp8bq_gemm_swiglu_quant": (I32, [P, I64, P, I64, P, I64, P, P, I64, P, I64, P, I64, I64, I64, I64, I32, P]),
     "fp8bq_grouped_gemm_swiglu_quant": (I32, [P, I64, P, I64, P, P, P, I32, I64, I64, I64, P, I64, P, I64, P, I64,
@@ -247,6 +249,25 @@ def decode_attention(q, kq, ks, vq, vs, seq_lens, softmax_scale=None, out=None, 
     return out
 
 
+def prefill_attention(qq, qs, kq, ks, vq, vs, seq_lens, softmax_scale=None, out=None, stream=None):
+    """Causal attention of FP8 queries over FP8 keys and values of the same
+    sequences.  qq uint8 [B, S, Hq, 128], qs fp32 [B, S, Hq]; kq, vq uint8
+    [B, S, Hkv, 128], ks, vs fp32 [B, S, Hkv]; seq_lens int32 [B] (device).
+    Returns bf16 [B, S, Hq, 128]."""
+    B, S, Hq, D = qq.shape
+    Hkv = kq.shape[2]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(D)
+    for t in (qq, qs, kq, ks, vq, vs, seq_lens):
+        assert t.is_contiguous(), "contiguous tensors expected"
+    if out is None:
+        out = torch.empty((B, S, Hq, D), dtype=torch.bfloat16, device=qq.device)
+    _check(lib().fp8bq_prefill_attention(_ptr(qq), _ptr(qs), _ptr(kq), _ptr(ks), _ptr(vq), _ptr(vs), _ptr(seq_lens),
+                                         B, S, Hq, Hkv, float(softmax_scale), _ptr(out), _stream(stream)),
+           "fp8bq_prefill_attention")
+    return out
+
+
 def adamw_recalibrate(tensors, lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=1, mode=SCALE_POW2,
                       stream=None):
     """One AdamW step on fp32 master weights fused with their 128x128 recalibration.
@@ -282,14 +303,16 @@ def gemm_decode_workspace_size(M, N, K):
 
 
 def gemm_decode(x, qw, sw, mode=SCALE_FP32, out=None, ws=None, stream=None):
-    """Small-M linear with on-the-fly 1x128 activation quantization."""
+    """Small-M linear with on-the-fly 1x128 activation quantization.  A caller
+    workspace `ws` (uint8, gemm_decode_workspace_size bytes) must be zero-filled
+    before its first use; every call leaves it reusable."""
     M, K = x.shape
     N = qw.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     need = gemm_decode_workspace_size(M, N, K)
-    if ws is None:
-        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    if ws is None:  # its counter area must start zeroed (each call leaves it so)
+        ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=x.device)
     _check(lib().fp8bq_gemm_decode(_ptr(x), _ld(x), _ptr(qw), _ld(qw), _ptr(sw), _ptr(out), _ld(out), M, N, K,
                                    mode, _ptr(ws), ws.numel(), _stream(stream)), "fp8bq_gemm_decode")
     return out

@@ -29,7 +29,7 @@ FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-ftz=false", "-prec-div=true"
 # Kernels that split registers between warpgroups with setmaxnreg: the launch
 # register count ptxas reports must equal the count the split assumes.
 SETMAXNREG_KERNELS = {"gemm_promote_kernel": 168, "decode_kernel": 168, "gemm_pair_kernel": 168,
-                      "gemm_native_kernel": 168}
+                      "gemm_native_kernel": 168, "prefill_attn_kernel": 168}
 
 
 def _check_registers(log_text):

@@ -1,6 +1,7 @@
 // C ABI of libfp8bq: argument validation, status codes, device error word,
 // TMA descriptor encoding.  Every entry point checks its arguments before it
 // launches anything, and never throws.
+#include <math.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -28,7 +29,8 @@ thread_local int g_last_cuda_code = 0;  // cudaError_t of this thread's last fai
 TensorMapCache g_maps;
 
 TensorMapKey map_key(int rank, CUtensorMapDataType dtype, const void *base, const uint64_t *dims,
-                     const uint64_t *strides, uint32_t box0, uint32_t box1, CUtensorMapSwizzle swizzle) {
+                     const uint64_t *strides, uint32_t box0, uint32_t box1, CUtensorMapSwizzle swizzle,
+                     uint32_t box2 = 0) {
   TensorMapKey k;
   memset(&k, 0, sizeof(k));
   k.base = base;
@@ -36,6 +38,7 @@ TensorMapKey map_key(int rank, CUtensorMapDataType dtype, const void *base, cons
   for (int i = 0; i + 1 < rank; ++i) k.strides[i] = strides[i];
   k.box[0] = box0;
   k.box[1] = box1;
+  k.box[2] = box2;
   k.rank = rank;
   k.dtype = (int32_t)dtype;
   k.swizzle = (int32_t)swizzle;
@@ -104,14 +107,14 @@ bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
 
 bool make_tmap_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
-                  CUtensorMapSwizzle swizzle) {
+                  CUtensorMapSwizzle swizzle, uint32_t box2) {
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
-  const TensorMapKey key = map_key(3, dtype, base, dims, strides, box0, box1, swizzle);
+  const TensorMapKey key = map_key(3, dtype, base, dims, strides, box0, box1, swizzle, box2);
   if (g_maps.find(key, map)) return true;
   CUtensorMap probe;
   if (!make_tmap_2d(&probe, dtype, base, d0, d1, stride1_bytes, box0, box1, swizzle)) return false;  // loads g_encode
-  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t box[3] = {box0, box1, box2};
   cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = g_encode(map, dtype, 3, const_cast<void *>(base), dims, strides, box, estride,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -232,7 +235,8 @@ fp8bq_status fp8bq_get_device_error(uint64_t *code) {
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
   cudaError_t (*takers[])(unsigned long long *) = {take_device_error_gemm, take_device_error_decode,
                                                     take_device_error_native, take_device_error_pair,
-                                                    take_device_error_swiglu, take_device_error_wgrad};
+                                                    take_device_error_swiglu, take_device_error_wgrad,
+                                                    take_device_error_prefill_attn};
   for (auto take : takers) {
     e = take(&w);
     if (e != cudaSuccess) return cuda_fail(e, "read device error word");
@@ -428,6 +432,21 @@ fp8bq_status fp8bq_decode_attention(const void *q, const uint8_t *kq, const floa
   }
   return launch_decode_attention(q, kq, ks, vq, vs, seq_lens, B, Hq, Hkv, S, softmax_scale, o, ws, ws_bytes,
                                  static_cast<cudaStream_t>(stream));
+}
+
+fp8bq_status fp8bq_prefill_attention(const uint8_t *qq, const float *qs, const uint8_t *kq, const float *ks,
+                                     const uint8_t *vq, const float *vs, const int32_t *seq_lens, int64_t B, int64_t S,
+                                     int64_t Hq, int64_t Hkv, float softmax_scale, void *o, void *stream) {
+  if (B < 0 || S < 0 || Hq < 0 || Hkv < 0) return FP8BQ_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !(softmax_scale < INFINITY)) return FP8BQ_ERR_INVALID_ARG;
+  if (B == 0 || S == 0 || Hq == 0) return FP8BQ_OK;
+  if (Hkv == 0 || Hq % Hkv != 0) return FP8BQ_ERR_INVALID_ARG;
+  if (Hq >= 65536 || B * S >= kMaxDim || B * Hq * ((S + 127) / 128) >= kMaxDim) return FP8BQ_ERR_UNSUPPORTED;
+  if (!qq || !qs || !kq || !ks || !vq || !vs || !seq_lens || !o) return FP8BQ_ERR_INVALID_ARG;
+  if (!aligned(qq, 16) || !aligned(kq, 16) || !aligned(vq, 16) || !aligned(o, 16)) return FP8BQ_ERR_INVALID_ARG;
+  if (!aligned(qs, 4) || !aligned(ks, 4) || !aligned(vs, 4) || !aligned(seq_lens, 4)) return FP8BQ_ERR_INVALID_ARG;
+  return launch_prefill_attention(qq, qs, kq, ks, vq, vs, seq_lens, B, S, Hq, Hkv, softmax_scale, o,
+                                  static_cast<cudaStream_t>(stream));
 }
 
 fp8bq_status fp8bq_kv_cache_append(const void *k_new, const void *v_new, const int32_t *positions, uint8_t *kq,

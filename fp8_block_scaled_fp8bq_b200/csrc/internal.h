@@ -71,8 +71,8 @@ class DeviceOnce {
 struct TensorMapKey {
   const void *base;
   uint64_t dims[3], strides[2];
-  uint32_t box[2];
-  int32_t rank, dtype, swizzle, pad;  // no implicit padding: compared and hashed as bytes
+  uint32_t box[3];
+  int32_t rank, dtype, swizzle;  // no implicit padding: compared and hashed as bytes
 };
 static_assert(sizeof(TensorMapKey) == 72, "TensorMapKey has no padding");
 
@@ -121,10 +121,10 @@ fp8bq_status check_launch(const char *what);
 bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
                   uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
-// 3-D variant: dims {d0 (innermost), d1, d2}, byte strides of dims 1 and 2, box {box0, box1, 1}.
+// 3-D variant: dims {d0 (innermost), d1, d2}, byte strides of dims 1 and 2, box {box0, box1, box2}.
 bool make_tmap_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
                   uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
-                  CUtensorMapSwizzle swizzle);
+                  CUtensorMapSwizzle swizzle, uint32_t box2 = 1);
 
 // Tile order of a persistent GEMM over an M x N output in bm x bn tiles with
 // depth K (bytes per operand row = K): picks the banded dimension and the band
@@ -139,6 +139,7 @@ cudaError_t take_device_error_native(unsigned long long *v);
 cudaError_t take_device_error_pair(unsigned long long *v);
 cudaError_t take_device_error_swiglu(unsigned long long *v);
 cudaError_t take_device_error_wgrad(unsigned long long *v);
+cudaError_t take_device_error_prefill_attn(unsigned long long *v);
 
 // Launchers (arguments already validated).
 fp8bq_status launch_encode(const float *x, int64_t n, uint8_t *q, cudaStream_t stream);
@@ -186,6 +187,9 @@ size_t decode_attention_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64
 fp8bq_status launch_decode_attention(const void *q, const uint8_t *kq, const float *ks, const uint8_t *vq,
                                      const float *vs, const int32_t *lens, int64_t B, int64_t Hq, int64_t Hkv,
                                      int64_t S, float scale, void *o, void *ws, size_t ws_bytes, cudaStream_t stream);
+fp8bq_status launch_prefill_attention(const uint8_t *qq, const float *qs, const uint8_t *kq, const float *ks,
+                                      const uint8_t *vq, const float *vs, const int32_t *lens, int64_t B, int64_t S,
+                                      int64_t Hq, int64_t Hkv, float scale, void *o, cudaStream_t stream);
 fp8bq_status launch_kv_append(const void *k_new, const void *v_new, const int32_t *pos, uint8_t *kq, float *ks,
                               uint8_t *vq, float *vs, int64_t B, int64_t Hkv, int64_t S, int mode,
                               cudaStream_t stream);

@@ -225,8 +225,15 @@ FP8BQ_API fp8bq_status fp8bq_gemm_ex(const uint8_t *qa, int64_t lda, const float
  * breakthrough": FP8 in both generation and training).
  *   x     bf16 [M][ldx]; qw, sw as in fp8bq_gemm; y bf16 [M][ldy].
  *   ws    device workspace of at least fp8bq_gemm_decode_workspace_size(M, N, K)
- *         bytes, 256-byte aligned; its contents need not be initialized and are
- *         overwritten.  Calls that share a workspace must be stream-ordered.
+ *         bytes, 256-byte aligned.  Its first 4096 bytes are arrival counters of
+ *         the weight blocks that several CTAs share: they must be zero before
+ *         the workspace's first use (e.g. cudaMemset once), and every call that
+ *         completes leaves them zero again, so a workspace can be reused for any
+ *         shape.  (After a call that reported FP8BQ_ERR_TIMEOUT, zero them
+ *         again.)  The rest is scratch.  Calls that share a workspace must be
+ *         stream-ordered.
+ * One launch for M <= 16 (the activation is quantized inside the GEMM kernel
+ * when x is 16-byte aligned with ldx % 8 == 0), two otherwise.
  * Requirements: as fp8bq_gemm, and M <= 256.  Output equals fp8bq_quant_act
  * followed by fp8bq_gemm up to FP32 summation order.
  */
@@ -248,11 +255,13 @@ FP8BQ_API fp8bq_status fp8bq_gemm_decode(const void *x, int64_t ldx,
  *   every GPU that loads it until the process exits; a shape whose workspace
  *   (fp8bq_gemm_decode_workspace_size) exceeds 32 MiB returns
  *   FP8BQ_ERR_WORKSPACE and launches nothing.  Nothing is allocated.
- *   The first call on a device looks up the array's device address (a CUDA
- *   runtime call); make that first call outside any stream capture.
+ *   The first call on a device looks up the array's device address and zeroes
+ *   the array's counter area (CUDA runtime calls, synchronous); make that first
+ *   call outside any stream capture.
  *   All calls share the one array: calls that may run at the same time on the
  *   GPU (different streams, or different host threads) race on it and must be
- *   ordered by the caller.  Each call rewrites the parts it reads.
+ *   ordered by the caller.  The counter area is left zero by every call and
+ *   the rest is rewritten before it is read.
  */
 FP8BQ_API fp8bq_status fp8bq_gemm_decode_noalloc(const void *x, int64_t ldx,
                                                  const uint8_t *qw, int64_t ldw, const float *sw,
@@ -439,6 +448,36 @@ FP8BQ_API fp8bq_status fp8bq_decode_attention(const void *q, const uint8_t *kq, 
                                               int64_t B, int64_t Hq, int64_t Hkv, int64_t S,
                                               float softmax_scale, void *o, void *ws, size_t ws_bytes,
                                               void *stream);
+
+/*
+ * Causal (prefill) attention over FP8 queries, keys and values ("Real-world
+ * performance gains": FP8 KV cache and FP8 attention; "Technical
+ * breakthrough": every head vector is one 1x128 tile with one scale).
+ * Sequence b holds tokens [0, seq_lens[b]) (int32, device; clamped to
+ * [0, S]); query row i < seq_lens[b] attends the keys j <= i of its own
+ * sequence, query head h reading key/value head h / (Hq / Hkv):
+ *   s_j   = softmax_scale * qs[b][i][h] * ks[b][j][g] * sum_d dec(qq[b][i][h][d]) dec(kq[b][j][g][d])
+ *   o[d]  = sum_j softmax(s)_j * vs[b][j][g] * dec(vq[b][j][g][d])
+ * Both contractions run on the tensor cores with E4M3 operands and FP32
+ * accumulation: the scores from the codes of q and k (exact products), the
+ * values with the softmax weights p_j (FP32) times vs[b][j][g] / vmax * 256
+ * rounded to E4M3 (vmax = the largest value scale of each 128-key block, so
+ * each weight enters with a relative rounding of at most 2^-4, or an absolute
+ * one of 2^-10 * vmax / 256 below the E4M3 normal range); the row sums use the
+ * unrounded weights; bf16 out.  Rows i >= seq_lens[b] are written as 0.
+ *   qq  E4M3 [B][S][Hq][128]   qs  fp32 [B][S][Hq]    (fp8bq_quant_act over
+ *                                                       [B*S*Hq][128] gives both)
+ *   kq, vq  E4M3 [B][S][Hkv][128]   ks, vs  fp32 [B][S][Hkv]   (the KV cache layout)
+ *   o   bf16 [B][S][Hq][128]
+ * Positions at or past seq_lens[b] of kq and vq inside a 128-token block that
+ * holds valid tokens are read with zero weight and must not hold NaN codes.
+ * Requirements: softmax_scale > 0 and finite; Hq % Hkv == 0; qq, kq, vq and o
+ * 16-byte aligned; qs, ks, vs, seq_lens 4-byte aligned; B * S < 2^31.
+ */
+FP8BQ_API fp8bq_status fp8bq_prefill_attention(const uint8_t *qq, const float *qs, const uint8_t *kq,
+                                               const float *ks, const uint8_t *vq, const float *vs,
+                                               const int32_t *seq_lens, int64_t B, int64_t S, int64_t Hq,
+                                               int64_t Hkv, float softmax_scale, void *o, void *stream);
 
 /*
  * One optimizer step fused with the recalibration it makes necessary

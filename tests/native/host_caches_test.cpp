@@ -35,6 +35,7 @@ static TensorMapKey key_for(int i) {
   k.strides[0] = 4096;
   k.box[0] = 128;
   k.box[1] = 128;
+  k.box[2] = 0;
   k.rank = 2;
   return k;
 }

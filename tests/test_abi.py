@@ -266,3 +266,14 @@ def test_interleave_gate_up_layout():
     assert torch.equal(col[256:384], 128 + r) and torch.equal(col[384:512], -129 - r)
     e = fq.interleave_gate_up(g.reshape(1, I, K).expand(3, I, K), u.reshape(1, I, K).expand(3, I, K))
     assert e.shape == (3, 2 * I, K) and torch.equal(e[2, :, 0].float(), col)
+
+
+def test_prefill_attention_validation(L):
+    f = L.fp8bq_prefill_attention
+    P = FAKE
+    assert f(P, P, P, P, P, P, P, 1, 128, 8, 3, 0.1, P, None) == INVALID           # Hq % Hkv
+    assert f(P, P, P, P, P, P, P, 1, 128, 8, 2, 0.0, P, None) == INVALID           # scale <= 0
+    assert f(P, P, P, P, P, P, P, 1, 128, 8, 2, float("inf"), P, None) == INVALID
+    assert f(ctypes.c_void_p(0x10004), P, P, P, P, P, P, 1, 128, 8, 2, 0.1, P, None) == INVALID  # alignment
+    assert f(P, P, P, P, P, P, None, 1, 128, 8, 2, 0.1, P, None) == INVALID        # no lengths
+    assert f(None, None, None, None, None, None, None, 0, 128, 8, 2, 0.1, None, None) == 0   # empty: no-op

@@ -42,9 +42,9 @@ def qweights(name, mode):
     return _W[key]
 
 
-def check_decode(x, qw, sw, mode):
+def check_decode(x, qw, sw, mode, ws=None):
     M, K = x.shape
-    y = fq.gemm_decode(x, qw, sw, mode)
+    y = fq.gemm_decode(x, qw, sw, mode, ws=ws)
     torch.cuda.synchronize()
     qa, sa = oracle.quant_act(bf16_bits(x), mode)
     oqw, osw = _OW[qw.data_ptr()]
@@ -103,3 +103,29 @@ def test_workspace_and_limits():
     with pytest.raises(fq.Fp8bqError) as e:
         fq.gemm_decode(big, qw, sw)
     assert e.value.status == 2
+
+
+def test_workspace_counters_left_zero_and_reused_across_shapes():
+    # one workspace for every shape: the arrival counters of the cut weight
+    # blocks (its first 4096 bytes) are zero after each call, and every call's
+    # rows match the oracle (the single-launch path at M <= 16, the two-launch
+    # one above, unaligned activations through the prologue)
+    need = max(fq.gemm_decode_workspace_size(M, N, K) for N, K in wl.LLAMA8B_SHAPES.values() for M in (1, 16, 40))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for name, (N, K) in wl.LLAMA8B_SHAPES.items():
+        qw, sw = qweights(name, fq.SCALE_FP32)
+        for M in (1, 16, 40):
+            x = wl.activations(M, K, seed=3 * M + K, device="cuda")
+            check_decode(x, qw, sw, fq.SCALE_FP32, ws=ws)
+            assert not ws[:4096].any(), "counters left nonzero after %s M=%d" % (name, M)
+        # a row view whose leading dimension is odd: not 16-byte loadable
+        xb = wl.activations(4, K + 1, seed=K, device="cuda")[:, :K]
+        check_decode(xb, qw, sw, fq.SCALE_FP32, ws=ws)
+        assert not ws[:4096].any()
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+def test_single_launch_pow2(M):
+    qw, sw = qweights("gate_up", fq.SCALE_POW2)
+    x = wl.activations(M, 4096, seed=40 + M, device="cuda")
+    check_decode(x, qw, sw, fq.SCALE_POW2)

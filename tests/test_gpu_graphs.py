@@ -79,7 +79,7 @@ def test_decode_gemm_in_a_graph():
         return [wl.activations(M, K, seed=seed, device="cuda")]
     (x,) = make(0)
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(max(fq.gemm_decode_workspace_size(M, N, K), 256), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(max(fq.gemm_decode_workspace_size(M, N, K), 256), dtype=torch.uint8, device="cuda")
 
     def run():
         fq.gemm_decode(x, qw, sw, fq.SCALE_FP32, out=y, ws=ws)
