@@ -15,7 +15,7 @@
 // weight-block-major order, into one contiguous equal share per CTA, so every
 // SM streams the same number of weight bytes whatever NB is.  Per work item:
 // the weight tile (16 KB) comes through a TMA stage ring; 4 x tcgen05.mma
-// 128xNTx32 go into one of two TMEM buffers; the epilogue warps (weight row =
+// 128xNTx32 go into one of eight TMEM buffers; the epilogue warps (weight row =
 // TMEM lane, token = column) add P * (sa[kb][token] * sw[nb][kb]) into FP32
 // registers.  A weight block whose whole K range lies inside one share is
 // written as bf16 at once.  A block cut between shares goes to FP32 partial
@@ -75,8 +75,11 @@ struct DCfg {
   static constexpr int kFit = (kStageBudget - kResBytes) / (kABytes + kBBytes + kSSlot);
   static constexpr int kStages = kFit < 8 ? kFit : 8;
   static constexpr int kCW = NT / 2;         // token columns per epilogue warpgroup
-  static constexpr int kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
-  static constexpr int kSmemBytes = kStages * (kABytes + kBBytes + kSSlot) + kResBytes + 256 + 64 + 1024;
+  // TMEM accumulator buffers: a work item's partial is only NT columns, so
+  // eight of them fit and the MMA can run eight items ahead of the epilogue
+  static constexpr int kTBufs = 8;
+  static constexpr int kTmemCols = kTBufs * NT;   // 128, 256 or 512: a power of two
+  static constexpr int kSmemBytes = kStages * (kABytes + kBBytes + kSSlot) + kResBytes + 512 + 1024;
   static_assert(!kRes || NT == kResMaxM, "resident activation codes only for NT = 16");
   static_assert(kStages >= 3 && kSmemBytes <= 232448, "decode shared memory budget");
 };
@@ -166,8 +169,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
   uint64_t *full = bars;
   uint64_t *empty = bars + C::kStages;
   uint64_t *tfull = empty + C::kStages;
-  uint64_t *tempty = tfull + 2;
-  uint64_t *drain = tempty + 2;
+  uint64_t *tempty = tfull + C::kTBufs;
+  uint64_t *drain = tempty + C::kTBufs;
   uint64_t *xready = drain + 1;
   uint64_t *fl_in = xready + 1;   // cut-block flush: all epilogue warps have written their partials
   uint64_t *fl_out = fl_in + 1;   // cut-block flush: the arrival has been counted
@@ -186,9 +189,10 @@ __global__ void __launch_bounds__(kDThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + kDEpiWarps);  // MMA commit + every epilogue warp (they read the scales)
+      // MMA commit, and with scales in the stage every epilogue warp too
+      mbar_init(&empty[s], kRes ? 1 : 1 + kDEpiWarps);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kTBufs; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], kDEpiWarps);
     }
@@ -261,7 +265,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(buf * NT);
         const uint32_t a0 = smem_addr(sA + stage * C::kABytes);
-        uint32_t b0;
+        uint32_t b0 = 0;
         if constexpr (kRes) {
           const int kb = (int)(p % KB);
           const int slot = kb - kb_first + (kb < kb_first ? KB : 0);
@@ -279,7 +283,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
           stage = 0;
           phase ^= 1;
         }
-        if (++buf == 2) {
+        if (++buf == C::kTBufs) {
           buf = 0;
           bphase ^= 1;
         }
@@ -367,10 +371,12 @@ __global__ void __launch_bounds__(kDThreads, 1)
         acc[4 * j + 2] = fmaf(__uint_as_float(v[4 * j + 2]), s4.z * w, acc[4 * j + 2]);
         acc[4 * j + 3] = fmaf(__uint_as_float(v[4 * j + 3]), s4.w * w, acc[4 * j + 3]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[stage]);  // the stage's scales have been read
+      if constexpr (!kRes) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);  // the stage's scales have been read
+      }
       if (++stage == C::kStages) stage = 0;
-      if (++buf == 2) {
+      if (++buf == C::kTBufs) {
         buf = 0;
         bphase ^= 1;
       }
