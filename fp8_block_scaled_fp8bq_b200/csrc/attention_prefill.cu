@@ -35,9 +35,10 @@
 // most 2^-4 each, as for any FP8 operand); the row sum l uses the unrounded
 // p_j.  Everything else is FP32.
 //
-// Roles (384 threads): warp 0 loads (TMA for Q, K and V; its lanes load the
-// key and value scales and form 256 vs_j / vmax); warp 1 owns TMEM and issues
-// the MMAs; warps 4-7 run the softmax, warps 8-11 the correction and output.
+// Roles (384 threads): warp 0 issues the TMA loads of Q, K and V; warp 1 owns
+// TMEM and issues the MMAs; warps 2 and 3 load the key and value scales of
+// alternate blocks and form 256 vs_j / vmax; warps 4-7 run the softmax,
+// warps 8-11 the correction and output.
 // Waits are bounded (a second); on expiry the kernel records the site in the
 // device error word and every role stops.
 #include <cuda_bf16.h>
@@ -105,6 +106,50 @@ __device__ __forceinline__ Unit unit_at(int u, const AttnArgs &a) {
   x.nblk = kBQ * x.t < x.L ? x.t + 1 : 0;
   return x;
 }
+
+// The key blocks a CTA processes, in its order (n counts them): units
+// blockIdx.x, blockIdx.x + gridDim.x, ..., blocks 0 .. nblk-1 of each.
+struct BlockIter {
+  const AttnArgs *a;
+  int nunits, u, kb;
+  Unit x;
+  uint32_t n;
+  bool valid;
+  __device__ BlockIter(const AttnArgs &args, int nu) : a(&args), nunits(nu), u((int)blockIdx.x - (int)gridDim.x),
+                                                        kb(0), n(0), valid(true) {
+    x.nblk = 0;
+    next_unit();
+  }
+  __device__ void next_unit() {
+    kb = 0;
+    for (u += gridDim.x; u < nunits; u += gridDim.x) {
+      x = unit_at(u, *a);
+      if (x.nblk > 0) return;
+    }
+    valid = false;
+  }
+  __device__ void advance() {
+    if (!valid) return;
+    ++n;
+    if (++kb == x.nblk) next_unit();
+  }
+  // advance to the first block at or after this one with n % 2 == parity
+  __device__ void skip_to(uint32_t parity) {
+    if (valid && (n & 1u) != parity) advance();
+  }
+  // key and value scales of keys 4 lane .. 4 lane + 3 of this block (0 past
+  // the sequence's length, and when there is no block)
+  __device__ void load(int lane, float (&k)[4], float (&v)[4]) const {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = kBK * kb + 4 * lane + i;
+      const bool live = valid && j < x.L;
+      const int64_t idx = ((int64_t)x.b * a->S + j) * a->Hkv + x.g;
+      k[i] = live ? __ldg(a->ks + idx) : 0.f;
+      v[i] = live ? __ldg(a->vs + idx) : 0.f;
+    }
+  }
+};
 
 // Shared-memory descriptor of an MN-major operand tile written by TMA with the
 // 128-byte swizzle: rows of 128 bytes hold 128 consecutive MN elements, one
@@ -246,32 +291,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
-          // key and value scales of the block: lane l takes keys 4l .. 4l+3;
-          // keys at or past the sequence's length are never visible and get 0
-          float *slot = reinterpret_cast<float *>(sScale + st * kScaleSlot);
-          float kscale[4], vscale[4], vmax = 0.f;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int j = kBK * kb + 4 * lane + i;
-            const bool live = j < x.L;
-            const int64_t idx = ((int64_t)x.b * args.S + j) * args.Hkv + x.g;
-            kscale[i] = live ? __ldg(args.ks + idx) : 0.f;
-            vscale[i] = live ? __ldg(args.vs + idx) : 0.f;
-            vmax = fmaxf(vmax, vscale[i]);
-          }
-#pragma unroll
-          for (int d = 16; d > 0; d >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, d));
-          float4 rv;
-          const float inv = vmax > 0.f ? __fdiv_rn(256.f, vmax) : 0.f;
-          rv.x = vscale[0] * inv;
-          rv.y = vscale[1] * inv;
-          rv.z = vscale[2] * inv;
-          rv.w = vscale[3] * inv;
-          reinterpret_cast<float4 *>(slot)[lane] = make_float4(kscale[0], kscale[1], kscale[2], kscale[3]);
-          reinterpret_cast<float4 *>(slot + kBK)[lane] = rv;
-          if (lane == 0) slot[2 * kBK] = vmax * (1.f / 256.f);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&B.kv_full[st]);
         }
         ++v;
       }
@@ -280,6 +299,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (armed >> s & 1u) mbar_wait(&B.kv_full[s], (armed_par >> s) & 1u, nullptr, kSiteDrain);
         for (int s = 0; s < 2; ++s)
           if (qarmed >> s & 1u) mbar_wait(&B.q_full[s], (qarmed_par >> s) & 1u, nullptr, kSiteDrain);
+      }
+    } else if (warp >= 2) {
+      // ------------------------------------------------------------------ key / value scales
+      // Warp 2 serves the even blocks (in the CTA's block order n), warp 3 the
+      // odd ones, each with the next block's loads in flight while it waits for
+      // the current block's stage: lane l takes keys 4l .. 4l+3 of the block;
+      // keys at or past the sequence's length are never visible and get 0.
+      const uint32_t mine = (uint32_t)(warp - 2);
+      BlockIter it(args, nunits);
+      it.skip_to(mine);
+      float kc[4], vc[4];
+      it.load(lane, kc, vc);
+      bool ok = true;
+      while (it.valid && ok) {
+        const uint32_t n = it.n;
+        BlockIter nx = it;
+        nx.advance();
+        nx.skip_to(mine);
+        float kn[4], vn[4];
+        nx.load(lane, kn, vn);  // in flight during the wait below
+        const int st = n % kStages;
+        if (lane == 0) ok = mbar_wait(&B.kv_empty[st], ((n / kStages) & 1) ^ 1, abort_flag, kSiteAttnKV);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        float vmax = fmaxf(fmaxf(vc[0], vc[1]), fmaxf(vc[2], vc[3]));
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, d));
+        const float inv = vmax > 0.f ? __fdiv_rn(256.f, vmax) : 0.f;
+        float *slot = reinterpret_cast<float *>(sScale + st * kScaleSlot);
+        reinterpret_cast<float4 *>(slot)[lane] = make_float4(kc[0], kc[1], kc[2], kc[3]);
+        reinterpret_cast<float4 *>(slot + kBK)[lane] = make_float4(vc[0] * inv, vc[1] * inv, vc[2] * inv, vc[3] * inv);
+        if (lane == 0) slot[2 * kBK] = vmax * (1.f / 256.f);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.kv_full[st]);
+        it = nx;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          kc[i] = kn[i];
+          vc[i] = vn[i];
+        }
       }
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------------ MMA issuer

@@ -129,13 +129,11 @@ __device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t *r) {
 // chunk position c ^ (m & 7)); lane qd of the group owns chunks qd, qd + 4,
 // qd + 8, qd + 12 of the row, as fp8bq_quant_act's vector kernel does.
 // Every lane of the warp calls it (the amax shuffles span the warp); lanes
-// with have == false load nothing and store nothing.
+// with have == false store nothing.  v: the lane's four 16-byte pieces of the
+// row (pieces qd, qd + 4, qd + 8, qd + 12), loaded by the caller.
 template <int MODE>
-__device__ __forceinline__ void quant_row_tile_to_smem(bool have, const uint16_t *__restrict__ xrow, int qd,
-                                                       uint8_t *tile, int m, float *scale) {
-  uint4 v[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) v[j] = have ? ld_nc_v4(xrow + (j * 4 + qd) * 8) : make_uint4(0, 0, 0, 0);
+__device__ __forceinline__ void quant_row_tile_to_smem(bool have, const uint4 (&v)[4], int qd, uint8_t *tile, int m,
+                                                       float *scale) {
   uint32_t am = max(max(qdev::absmax_bits8(v[0]), qdev::absmax_bits8(v[1])),
                     max(qdev::absmax_bits8(v[2]), qdev::absmax_bits8(v[3])));
   am = max(am, __shfl_xor_sync(0xffffffffu, am, 1));
@@ -176,7 +174,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
   uint64_t *fl_out = fl_in + 1;   // cut-block flush: the arrival has been counted
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fl_out + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  volatile int *last_flag = abort_flag + 1;
+  volatile int *last_flag = abort_flag + 1;  // [2]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KB = args.KB;
@@ -306,16 +304,29 @@ __global__ void __launch_bounds__(kDThreads, 1)
       }
       for (int z = et; z < nkb * NT; z += 256) sXs[z] = 0.f;
       __syncwarp();
-      // tile (i, m) for i < nkb, m < M, four lanes each; groups never straddle a warp
+      // tile (i, m) for i < nkb, m < M, four lanes each; groups never straddle a
+      // warp.  Passes of 64 tiles; the loads of up to kChunk passes are issued
+      // together so that their latencies overlap
+      constexpr int kChunk = 4;
       const int grp = et >> 2, qd = et & 3;
       const int ntile = nkb * args.M;
-      for (int t0 = 0; t0 < ntile; t0 += 64) {
-        const int t = t0 + grp;
-        const bool have = t < ntile;
-        const int i = have ? t / args.M : 0, m = have ? t - (t / args.M) * args.M : 0;
-        const int kb = (kb_first + i) % KB;
-        quant_row_tile_to_smem<QM < 0 ? 0 : QM>(have, args.x + (int64_t)m * args.ldx + (int64_t)kb * DBK, qd,
-                                                sXr + i * (NT * DBK), m, sXs + i * NT + m);
+      for (int c0 = 0; c0 < ntile; c0 += 64 * kChunk) {
+        uint4 v[kChunk][4];
+#pragma unroll
+        for (int u = 0; u < kChunk; ++u) {
+          const int t = c0 + 64 * u + grp;
+          const int i = t / args.M, m = t - (t / args.M) * args.M;
+          const uint16_t *xrow = args.x + (int64_t)m * args.ldx + (int64_t)((kb_first + i) % KB) * DBK;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) v[u][j] = t < ntile ? ld_nc_v4(xrow + (j * 4 + qd) * 8) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kChunk; ++u) {
+          const int t = c0 + 64 * u + grp;
+          const bool have = t < ntile;
+          const int i = have ? t / args.M : 0, m = have ? t - (t / args.M) * args.M : 0;
+          quant_row_tile_to_smem<QM < 0 ? 0 : QM>(have, v[u], qd, sXr + i * (NT * DBK), m, sXs + i * NT + m);
+        }
       }
       __syncwarp();
       fence_proxy_async_smem();
@@ -328,7 +339,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
     const int c0 = h * C::kCW;          // first token column of this warpgroup
     const int r = quarter * 32 + lane;  // weight row within the block = output column
     int stage = 0, buf = 0;
-    uint32_t bphase = 0, fphase = 0;
+    uint32_t bphase = 0;
+    int cut_nb[2] = {0, 0}, ncut = 0;  // weight blocks of this share that other shares hold too
+    bool done = true;
     float acc[C::kCW];
 #pragma unroll
     for (int j = 0; j < C::kCW; ++j) acc[j] = 0.f;
@@ -342,7 +355,10 @@ __global__ void __launch_bounds__(kDThreads, 1)
       w0 = w1;
       if (p + 2 < p_end) w1 = __ldg(args.sw + p + 2);
       const bool got = mbar_wait(&tfull[buf], bphase, abort_flag, kSiteEpiTmemFull);
-      if (!__all_sync(0xffffffffu, got)) break;
+      if (!__all_sync(0xffffffffu, got)) {
+        done = false;
+        break;
+      }
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * NT + c0);
       const float4 *sc4;
@@ -392,54 +408,71 @@ __global__ void __launch_bounds__(kDThreads, 1)
               if (c0 + j < args.M) args.y[(int64_t)(c0 + j) * args.ldy + n] = bf16_bits(acc[j]);
           }
         } else {
-          // slot 0: the run holding the share's first item; slot 1: the last run
+          // slot 0: the run holding the share's first item; slot 1: the last
+          // run.  The block is counted and reduced after the share's last item.
           const int which = (run0 == p_begin) ? 0 : 1;
           float *dst = args.part + ((int64_t)(blockIdx.x * 2 + which) * args.M) * DBM + r;
 #pragma unroll
           for (int j = 0; j < C::kCW; ++j)
             if (c0 + j < args.M) dst[(int64_t)(c0 + j) * DBM] = acc[j];
-          // count this CTA on the block; the last of its CTAs to arrive adds
-          // every CTA's partial slot in CTA order
-          const int64_t first = (int64_t)nb * KB, last = first + KB - 1;
-          const int64_t cf = share_of(first, args.W, args.G), cl = share_of(last, args.W, args.G);
-          // (mbarrier hand-offs with bounded waits, so an abort elsewhere in
-          // the CTA cannot leave a warp waiting here)
-          __threadfence();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(fl_in);
-          bool fine = true;
-          if (et == 0) {
-            fine = mbar_wait(fl_in, fphase, abort_flag, kSiteEpiTmemFull);
-            int is_last = 0;
-            if (fine) {
-              const int prior = atomicAdd(args.cnt + cf, 1);
-              is_last = prior == (int)(cl - cf);
-              if (is_last) {
-                __threadfence();
-                args.cnt[cf] = 0;  // left zero for the next call (every arrival has been counted)
-              }
-            }
-            *last_flag = is_last;
-            mbar_arrive(fl_out);
-          }
-          fine = mbar_wait(fl_out, fphase, abort_flag, kSiteEpiTmemFull) && fine;
-          fphase ^= 1;
-          if (!__all_sync(0xffffffffu, fine)) break;
-          if (*last_flag && n < args.N) {
-#pragma unroll
-            for (int j = 0; j < C::kCW; ++j) {
-              if (c0 + j >= args.M) continue;
-              float sum = 0.f;
-              for (int64_t c = cf; c <= cl; ++c) {
-                const int wc = share_begin(c, args.W, args.G) >= first ? 0 : 1;
-                sum += __ldcg(args.part + ((c * 2 + wc) * args.M + c0 + j) * DBM + r);
-              }
-              args.y[(int64_t)(c0 + j) * args.ldy + n] = bf16_bits(sum);
-            }
-          }
+          cut_nb[ncut++] = nb;
         }
 #pragma unroll
         for (int j = 0; j < C::kCW; ++j) acc[j] = 0.f;
+      }
+    }
+    // Count this CTA on each cut block it holds; the last CTA to arrive adds
+    // every sharing CTA's partial slot in CTA order.  (Hand-offs on bounded
+    // mbarriers, so an abort elsewhere in the CTA cannot leave a warp waiting.)
+    if (done && ncut > 0) {
+      __threadfence();  // this thread's partial slots are visible to the other CTAs
+      __syncwarp();
+      if (lane == 0) mbar_arrive(fl_in);
+      bool fine = true;
+      if (et == 0) {
+        fine = mbar_wait(fl_in, 0, abort_flag, kSiteEpiTmemFull);
+        for (int i = 0; i < ncut; ++i) {
+          int is_last = 0;
+          if (fine) {
+            const int64_t first = (int64_t)cut_nb[i] * KB;
+            const int64_t cf = share_of(first, args.W, args.G), cl = share_of(first + KB - 1, args.W, args.G);
+            const int prior = atomicAdd(args.cnt + cf, 1);
+            is_last = prior == (int)(cl - cf);
+            if (is_last) {
+              __threadfence();
+              args.cnt[cf] = 0;  // left zero for the next call (every arrival has been counted)
+            }
+          }
+          last_flag[i] = is_last;
+        }
+        mbar_arrive(fl_out);
+      }
+      fine = mbar_wait(fl_out, 0, abort_flag, kSiteEpiTmemFull) && fine;
+      if (__all_sync(0xffffffffu, fine)) {
+        for (int i = 0; i < ncut; ++i) {
+          if (!last_flag[i]) continue;
+          const int nb = cut_nb[i];
+          const int n = nb * DBM + r;
+          const int64_t first = (int64_t)nb * KB;
+          const int64_t cf = share_of(first, args.W, args.G), cl = share_of(first + KB - 1, args.W, args.G);
+          float sum[C::kCW];
+#pragma unroll
+          for (int j = 0; j < C::kCW; ++j) sum[j] = 0.f;
+          for (int64_t c = cf; c <= cl; ++c) {
+            const int wc = share_begin(c, args.W, args.G) >= first ? 0 : 1;
+            const float *src = args.part + ((c * 2 + wc) * args.M + c0) * DBM + r;
+            float v[C::kCW];  // one CTA's slot: independent loads, issued together
+#pragma unroll
+            for (int j = 0; j < C::kCW; ++j) v[j] = (c0 + j < args.M) ? __ldcg(src + (int64_t)j * DBM) : 0.f;
+#pragma unroll
+            for (int j = 0; j < C::kCW; ++j) sum[j] += v[j];
+          }
+          if (n < args.N) {
+#pragma unroll
+            for (int j = 0; j < C::kCW; ++j)
+              if (c0 + j < args.M) args.y[(int64_t)(c0 + j) * args.ldy + n] = bf16_bits(sum[j]);
+          }
+        }
       }
     }
   }
@@ -530,7 +563,8 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
   if (M > kMaxDecodeM) return FP8BQ_ERR_UNSUPPORTED;
   const bool vec = aligned(x, 16) && ldx % 8 == 0;  // K % 128 == 0 already
   const Plan p = make_plan(M, N, K, vec);
-  if (ws == nullptr || ws_bytes < p.total || !aligned(ws, 256)) return FP8BQ_ERR_WORKSPACE;
+  // the documented size (the larger plan's), whichever path this call takes
+  if (ws == nullptr || ws_bytes < make_plan(M, N, K, false).total || !aligned(ws, 256)) return FP8BQ_ERR_WORKSPACE;
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   uint8_t *q = wsb + p.off_q;
   float *sa = reinterpret_cast<float *>(wsb + p.off_sa);
