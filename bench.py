@@ -689,7 +689,8 @@ def reference(args):
 CASES = (["gemm:" + n for n in NAMES] + ["decode:" + n for n in NAMES] + ["cublas:" + n for n in NAMES] +
          ["quant_act:4096", "quant_act:14336", "recalibrate:layer", "quant_weight:gate_up", "moe:up", "moe:down",
           "swiglu:gate_up", "moe_swiglu:up", "adamw_recal:layer", "quant_act_t:4096", "quant_act_t:14336",
-          "transpose_weight:gate_up", "prefill_attn:4x2048", "prefill_attn:1x8192", "decode_attn:1x32768", "decode_attn:16x8192", "decode_attn:64x4096",
+          "transpose_weight:gate_up", "prefill_attn:4x2048", "prefill_attn:1x2048", "prefill_attn:1x8192",
+          "decode_attn:1x32768", "decode_attn:16x8192", "decode_attn:64x4096",
           "decode_attn:256x2048", "recalibrate:model"] + ["dgrad:" + n for n in NAMES] +
          ["wgrad:" + n for n in NAMES])
 

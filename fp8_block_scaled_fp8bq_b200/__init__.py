@@ -303,16 +303,15 @@ def gemm_decode_workspace_size(M, N, K):
 
 
 def gemm_decode(x, qw, sw, mode=SCALE_FP32, out=None, ws=None, stream=None):
-    """Small-M linear with on-the-fly 1x128 activation quantization.  A caller
-    workspace `ws` (uint8, gemm_decode_workspace_size bytes) must be zero-filled
-    before its first use; every call leaves it reusable."""
+    """Small-M linear with on-the-fly 1x128 activation quantization (`ws`: an
+    optional uint8 workspace of gemm_decode_workspace_size bytes)."""
     M, K = x.shape
     N = qw.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     need = gemm_decode_workspace_size(M, N, K)
-    if ws is None:  # its counter area must start zeroed (each call leaves it so)
-        ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=x.device)
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
     _check(lib().fp8bq_gemm_decode(_ptr(x), _ld(x), _ptr(qw), _ld(qw), _ptr(sw), _ptr(out), _ld(out), M, N, K,
                                    mode, _ptr(ws), ws.numel(), _stream(stream)), "fp8bq_gemm_decode")
     return out

@@ -174,6 +174,39 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x for x <= 0 on the FMA and integer pipes instead of the special-function
+// unit (which is the softmax's bottleneck when it computes every
+// exponential): x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the
+// low bits of the sum) and f in [-1/2, 1/2]; 2^f by a cubic fitted to it
+// (maximum relative error 1.0e-4, evaluated by Horner's rule in FP32); 2^n
+// enters by adding n to the exponent field.  x is clamped to -125, below
+// which the weight is far under the E4M3 weights' smallest step anyway.
+__device__ __forceinline__ float ex2_poly(float x) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  x = fmaxf(x, -125.f);
+  const float j = __fadd_rn(x, kShift);
+  const float f = __fsub_rn(x, __fsub_rn(j, kShift));
+  float p = __fmaf_rn(0.05500892922282219f, f, 0.24221095442771912f);
+  p = __fmaf_rn(p, f, 0.6932829022407532f);
+  p = __fmaf_rn(p, f, 1.f);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(j) << 23));
+}
+
+// E4M3 code (round to nearest even) of w in [0, 448] on the integer and FMA
+// pipes instead of the conversion unit.  Normal range (w >= 2^-6): round the
+// binary32 pattern to 3 fraction bits (add 0x7FFFF plus the lowest kept bit),
+// then rebias the exponent from 127 to 7.  Below 2^-6 (E4M3 subnormals, steps
+// of 2^-9): adding 1.5 * 2^14 rounds w to a multiple of 2^-9 whose count is
+// left in the low bits of the sum (count 8 is 2^-6, the smallest normal code).
+// Checked against the conversion's definition on every binary32 value in
+// [0, 448].
+__device__ __forceinline__ uint32_t e4m3_nonneg(float w) {
+  const uint32_t u = __float_as_uint(w);
+  const uint32_t normal = ((u + 0x7FFFFu + ((u >> 20) & 1u)) >> 20) - (120u << 3);
+  const uint32_t sub = __float_as_uint(__fadd_rn(w, 24576.f)) - 0x46C00000u;
+  return w < 0.015625f ? sub : normal;
+}
+
 struct Bars {
   uint64_t *kv_full, *kv_empty;   // [kStages]
   uint64_t *q_full, *q_empty;     // [2]
@@ -448,30 +481,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float *slot = reinterpret_cast<const float *>(sScale + st * kScaleSlot);
         const float4 *ks4 = reinterpret_cast<const float4 *>(slot);
         const float4 *rv4 = reinterpret_cast<const float4 *>(slot + kBK);
-        // s_j = S_rj * ks_j and the block's row max (visible keys only)
+        // s_j = S_rj * ks_j and the block's row max over the visible keys.
+        // Masking is by selects (no branches); four partial maxima and four
+        // partial sums keep the dependency chains short, since one warp per
+        // scheduler runs this loop.
         const int vis = kb == x.t ? r : kBK - 1;  // last visible key of the block
-        float mx = -INFINITY;
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int j4 = 0; j4 < kBK / 4; ++j4) {
           const float4 k4 = ks4[j4];
-          const float s0 = __uint_as_float(sr[4 * j4 + 0]) * k4.x, s1 = __uint_as_float(sr[4 * j4 + 1]) * k4.y;
-          const float s2 = __uint_as_float(sr[4 * j4 + 2]) * k4.z, s3 = __uint_as_float(sr[4 * j4 + 3]) * k4.w;
-          sr[4 * j4 + 0] = __float_as_uint(s0);
-          sr[4 * j4 + 1] = __float_as_uint(s1);
-          sr[4 * j4 + 2] = __float_as_uint(s2);
-          sr[4 * j4 + 3] = __float_as_uint(s3);
-          if (4 * j4 + 3 <= vis) {
-            mx = fmaxf(mx, fmaxf(fmaxf(s0, s1), fmaxf(s2, s3)));
-          } else {
-            if (4 * j4 + 0 <= vis) mx = fmaxf(mx, s0);
-            if (4 * j4 + 1 <= vis) mx = fmaxf(mx, s1);
-            if (4 * j4 + 2 <= vis) mx = fmaxf(mx, s2);
+          float sv[4] = {__uint_as_float(sr[4 * j4 + 0]) * k4.x, __uint_as_float(sr[4 * j4 + 1]) * k4.y,
+                         __uint_as_float(sr[4 * j4 + 2]) * k4.z, __uint_as_float(sr[4 * j4 + 3]) * k4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            sv[e] = 4 * j4 + e <= vis ? sv[e] : -INFINITY;
+            sr[4 * j4 + e] = __float_as_uint(sv[e]);
+            mx4[e] = fmaxf(mx4[e], sv[e]);
           }
         }
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
         // c > 0, so the max of c s is c times the max of s
         const float m_new = fmaxf(m, c * mx);
         const float alpha = ex2(m - m_new);  // 0 on the first block (m = -inf)
-        float sum = 0.f;
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[32];  // 128 E4M3 codes, 4 per word
 #pragma unroll
         for (int j4 = 0; j4 < kBK / 4; ++j4) {
@@ -479,14 +511,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           float p[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int j = 4 * j4 + e;
-            p[e] = j <= vis ? ex2(__fmaf_rn(c, __uint_as_float(sr[j]), -m_new)) : 0.f;
-            sum += p[e];
+            p[e] = ex2(__fmaf_rn(c, __uint_as_float(sr[4 * j4 + e]), -m_new));  // masked keys: 2^-inf = 0
+            sum4[e] += p[e];
           }
           const uint32_t lo = qdev::e4m3x2(p[0] * w4.x, p[1] * w4.y);
           const uint32_t hi = qdev::e4m3x2(p[2] * w4.z, p[3] * w4.w);
           pk[j4] = lo | (hi << 16);
         }
+        const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
         l = alpha * l + sum;
         m = m_new;
         // P' row r into the 128-byte-swizzled K-major tile (the A operand)

@@ -10,30 +10,29 @@
 //
 // The GEMM runs with the operands swapped so that the tensor cores do useful
 // work at small M: the weight is the 128-row MMA operand and the tokens are
-// the MMA's N dimension (NT = M rounded up to 16, 32 or 64).  The NB x KB grid
-// of (128-row weight block, 128-deep K-block) work items is cut, in
-// weight-block-major order, into one contiguous equal share per CTA, so every
-// SM streams the same number of weight bytes whatever NB is.  Per work item:
-// the weight tile (16 KB) comes through a TMA stage ring; 4 x tcgen05.mma
-// 128xNTx32 go into one of eight TMEM buffers; the epilogue warps (weight row =
-// TMEM lane, token = column) add P * (sa[kb][token] * sw[nb][kb]) into FP32
-// registers.  A weight block whose whole K range lies inside one share is
-// written as bf16 at once.  A block cut between shares goes to FP32 partial
-// slots in the workspace; each CTA that holds part of it then counts itself
-// on the block's counter, and the last one to arrive adds all the partial
-// slots in CTA order (deterministic) and writes the bf16 result, then resets
-// the counter to 0 (so the workspace's counter area must be zero before the
-// first call and is left zero by every call).
+// the MMA's N dimension (NT = M rounded up to 16, 32 or 64).  A work item is a
+// (128-row weight block nb, 128-deep K-block kb) pair: the weight tile (16 KB)
+// comes through a TMA stage ring; 4 x tcgen05.mma 128xNTx32 go into one of
+// eight TMEM buffers; the epilogue warps (weight row = TMEM lane, token =
+// column) add P * (sa[kb][token] * sw[nb][kb]) into FP32 registers.
+//
+// Split over K in thread-block clusters: a cluster of S CTAs owns whole weight
+// blocks (blocks c, c + C, c + 2C, ... for cluster c of C), and CTA rank r of
+// the cluster takes K-blocks [r KB / S, (r + 1) KB / S) of each.  The host
+// picks S (1..8) and C so that the largest per-CTA item count is smallest.
+// At the end of a block every rank r > 0 leaves its FP32 partial in its own
+// shared memory and signals rank 0, which adds the partials in rank order
+// (over distributed shared memory: deterministic, no global atomics) and
+// writes the bf16 result.
 //
 // The activation's 1x128 quantization (the device code of fp8bq_quant_act):
-//   M <= 16: inside the same kernel.  Each CTA quantizes the K-blocks its share
-//     touches (at most kMaxResKB) into shared memory, in the MMA's operand
-//     layout, while the weight ring is filling: one launch per call;
-//   16 < M <= 64: a prologue kernel writes the codes and scales to the
-//     workspace and the GEMM's producer loads them with TMA beside the weight
-//     tiles (two launches);
-//   M > 64: the per-token promotion costs more than the weight stream, so the
-//     prologue is followed by the prefill GEMM.
+//   inside the same kernel when M <= 16 and a CTA's K range holds at most 256
+//     1x128 tiles of X: the epilogue warps quantize them into shared memory in
+//     the MMA's operand layout while the weight ring fills (one launch);
+//   otherwise a prologue kernel writes the codes and scales to the workspace
+//     and the producer loads them with TMA beside the weight tiles (M <= 64),
+//     or the prologue is followed by the prefill GEMM (M > 64, where the
+//     per-token promotion costs more than the weight stream).
 #include <cuda_bf16.h>
 #include <string.h>
 
@@ -54,12 +53,13 @@ constexpr int kDHighRegs = 224;
 static_assert(128 * kDLowRegs + 256 * kDHighRegs <= kDThreads * kDLaunchRegs, "register split");
 constexpr int kMaxDecodeM = 256;
 constexpr int kSwapMaxM = 64;
-constexpr int kResMaxM = 16;        // activation quantized inside the GEMM kernel up to this M
+constexpr int kResMaxM = 16;        // activation quantized inside the GEMM kernel up to this M ...
+constexpr int kResMaxTiles = 256;   // ... when a CTA's K range holds at most this many 1x128 tiles of X
 constexpr int kMaxResKB = 48;       // K-blocks of resident activation codes per CTA
+constexpr int kMaxSplit = 8;        // CTAs of a cluster (split of K)
 constexpr int kDEpiWarps = 8;
 constexpr int kStageBudget = 212992;
-constexpr int kMaxShares = 1024;    // CTAs of one call (counter area: kMaxShares ints)
-constexpr size_t kCounterBytes = kMaxShares * 4;
+constexpr int kSwSlots = 512;       // weight scales of a CTA's first work items, staged in shared memory
 
 // QM < 0: activation codes and scales come from the workspace (TMA, beside the
 // weight tiles); QM = FP8BQ_SCALE_FP32 / POW2: quantized in the kernel (NT = 16).
@@ -72,14 +72,16 @@ struct DCfg {
   static constexpr int kSSlot = (kSBytes + 127) / 128 * 128;
   static constexpr int kTx = kABytes + kBBytes + kSBytes;
   static constexpr int kResBytes = kRes ? kMaxResKB * (NT * DBK + NT * 4) : 0;
-  static constexpr int kFit = (kStageBudget - kResBytes) / (kABytes + kBBytes + kSSlot);
+  static constexpr int kPartBytes = NT * DBM * 4;           // a block's FP32 partial, for rank 0 of the cluster
+  static constexpr int kFit = (kStageBudget - kResBytes - kPartBytes) / (kABytes + kBBytes + kSSlot);
   static constexpr int kStages = kFit < 8 ? kFit : 8;
   static constexpr int kCW = NT / 2;         // token columns per epilogue warpgroup
   // TMEM accumulator buffers: a work item's partial is only NT columns, so
   // eight of them fit and the MMA can run eight items ahead of the epilogue
   static constexpr int kTBufs = 8;
   static constexpr int kTmemCols = kTBufs * NT;   // 128, 256 or 512: a power of two
-  static constexpr int kSmemBytes = kStages * (kABytes + kBBytes + kSSlot) + kResBytes + 512 + 1024;
+  static constexpr int kSmemBytes =
+      kStages * (kABytes + kBBytes + kSSlot) + kResBytes + kPartBytes + kSwSlots * 4 + 512 + 1024;
   static_assert(!kRes || NT == kResMaxM, "resident activation codes only for NT = 16");
   static_assert(kStages >= 3 && kSmemBytes <= 232448, "decode shared memory budget");
 };
@@ -87,26 +89,30 @@ struct DCfg {
 struct DecodeArgs {
   const float *sw;
   int32_t M, N, KB, NB;
-  int64_t W;      // NB * KB work items
-  int32_t G;      // CTAs (shares)
-  float *part;    // [G][2][M][128] partial slots
-  int *cnt;       // [kMaxShares] arrival counters of cut weight blocks (zero between calls)
-  uint16_t *y;    // bf16 bits
+  int32_t split;      // CTAs per cluster (S)
+  uint16_t *y;        // bf16 bits
   int64_t ldy;
   const uint16_t *x;  // resident quantization: bf16 activations [M][ldx]
   int64_t ldx;
 };
 
-// First work item of CTA c's share.
-__host__ __device__ __forceinline__ int64_t share_begin(int64_t c, int64_t W, int64_t G) { return c * W / G; }
-
-// The CTA whose share holds work item p.
-__host__ __device__ __forceinline__ int64_t share_of(int64_t p, int64_t W, int64_t G) {
-  int64_t c = p * G / W;
-  while (c + 1 < G && share_begin(c + 1, W, G) <= p) ++c;
-  while (c > 0 && share_begin(c, W, G) > p) --c;
-  return c;
-}
+// The work of CTA `rank` of cluster `cid` (of `ncl`): weight blocks cid,
+// cid + ncl, ... and K-blocks [kb0, kb1) of each; item q is block
+// nb0 + (q / nk) * ncl, K-block kb0 + q % nk.
+struct Share {
+  int nb0, ncl, kb0, kb1, nk, nblk, items;
+  __device__ Share(const DecodeArgs &a, int cid, int ncls, int rank) {
+    nb0 = cid;
+    ncl = ncls;
+    kb0 = (int)((int64_t)rank * a.KB / a.split);
+    kb1 = (int)((int64_t)(rank + 1) * a.KB / a.split);
+    nk = kb1 - kb0;
+    nblk = cid < a.NB ? (a.NB - cid + ncls - 1) / ncls : 0;
+    items = nblk * nk;
+  }
+  __device__ int nb(int q) const { return nb0 + (q / nk) * ncl; }
+  __device__ int kb(int q) const { return kb0 + q % nk; }
+};
 
 __device__ __forceinline__ uint16_t bf16_bits(float v) {
   __nv_bfloat16 b = __float2bfloat16_rn(v);
@@ -163,26 +169,25 @@ __global__ void __launch_bounds__(kDThreads, 1)
   uint8_t *sS = sB + C::kStages * C::kBBytes;  // kStages slots of kSSlot bytes (128-byte aligned)
   uint8_t *sXr = sS + C::kStages * C::kSSlot;  // resident codes: kMaxResKB tiles of NT x 128 B
   float *sXs = reinterpret_cast<float *>(sXr + (kRes ? kMaxResKB * NT * DBK : 0));  // [kMaxResKB][NT]
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sXr + C::kResBytes);
+  float *sPart = reinterpret_cast<float *>(sXr + C::kResBytes);  // [NT][128]: this CTA's partial of a block
+  float *sSw = sPart + NT * DBM;                                  // [kSwSlots]: sw of items 0, 1, ...
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sSw + kSwSlots);
   uint64_t *full = bars;
   uint64_t *empty = bars + C::kStages;
   uint64_t *tfull = empty + C::kStages;
   uint64_t *tempty = tfull + C::kTBufs;
   uint64_t *drain = tempty + C::kTBufs;
   uint64_t *xready = drain + 1;
-  uint64_t *fl_in = xready + 1;   // cut-block flush: all epilogue warps have written their partials
-  uint64_t *fl_out = fl_in + 1;   // cut-block flush: the arrival has been counted
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fl_out + 1);
+  uint64_t *red_full = xready + 1;  // rank 0: the other ranks' partials of the current block are in place
+  uint64_t *red_free = red_full + 1;  // rank > 0: rank 0 has read this CTA's partial
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(red_free + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  volatile int *last_flag = abort_flag + 1;  // [2]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int KB = args.KB;
-  const int64_t p_begin = share_begin(blockIdx.x, args.W, args.G);
-  const int64_t p_end = share_begin(blockIdx.x + 1, args.W, args.G);
-  // the K-blocks this share touches: slot i holds K-block (kb_first + i) % KB
-  const int kb_first = (int)(p_begin % KB);
-  const int nkb = (int)(p_end - p_begin < (int64_t)KB ? p_end - p_begin : (int64_t)KB);
+  const int S = args.split;
+  const int rank = S > 1 ? (int)cluster_ctarank() : 0;
+  const Share sh(args, S > 1 ? (int)cluster_id_x() : (int)blockIdx.x, S > 1 ? (int)nclusters_x() : (int)gridDim.x,
+                 rank);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -196,8 +201,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
     }
     mbar_init(drain, 1);
     mbar_init(xready, kDEpiWarps);
-    mbar_init(fl_in, kDEpiWarps);
-    mbar_init(fl_out, 1);
+    mbar_init(red_full, (S - 1) * kDEpiWarps);
+    mbar_init(red_free, kDEpiWarps);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -214,6 +219,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (S > 1) cluster_sync();  // every CTA's barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -224,8 +230,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       bool ok = true;
-      for (int64_t p = p_begin; p < p_end; ++p) {
-        const int nb = (int)(p / KB), kb = (int)(p - (int64_t)nb * KB);
+      for (int q = 0; q < sh.items; ++q) {
+        const int nb = sh.nb(q), kb = sh.kb(q);
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, kSiteProducerEmpty)) {
           ok = false;
           break;
@@ -254,7 +260,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
       uint32_t phase = 0, bphase = 0;
       bool ok = true, issued = false;
       if constexpr (kRes) ok = mbar_wait(xready, 0, abort_flag, kSiteMmaFull);  // the resident codes are written
-      for (int64_t p = p_begin; p < p_end && ok; ++p) {
+      for (int q = 0; q < sh.items && ok; ++q) {
         if (!mbar_wait(&tempty[buf], bphase ^ 1, abort_flag, kSiteMmaTmemEmpty) ||
             !mbar_wait(&full[stage], phase, abort_flag, kSiteMmaFull)) {
           ok = false;
@@ -264,13 +270,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
         const uint32_t d = tmem_base + (uint32_t)(buf * NT);
         const uint32_t a0 = smem_addr(sA + stage * C::kABytes);
         uint32_t b0 = 0;
-        if constexpr (kRes) {
-          const int kb = (int)(p % KB);
-          const int slot = kb - kb_first + (kb < kb_first ? KB : 0);
-          b0 = smem_addr(sXr + slot * (NT * DBK));
-        } else {
-          b0 = smem_addr(sB + stage * C::kBBytes);
-        }
+        if constexpr (kRes) b0 = smem_addr(sXr + (sh.kb(q) - sh.kb0) * (NT * DBK));
+        else b0 = smem_addr(sB + stage * C::kBBytes);
 #pragma unroll
         for (int k = 0; k < DBK / 32; ++k)
           mma_f8f6f4(d, smem_desc_k_sw128(a0 + 32 * k), smem_desc_k_sw128(b0 + 32 * k), idesc, k > 0 ? 1u : 0u);
@@ -294,15 +295,26 @@ __global__ void __launch_bounds__(kDThreads, 1)
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kDHighRegs));
     const int et = threadIdx.x - 128;   // 0..255
+    // the weight scale of every work item (sw is [NB][KB] row-major): read
+    // once, not per item
+    for (int q = et; q < kSwSlots && q < sh.items; q += 256)
+      sSw[q] = __ldg(args.sw + (int64_t)sh.nb(q) * args.KB + sh.kb(q));
+    if constexpr (!kRes) named_barrier_sync(1, 256);
     if constexpr (kRes) {
       // ------------------------------------------------------------ activation quantization
+      const int nkb = sh.nk;
       // rows M..NT-1 of every tile are zero (the MMA reads all NT rows)
       for (int z = et; z < nkb * (NT - args.M) * 8; z += 256) {
         const int i = z / ((NT - args.M) * 8), rr = z - i * (NT - args.M) * 8;
         const int m = args.M + rr / 8, c = rr % 8;
         *reinterpret_cast<uint4 *>(sXr + i * (NT * DBK) + m * 128 + c * 16) = make_uint4(0, 0, 0, 0);
       }
-      for (int z = et; z < nkb * NT; z += 256) sXs[z] = 0.f;
+      // and so are their scales (only those: rows below M get theirs from the
+      // quantization below, which may run first in another warp)
+      for (int z = et; z < nkb * (NT - args.M); z += 256) {
+        const int i = z / (NT - args.M);
+        sXs[i * NT + args.M + (z - i * (NT - args.M))] = 0.f;
+      }
       __syncwarp();
       // tile (i, m) for i < nkb, m < M, four lanes each; groups never straddle a
       // warp.  Passes of 64 tiles; the loads of up to kChunk passes are issued
@@ -316,7 +328,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
         for (int u = 0; u < kChunk; ++u) {
           const int t = c0 + 64 * u + grp;
           const int i = t / args.M, m = t - (t / args.M) * args.M;
-          const uint16_t *xrow = args.x + (int64_t)m * args.ldx + (int64_t)((kb_first + i) % KB) * DBK;
+          const uint16_t *xrow = args.x + (int64_t)m * args.ldx + (int64_t)(sh.kb0 + i) * DBK;
 #pragma unroll
           for (int j = 0; j < 4; ++j) v[u][j] = t < ntile ? ld_nc_v4(xrow + (j * 4 + qd) * 8) : make_uint4(0, 0, 0, 0);
         }
@@ -339,35 +351,20 @@ __global__ void __launch_bounds__(kDThreads, 1)
     const int c0 = h * C::kCW;          // first token column of this warpgroup
     const int r = quarter * 32 + lane;  // weight row within the block = output column
     int stage = 0, buf = 0;
-    uint32_t bphase = 0;
-    int cut_nb[2] = {0, 0}, ncut = 0;  // weight blocks of this share that other shares hold too
-    bool done = true;
+    uint32_t bphase = 0, rphase = 0;
     float acc[C::kCW];
 #pragma unroll
     for (int j = 0; j < C::kCW; ++j) acc[j] = 0.f;
-    // sw is [NB][KB] row-major, so work item p's weight scale is sw[p]; the
-    // next two are loaded ahead
-    float w0 = p_begin < p_end ? __ldg(args.sw + p_begin) : 0.f;
-    float w1 = p_begin + 1 < p_end ? __ldg(args.sw + p_begin + 1) : 0.f;
-    for (int64_t p = p_begin; p < p_end; ++p) {
-      const int nb = (int)(p / KB), kb = (int)(p - (int64_t)nb * KB);
-      const float w = w0;
-      w0 = w1;
-      if (p + 2 < p_end) w1 = __ldg(args.sw + p + 2);
+    for (int q = 0; q < sh.items; ++q) {
+      const int kb = sh.kb(q);
+      const float w = q < kSwSlots ? sSw[q] : __ldg(args.sw + (int64_t)sh.nb(q) * args.KB + kb);
       const bool got = mbar_wait(&tfull[buf], bphase, abort_flag, kSiteEpiTmemFull);
-      if (!__all_sync(0xffffffffu, got)) {
-        done = false;
-        break;
-      }
+      if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * NT + c0);
       const float4 *sc4;
-      if constexpr (kRes) {
-        const int slot = kb - kb_first + (kb < kb_first ? KB : 0);
-        sc4 = reinterpret_cast<const float4 *>(sXs + slot * NT + c0);
-      } else {
-        sc4 = reinterpret_cast<const float4 *>(sS + stage * C::kSSlot) + c0 / 4;
-      }
+      if constexpr (kRes) sc4 = reinterpret_cast<const float4 *>(sXs + (kb - sh.kb0) * NT + c0);
+      else sc4 = reinterpret_cast<const float4 *>(sS + stage * C::kSSlot) + c0 / 4;
       uint32_t v[C::kCW];
       if constexpr (C::kCW <= 16) {
         load_cols<C::kCW>(taddr, v);
@@ -396,77 +393,45 @@ __global__ void __launch_bounds__(kDThreads, 1)
         buf = 0;
         bphase ^= 1;
       }
-      // end of this weight block's run inside the share: flush it
-      if (kb == KB - 1 || p + 1 == p_end) {
-        const int64_t run0 = (p - kb > p_begin) ? p - kb : p_begin;  // first work item of the run
-        const bool whole = (run0 == p - kb) && kb == KB - 1;
-        const int n = nb * DBM + r;
-        if (whole) {
-          if (n < args.N) {
-#pragma unroll
-            for (int j = 0; j < C::kCW; ++j)
-              if (c0 + j < args.M) args.y[(int64_t)(c0 + j) * args.ldy + n] = bf16_bits(acc[j]);
-          }
-        } else {
-          // slot 0: the run holding the share's first item; slot 1: the last
-          // run.  The block is counted and reduced after the share's last item.
-          const int which = (run0 == p_begin) ? 0 : 1;
-          float *dst = args.part + ((int64_t)(blockIdx.x * 2 + which) * args.M) * DBM + r;
+      if (kb != sh.kb1 - 1) continue;
+      // ----------------------------------------------- end of this CTA's part of a block
+      const int n = sh.nb(q) * DBM + r;
+      bool fine = true;
+      if (S == 1) {
+        if (n < args.N) {
 #pragma unroll
           for (int j = 0; j < C::kCW; ++j)
-            if (c0 + j < args.M) dst[(int64_t)(c0 + j) * DBM] = acc[j];
-          cut_nb[ncut++] = nb;
+            if (c0 + j < args.M) args.y[(int64_t)(c0 + j) * args.ldy + n] = bf16_bits(acc[j]);
         }
+      } else if (rank > 0) {
+        // hand the partial to rank 0 through this CTA's shared memory (once
+        // rank 0 has read the previous block's)
+        fine = mbar_wait_cluster(red_free, rphase ^ 1, abort_flag, kSiteEpiTmemFull);
 #pragma unroll
-        for (int j = 0; j < C::kCW; ++j) acc[j] = 0.f;
-      }
-    }
-    // Count this CTA on each cut block it holds; the last CTA to arrive adds
-    // every sharing CTA's partial slot in CTA order.  (Hand-offs on bounded
-    // mbarriers, so an abort elsewhere in the CTA cannot leave a warp waiting.)
-    if (done && ncut > 0) {
-      __threadfence();  // this thread's partial slots are visible to the other CTAs
-      __syncwarp();
-      if (lane == 0) mbar_arrive(fl_in);
-      bool fine = true;
-      if (et == 0) {
-        fine = mbar_wait(fl_in, 0, abort_flag, kSiteEpiTmemFull);
-        for (int i = 0; i < ncut; ++i) {
-          int is_last = 0;
-          if (fine) {
-            const int64_t first = (int64_t)cut_nb[i] * KB;
-            const int64_t cf = share_of(first, args.W, args.G), cl = share_of(first + KB - 1, args.W, args.G);
-            const int prior = atomicAdd(args.cnt + cf, 1);
-            is_last = prior == (int)(cl - cf);
-            if (is_last) {
-              __threadfence();
-              args.cnt[cf] = 0;  // left zero for the next call (every arrival has been counted)
-            }
-          }
-          last_flag[i] = is_last;
-        }
-        mbar_arrive(fl_out);
-      }
-      fine = mbar_wait(fl_out, 0, abort_flag, kSiteEpiTmemFull) && fine;
-      if (__all_sync(0xffffffffu, fine)) {
-        for (int i = 0; i < ncut; ++i) {
-          if (!last_flag[i]) continue;
-          const int nb = cut_nb[i];
-          const int n = nb * DBM + r;
-          const int64_t first = (int64_t)nb * KB;
-          const int64_t cf = share_of(first, args.W, args.G), cl = share_of(first + KB - 1, args.W, args.G);
+        for (int j = 0; j < C::kCW; ++j) sPart[(c0 + j) * DBM + r] = acc[j];
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(red_full), 0));
+        rphase ^= 1;
+      } else {
+        // rank 0: the sum over the ranks, in rank order
+        fine = mbar_wait_cluster(red_full, rphase, abort_flag, kSiteEpiTmemFull);
+        rphase ^= 1;
+        if (__all_sync(0xffffffffu, fine)) {
           float sum[C::kCW];
 #pragma unroll
-          for (int j = 0; j < C::kCW; ++j) sum[j] = 0.f;
-          for (int64_t c = cf; c <= cl; ++c) {
-            const int wc = share_begin(c, args.W, args.G) >= first ? 0 : 1;
-            const float *src = args.part + ((c * 2 + wc) * args.M + c0) * DBM + r;
-            float v[C::kCW];  // one CTA's slot: independent loads, issued together
+          for (int j = 0; j < C::kCW; ++j) sum[j] = acc[j];
+          for (int pr = 1; pr < S; ++pr) {
+            const uint32_t src = mapa_shared(smem_addr(sPart + c0 * DBM + r), (uint32_t)pr);
+            float t[C::kCW];
 #pragma unroll
-            for (int j = 0; j < C::kCW; ++j) v[j] = (c0 + j < args.M) ? __ldcg(src + (int64_t)j * DBM) : 0.f;
+            for (int j = 0; j < C::kCW; ++j) t[j] = ld_shared_cluster_f32(src + (uint32_t)(j * DBM * 4));
 #pragma unroll
-            for (int j = 0; j < C::kCW; ++j) sum[j] += v[j];
+            for (int j = 0; j < C::kCW; ++j) sum[j] += t[j];
           }
+          __syncwarp();
+          if (lane == 0)  // every rank's partial has been read: its buffer may be reused
+            for (int pr = 1; pr < S; ++pr) mbar_arrive_cluster(mapa_shared(smem_addr(red_free), (uint32_t)pr));
           if (n < args.N) {
 #pragma unroll
             for (int j = 0; j < C::kCW; ++j)
@@ -474,7 +439,12 @@ __global__ void __launch_bounds__(kDThreads, 1)
           }
         }
       }
+      if (!__all_sync(0xffffffffu, fine)) break;
+#pragma unroll
+      for (int j = 0; j < C::kCW; ++j) acc[j] = 0.f;
     }
+    // a rank > 0 keeps its shared memory until rank 0 has read its last partial
+    if (S > 1 && rank > 0 && sh.nblk > 0) mbar_wait_cluster(red_free, rphase ^ 1, abort_flag, kSiteEpiTmemFull);
   }
 
   tc_fence_before();
@@ -483,6 +453,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
+  if (S > 1) cluster_sync();  // no CTA leaves while another may still address its shared memory
 }
 
 // Prologue: 1x128 quantization of X into the workspace.
@@ -495,10 +466,10 @@ __global__ void __launch_bounds__(256) decode_prologue_kernel(const uint16_t *__
 }
 
 struct Plan {
-  int NT, NB, KB, G;
-  bool res;     // activation quantized inside the GEMM kernel (one launch)
-  int64_t W, ldsa;
-  size_t off_q, off_sa, off_part, total;  // the counter area is [0, kCounterBytes)
+  int NT, NB, KB, S, C;   // S CTAs per cluster, C clusters
+  bool res;               // activation quantized inside the GEMM kernel (one launch)
+  int64_t ldsa;
+  size_t off_q, off_sa, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -509,27 +480,45 @@ int pick_nt(int64_t M) {
   return 64;
 }
 
+// The split S (CTAs per cluster, each a contiguous K range of every block of
+// its cluster) and the cluster count C that make the largest per-CTA item
+// count ceil(NB / C) * ceil(KB / S) smallest with C * S <= SMs; ties go to
+// the smaller S (fewer partials to add).
+void pick_split(int NB, int KB, int sms, int *S, int *C) {
+  int best = 0x7fffffff;
+  *S = 1;
+  *C = std::min(NB, sms);
+  for (int s = 1; s <= kMaxSplit && s <= KB; ++s) {
+    const int c = std::min(NB, sms / s);
+    if (c < 1) break;
+    const int items = ((NB + c - 1) / c) * ((KB + s - 1) / s);
+    if (items < best) {
+      best = items;
+      *S = s;
+      *C = c;
+    }
+  }
+}
+
 // vec: the activations allow 16-byte loads (x 16-byte aligned, ldx % 8 == 0).
 Plan make_plan(int64_t M, int64_t N, int64_t K, bool vec) {
   Plan p;
   p.NT = M <= kSwapMaxM ? pick_nt(M) : 0;  // 0: the prefill GEMM
   p.NB = (int)((N + 127) / 128);
   p.KB = (int)(K / 128);
-  p.W = (int64_t)p.NB * p.KB;
-  p.G = (int)std::min<int64_t>(std::min<int64_t>(p.W, num_sms()), kMaxShares);
-  const int64_t longest = (p.W + p.G - 1) / p.G;  // the largest share
-  p.res = p.NT == kResMaxM && vec && std::min<int64_t>(longest, p.KB) <= kMaxResKB;
+  pick_split(p.NB, p.KB, num_sms(), &p.S, &p.C);
+  const int nk = (p.KB + p.S - 1) / p.S;    // K-blocks per CTA (at most)
+  p.res = p.NT == kResMaxM && vec && nk <= kMaxResKB && nk * M <= kResMaxTiles;
   p.ldsa = (M + 3) / 4 * 4;
-  p.off_q = kCounterBytes;
-  p.off_sa = p.off_q + (p.res ? 0 : align256((size_t)(M * K)));
-  p.off_part = p.off_sa + (p.res ? 0 : align256((size_t)p.KB * p.ldsa * 4));
-  p.total = p.off_part + (p.NT ? align256((size_t)p.G * 2 * M * DBM * 4) : 0);
+  p.off_q = 0;
+  p.off_sa = align256((size_t)(M * K));
+  p.total = p.res ? 0 : p.off_sa + align256((size_t)p.KB * p.ldsa * 4);
   return p;
 }
 
 template <int NT, int QM>
 fp8bq_status launch_decode_nt(const CUtensorMap &tW, const CUtensorMap &tX, const CUtensorMap &tS,
-                              const DecodeArgs &a, cudaStream_t stream) {
+                              const DecodeArgs &a, int clusters, cudaStream_t stream) {
   static DeviceOnce once;  // one per instantiation
   const fp8bq_status ready = once.get([](int) {
     cudaFuncAttributes fa;
@@ -539,10 +528,46 @@ fp8bq_status launch_decode_nt(const CUtensorMap &tW, const CUtensorMap &tX, cons
     e = cudaFuncSetAttribute(decode_kernel<NT, QM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              DCfg<NT, QM>::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+    e = cudaFuncSetAttribute(decode_kernel<NT, QM>, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+    (void)e;
     return FP8BQ_OK;
   });
   if (ready != FP8BQ_OK) return ready;
-  decode_kernel<NT, QM><<<a.G, kDThreads, DCfg<NT, QM>::kSmemBytes, stream>>>(tW, tX, tS, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kDThreads);
+  cfg.dynamicSmemBytes = DCfg<NT, QM>::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)a.split;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.split > 1 ? 1 : 0;
+  if (a.split > 1) {
+    // no more clusters than can be resident at once (clusters live inside one
+    // GPC, so C * S <= SMs alone does not guarantee it): a second wave of
+    // clusters would double the time
+    static std::atomic<int> max_active[kMaxDevices][kMaxSplit + 1] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return FP8BQ_ERR_UNSUPPORTED;
+    int n = max_active[dev][a.split].load(std::memory_order_relaxed);
+    if (n == 0) {
+      cfg.gridDim = dim3((unsigned)(a.split * 256));
+      e = cudaOccupancyMaxActiveClusters(&n, decode_kernel<NT, QM>, &cfg);
+      if (e != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        return e != cudaSuccess ? cuda_fail(e, "cudaOccupancyMaxActiveClusters(decode)") : FP8BQ_ERR_UNSUPPORTED;
+      }
+      max_active[dev][a.split].store(n, std::memory_order_relaxed);
+    }
+    clusters = std::min(clusters, n);
+  }
+  cfg.gridDim = dim3((unsigned)(clusters * a.split));
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<NT, QM>, tW, tX, tS, a);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm_decode launch");
   return check_launch("gemm_decode");
 }
 
@@ -564,11 +589,11 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
   const bool vec = aligned(x, 16) && ldx % 8 == 0;  // K % 128 == 0 already
   const Plan p = make_plan(M, N, K, vec);
   // the documented size (the larger plan's), whichever path this call takes
-  if (ws == nullptr || ws_bytes < make_plan(M, N, K, false).total || !aligned(ws, 256)) return FP8BQ_ERR_WORKSPACE;
+  const size_t need = make_plan(M, N, K, false).total;
+  if (ws_bytes < need || (need > 0 && (ws == nullptr || !aligned(ws, 256)))) return FP8BQ_ERR_WORKSPACE;
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   uint8_t *q = wsb + p.off_q;
   float *sa = reinterpret_cast<float *>(wsb + p.off_sa);
-  float *part = reinterpret_cast<float *>(wsb + p.off_part);
   const uint16_t *xs = static_cast<const uint16_t *>(x);
 
   // 1. quantize X into the workspace, unless the GEMM kernel does it
@@ -592,7 +617,7 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
       return launch_gemm(q, K, sa, p.ldsa, qw, ldw, sw, y, ldy, M, N, K, mode, FP8BQ_GEMM_AUTO, stream);
   }
 
-  // 2. the GEMM, with the cut weight blocks reduced by their last CTA
+  // 2. the GEMM, K split over the CTAs of each cluster
   CUtensorMap tW, tX, tS;
   if (!make_tmap_2d(&tW, CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, (uint64_t)K, (uint64_t)N, (uint64_t)ldw, DBK, DBM,
                     CU_TENSOR_MAP_SWIZZLE_128B))
@@ -612,21 +637,18 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
   a.N = (int32_t)N;
   a.KB = p.KB;
   a.NB = p.NB;
-  a.W = p.W;
-  a.G = p.G;
-  a.part = part;
-  a.cnt = reinterpret_cast<int *>(wsb);
+  a.split = p.S;
   a.y = static_cast<uint16_t *>(y);
   a.ldy = ldy;
   a.x = xs;
   a.ldx = ldx;
   if (p.res)
-    return mode == FP8BQ_SCALE_FP32 ? launch_decode_nt<16, FP8BQ_SCALE_FP32>(tW, tX, tS, a, stream)
-                                    : launch_decode_nt<16, FP8BQ_SCALE_POW2>(tW, tX, tS, a, stream);
+    return mode == FP8BQ_SCALE_FP32 ? launch_decode_nt<16, FP8BQ_SCALE_FP32>(tW, tX, tS, a, p.C, stream)
+                                    : launch_decode_nt<16, FP8BQ_SCALE_POW2>(tW, tX, tS, a, p.C, stream);
   switch (p.NT) {
-    case 16: return launch_decode_nt<16, -1>(tW, tX, tS, a, stream);
-    case 32: return launch_decode_nt<32, -1>(tW, tX, tS, a, stream);
-    default: return launch_decode_nt<64, -1>(tW, tX, tS, a, stream);
+    case 16: return launch_decode_nt<16, -1>(tW, tX, tS, a, p.C, stream);
+    case 32: return launch_decode_nt<32, -1>(tW, tX, tS, a, p.C, stream);
+    default: return launch_decode_nt<64, -1>(tW, tX, tS, a, p.C, stream);
   }
 }
 

@@ -38,10 +38,6 @@ fp8bq_status scratch_for_current_device(void **out) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess || p == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
-    // the decode GEMM's arrival counters (the first 4 KB of any workspace)
-    // must start at zero; every call leaves them zero
-    e = cudaMemset(p, 0, 4096);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(decode scratch counters)");
     g_scratch_addr[dev] = p;
   }
   *out = g_scratch_addr[dev];

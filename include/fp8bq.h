@@ -225,15 +225,13 @@ FP8BQ_API fp8bq_status fp8bq_gemm_ex(const uint8_t *qa, int64_t lda, const float
  * breakthrough": FP8 in both generation and training).
  *   x     bf16 [M][ldx]; qw, sw as in fp8bq_gemm; y bf16 [M][ldy].
  *   ws    device workspace of at least fp8bq_gemm_decode_workspace_size(M, N, K)
- *         bytes, 256-byte aligned.  Its first 4096 bytes are arrival counters of
- *         the weight blocks that several CTAs share: they must be zero before
- *         the workspace's first use (e.g. cudaMemset once), and every call that
- *         completes leaves them zero again, so a workspace can be reused for any
- *         shape.  (After a call that reported FP8BQ_ERR_TIMEOUT, zero them
- *         again.)  The rest is scratch.  Calls that share a workspace must be
- *         stream-ordered.
- * One launch for M <= 16 (the activation is quantized inside the GEMM kernel
- * when x is 16-byte aligned with ldx % 8 == 0), two otherwise.
+ *         bytes, 256-byte aligned; its contents need not be initialized and are
+ *         overwritten.  Calls that share a workspace must be stream-ordered.
+ * One launch when M <= 16, x is 16-byte aligned with ldx % 8 == 0 and each CTA's
+ * share of K holds at most 256 of X's 1x128 tiles (the activation is then
+ * quantized inside the GEMM kernel); two launches otherwise.  K is split over
+ * the CTAs of thread-block clusters, whose partial sums are added over
+ * distributed shared memory in a fixed order (results are deterministic).
  * Requirements: as fp8bq_gemm, and M <= 256.  Output equals fp8bq_quant_act
  * followed by fp8bq_gemm up to FP32 summation order.
  */
@@ -255,13 +253,11 @@ FP8BQ_API fp8bq_status fp8bq_gemm_decode(const void *x, int64_t ldx,
  *   every GPU that loads it until the process exits; a shape whose workspace
  *   (fp8bq_gemm_decode_workspace_size) exceeds 32 MiB returns
  *   FP8BQ_ERR_WORKSPACE and launches nothing.  Nothing is allocated.
- *   The first call on a device looks up the array's device address and zeroes
- *   the array's counter area (CUDA runtime calls, synchronous); make that first
- *   call outside any stream capture.
+ *   The first call on a device looks up the array's device address (a CUDA
+ *   runtime call); make that first call outside any stream capture.
  *   All calls share the one array: calls that may run at the same time on the
  *   GPU (different streams, or different host threads) race on it and must be
- *   ordered by the caller.  The counter area is left zero by every call and
- *   the rest is rewritten before it is read.
+ *   ordered by the caller.  Each call rewrites the parts it reads.
  */
 FP8BQ_API fp8bq_status fp8bq_gemm_decode_noalloc(const void *x, int64_t ldx,
                                                  const uint8_t *qw, int64_t ldw, const float *sw,

@@ -105,23 +105,20 @@ def test_workspace_and_limits():
     assert e.value.status == 2
 
 
-def test_workspace_counters_left_zero_and_reused_across_shapes():
-    # one workspace for every shape: the arrival counters of the cut weight
-    # blocks (its first 4096 bytes) are zero after each call, and every call's
-    # rows match the oracle (the single-launch path at M <= 16, the two-launch
-    # one above, unaligned activations through the prologue)
+def test_one_workspace_reused_across_shapes():
+    # one workspace for every shape, its contents left from the previous call:
+    # the single-launch path (M <= 16), the two-launch one above it, and
+    # unaligned activations (through the prologue), every row against the oracle
     need = max(fq.gemm_decode_workspace_size(M, N, K) for N, K in wl.LLAMA8B_SHAPES.values() for M in (1, 16, 40))
-    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    ws = torch.full((need,), 0xAB, dtype=torch.uint8, device="cuda")
     for name, (N, K) in wl.LLAMA8B_SHAPES.items():
         qw, sw = qweights(name, fq.SCALE_FP32)
         for M in (1, 16, 40):
             x = wl.activations(M, K, seed=3 * M + K, device="cuda")
             check_decode(x, qw, sw, fq.SCALE_FP32, ws=ws)
-            assert not ws[:4096].any(), "counters left nonzero after %s M=%d" % (name, M)
         # a row view whose leading dimension is odd: not 16-byte loadable
         xb = wl.activations(4, K + 1, seed=K, device="cuda")[:, :K]
         check_decode(xb, qw, sw, fq.SCALE_FP32, ws=ws)
-        assert not ws[:4096].any()
 
 
 @pytest.mark.parametrize("M", [1, 5, 16])
