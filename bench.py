@@ -23,6 +23,7 @@ roofline fraction are the headline, not this ratio).
 """
 import argparse
 import hashlib
+import itertools
 import json
 import os
 import statistics
@@ -775,9 +776,12 @@ def run_case(args):
         x = wl.activations(M, K, seed=1, device=dev)
         w = wl.weights(N, K, seed=2, device=dev)
         qw, sw = fq.quant_weight(w, mode)
+        del w
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         ws = torch.zeros(max(256, fq.gemm_decode_workspace_size(M, N, K)), dtype=torch.uint8, device=dev)
-        fn = lambda: fq.gemm_decode(x, qw, sw, mode, out=y, ws=ws)  # noqa: E731
+        # successive calls read different copies of the weight (none finds it in L2)
+        qws = itertools.cycle([qw] + [qw.clone() for _ in range(rotations(N * K) - 1)])
+        fn = lambda: fq.gemm_decode(x, next(qws), sw, mode, out=y, ws=ws)  # noqa: E731
         work, unit = decode_bytes(M, N, K) / 1e9, "GB/s"
     elif kind == "moe":
         moe = wl.moe_layer(seed=0, device=dev)
