@@ -405,6 +405,11 @@ fp8bq_status fp8bq_gemm_wgrad(const uint8_t *qa, int64_t lda, const float *sa, i
     return FP8BQ_ERR_INVALID_ARG;
   if (ldsa < N || ldsa % 4 != 0 || !aligned(sa, 16)) return FP8BQ_ERR_INVALID_ARG;
   if (ldsb < K || ldsb % 4 != 0 || !aligned(sb, 16)) return FP8BQ_ERR_INVALID_ARG;
+  // power-of-two scales: the native block-scaled MMA applies both operands'
+  // scales (exact, no promotion); FP32 scales: FP32 promotion per token block
+  if (mode == FP8BQ_SCALE_POW2)
+    return launch_gemm_native_wgrad(qa, lda, sa, ldsa, qb, ldb, sb, ldsb, y, ldy, N, K, M,
+                                    static_cast<cudaStream_t>(stream));
   return launch_gemm_wgrad(qa, lda, sa, ldsa, qb, ldb, sb, ldsb, y, ldy, N, K, M, static_cast<cudaStream_t>(stream));
 }
 

@@ -65,8 +65,9 @@ static_assert(kAccCols + kStages * kSFCols <= kTmemCols, "TMEM budget");
 
 struct NativeArgs {
   const float *sa;
-  const float *sw;
+  const float *sw;    // ROWB: B row scales sw[kb * ldsw + n]; else 128x128 tile scales sw[nb * KB + kb]
   int64_t ldsa;
+  int64_t ldsw;
   int32_t M, N, KB, NB;
   int32_t num_m, num_n;
   int32_t band, n_major;  // tile order (raster_tile)
@@ -85,6 +86,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// ROWB: B's scales vary per B row (the weight-gradient GEMM, where B = X^T
+// is 1x128-quantized along the tokens); otherwise one scale per 128x128 tile.
+template <bool ROWB>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_native_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmY, const NativeArgs args) {
@@ -164,41 +168,65 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == 2) {
       // ---------------------------------------------------------------- scale factors
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      // The CTA's (tile, K-block) steps in order; each step's scales are
+      // loaded one step ahead, so their latency hides behind the wait for the
+      // stage.  Lane l writes A rows l + 32 c and B rows l + 32 c of both
+      // 128-row halves; an absent row's scale loads as 0 (UE8M0 byte 0).
+      constexpr int NBV = ROWB ? 8 : 2;
+      const int my_tiles = (int)blockIdx.x < total ? (total - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+      const int steps = my_tiles * KB;
+      auto load = [&](int s, float (&av)[4], float (&bv)[NBV]) {
+        const int t = (int)blockIdx.x + (s / KB) * (int)gridDim.x, kb = s % KB;
         int mb, nb;
         tile_mn(t, args, mb, nb);
-        const int wb0 = nb * 2, wb1 = nb * 2 + 1;
-        bool ok = true;
-        for (int kb = 0; kb < KB; ++kb) {
-          const bool got = mbar_wait(&empty[stage], phase ^ 1, abort_flag, kSiteProducerEmpty);
-          if (!__all_sync(0xffffffffu, got)) {
-            ok = false;
-            break;
-          }
-          uint4 a;
-          const float *sap = args.sa + (int64_t)kb * args.ldsa + mb * BM + lane;
-          const int m = mb * BM + lane;
-          a.x = (m < args.M) ? ue8m0x4(__ldg(sap)) : 0u;
-          a.y = (m + 32 < args.M) ? ue8m0x4(__ldg(sap + 32)) : 0u;
-          a.z = (m + 64 < args.M) ? ue8m0x4(__ldg(sap + 64)) : 0u;
-          a.w = (m + 96 < args.M) ? ue8m0x4(__ldg(sap + 96)) : 0u;
-          const uint32_t b0 = (wb0 < args.NB) ? ue8m0x4(__ldg(args.sw + (int64_t)wb0 * KB + kb)) : 0u;
-          const uint32_t b1 = (wb1 < args.NB) ? ue8m0x4(__ldg(args.sw + (int64_t)wb1 * KB + kb)) : 0u;
-          uint8_t *sf = sSF + stage * kSFBytes;
-          *reinterpret_cast<uint4 *>(sf + lane * 16) = a;
-          *reinterpret_cast<uint4 *>(sf + kSFABytes + lane * 16) = make_uint4(b0, b0, b0, b0);
-          *reinterpret_cast<uint4 *>(sf + kSFABytes + 512 + lane * 16) = make_uint4(b1, b1, b1, b1);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full[stage]);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
+        const float *sap = args.sa + (int64_t)kb * args.ldsa + mb * BM + lane;
+        const int m = mb * BM + lane;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) av[c] = m + 32 * c < args.M ? __ldg(sap + 32 * c) : 0.f;
+        if constexpr (ROWB) {
+          const float *sbp = args.sw + (int64_t)kb * args.ldsw;
+          const int n0 = nb * BN + lane;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) bv[c] = n0 + 32 * c < args.N ? __ldg(sbp + n0 + 32 * c) : 0.f;
+        } else {
+          const int wb0 = nb * 2, wb1 = nb * 2 + 1;
+          bv[0] = wb0 < args.NB ? __ldg(args.sw + (int64_t)wb0 * KB + kb) : 0.f;
+          bv[1] = wb1 < args.NB ? __ldg(args.sw + (int64_t)wb1 * KB + kb) : 0.f;
         }
-        if (!ok) break;
+      };
+      float a0[4], b0[NBV];
+      if (steps > 0) load(0, a0, b0);
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int s = 0; s < steps; ++s) {
+        float a1[4], b1[NBV];
+        if (s + 1 < steps) load(s + 1, a1, b1);
+        const bool got = mbar_wait(&empty[stage], phase ^ 1, abort_flag, kSiteProducerEmpty);
+        if (!__all_sync(0xffffffffu, got)) break;
+        uint8_t *sf = sSF + stage * kSFBytes;
+        *reinterpret_cast<uint4 *>(sf + lane * 16) =
+            make_uint4(ue8m0x4(a0[0]), ue8m0x4(a0[1]), ue8m0x4(a0[2]), ue8m0x4(a0[3]));
+        if constexpr (ROWB) {
+          *reinterpret_cast<uint4 *>(sf + kSFABytes + lane * 16) =
+              make_uint4(ue8m0x4(b0[0]), ue8m0x4(b0[1]), ue8m0x4(b0[2]), ue8m0x4(b0[3]));
+          *reinterpret_cast<uint4 *>(sf + kSFABytes + 512 + lane * 16) =
+              make_uint4(ue8m0x4(b0[4]), ue8m0x4(b0[5]), ue8m0x4(b0[6]), ue8m0x4(b0[7]));
+        } else {
+          const uint32_t w0 = ue8m0x4(b0[0]), w1 = ue8m0x4(b0[1]);
+          *reinterpret_cast<uint4 *>(sf + kSFABytes + lane * 16) = make_uint4(w0, w0, w0, w0);
+          *reinterpret_cast<uint4 *>(sf + kSFABytes + 512 + lane * 16) = make_uint4(w1, w1, w1, w1);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[stage]);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) a0[c] = a1[c];
+#pragma unroll
+        for (int c = 0; c < NBV; ++c) b0[c] = b1[c];
       }
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
@@ -307,7 +335,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-DeviceOnce g_native_once;
+template <bool ROWB>
+fp8bq_status native_ready() {
+  static DeviceOnce once;  // one per instantiation
+  return once.get([](int) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, gemm_native_kernel<ROWB>);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(gemm_native)");
+    if (fa.numRegs != kLaunchRegs) return FP8BQ_ERR_UNSUPPORTED;
+    e = cudaFuncSetAttribute(gemm_native_kernel<ROWB>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm_native)");
+    return FP8BQ_OK;
+  });
+}
 
 }  // namespace
 
@@ -324,20 +364,13 @@ fp8bq_status launch_gemm_native(const uint8_t *qa, int64_t lda, const float *sa,
       !make_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M, (uint64_t)ldy * 2, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_64B))
     return FP8BQ_ERR_INVALID_ARG;
-  const fp8bq_status ready = g_native_once.get([](int) {
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, gemm_native_kernel);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(gemm_native)");
-    if (fa.numRegs != kLaunchRegs) return FP8BQ_ERR_UNSUPPORTED;
-    e = cudaFuncSetAttribute(gemm_native_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm_native)");
-    return FP8BQ_OK;
-  });
+  const fp8bq_status ready = native_ready<false>();
   if (ready != FP8BQ_OK) return ready;
   NativeArgs a;
   a.sa = sa;
   a.sw = sw;
   a.ldsa = ldsa;
+  a.ldsw = 0;
   a.M = (int32_t)M;
   a.N = (int32_t)N;
   a.KB = (int32_t)(K / BK);
@@ -347,8 +380,42 @@ fp8bq_status launch_gemm_native(const uint8_t *qa, int64_t lda, const float *sa,
   choose_raster(M, N, K, BM, BN, &a.band, &a.n_major);
   const int64_t tiles = (int64_t)a.num_m * a.num_n;
   const int grid = (int)std::min<int64_t>(tiles, num_sms());
-  gemm_native_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tA, tB, tY, a);
+  gemm_native_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(tA, tB, tY, a);
   return check_launch("gemm_native");
+}
+
+// The weight-gradient GEMM with power-of-two scales on the native block-scaled
+// MMA: dW[N][K] = dY^T [N][M] . (X^T [K][M])^T, both operands' 1x128 scales
+// along the tokens (A: sa[mb * ldsa + n], B: sb[mb * ldsb + k]).
+fp8bq_status launch_gemm_native_wgrad(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa,
+                                      const uint8_t *qb, int64_t ldb, const float *sb, int64_t ldsb, void *y,
+                                      int64_t ldy, int64_t N, int64_t K, int64_t M, cudaStream_t stream) {
+  CUtensorMap tA, tB, tY;
+  if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qa, (uint64_t)M, (uint64_t)N, (uint64_t)lda, BK, BM,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qb, (uint64_t)M, (uint64_t)K, (uint64_t)ldb, BK, BN,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)K, (uint64_t)N, (uint64_t)ldy * 2, 32, 32,
+                    CU_TENSOR_MAP_SWIZZLE_64B))
+    return FP8BQ_ERR_INVALID_ARG;
+  const fp8bq_status ready = native_ready<true>();
+  if (ready != FP8BQ_OK) return ready;
+  NativeArgs a;
+  a.sa = sa;
+  a.sw = sb;
+  a.ldsa = ldsa;
+  a.ldsw = ldsb;
+  a.M = (int32_t)N;
+  a.N = (int32_t)K;
+  a.KB = (int32_t)(M / BK);
+  a.NB = (int32_t)((K + 127) / 128);
+  a.num_m = (int32_t)((N + BM - 1) / BM);
+  a.num_n = (int32_t)((K + BN - 1) / BN);
+  choose_raster(N, K, M, BM, BN, &a.band, &a.n_major);
+  const int64_t tiles = (int64_t)a.num_m * a.num_n;
+  const int grid = (int)std::min<int64_t>(tiles, num_sms());
+  gemm_native_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(tA, tB, tY, a);
+  return check_launch("gemm_native_wgrad");
 }
 
 }  // namespace fp8bq

@@ -180,6 +180,9 @@ fp8bq_status launch_quant_act_t(const void *x, int64_t M, int64_t K, int64_t ldx
                                 int64_t ldst, int mode, cudaStream_t stream);
 fp8bq_status launch_transpose_weight(const uint8_t *q, int64_t N, int64_t K, int64_t ldq, const float *sw,
                                      uint8_t *qt, int64_t ldqt, float *swt, cudaStream_t stream);
+fp8bq_status launch_gemm_native_wgrad(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa,
+                                      const uint8_t *qb, int64_t ldb, const float *sb, int64_t ldsb, void *y,
+                                      int64_t ldy, int64_t N, int64_t K, int64_t M, cudaStream_t stream);
 fp8bq_status launch_gemm_wgrad(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qb,
                                int64_t ldb, const float *sb, int64_t ldsb, void *y, int64_t ldy, int64_t N, int64_t K,
                                int64_t M, cudaStream_t stream);

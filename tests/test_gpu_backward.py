@@ -50,7 +50,8 @@ def _int_codes(rng, shape, vmax):
     return torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
 
 
-def test_wgrad_exact_integer_pow2_case_bit_exact():
+@pytest.mark.parametrize("mode", [fq.SCALE_FP32, fq.SCALE_POW2])   # FP32 promotion / native block-scaled MMA
+def test_wgrad_exact_integer_pow2_case_bit_exact(mode):
     rng = np.random.default_rng(4)
     N, K, M = 200, 264, 384                          # ragged tiles on both output axes
     qa = _int_codes(rng, (N, M), 4)
@@ -63,7 +64,7 @@ def test_wgrad_exact_integer_pow2_case_bit_exact():
     sa_d[:, :N] = torch.from_numpy(sa)
     sb_d = torch.zeros((MB, 264), dtype=torch.float32)
     sb_d[:, :K] = torch.from_numpy(sb)
-    y = fq.gemm_wgrad(torch.from_numpy(qa).cuda(), sa_d.cuda(), torch.from_numpy(qb).cuda(), sb_d.cuda(), M)
+    y = fq.gemm_wgrad(torch.from_numpy(qa).cuda(), sa_d.cuda(), torch.from_numpy(qb).cuda(), sb_d.cuda(), M, mode)
     torch.cuda.synchronize()
     assert np.array_equal(bf16_bits(y), ref)
 
@@ -82,22 +83,24 @@ def test_wgrad_within_tolerance(mode):
     assert_gemm_close(bf16_to_f64(y), oracle.gemm_wgrad(oa, osa, ob, osb), "wgrad")
 
 
+@pytest.mark.parametrize("mode", [fq.SCALE_FP32, fq.SCALE_POW2])
 @pytest.mark.parametrize("name", ["qkv", "down"])
-def test_wgrad_llama_full_size_sampled_rows(name):
+def test_wgrad_llama_full_size_sampled_rows(name, mode):
     """dW of a Llama-8B-shaped projection at M = 8192 tokens; the oracle
-    quantizes dY and X itself and computes one row of dW in every 128-row tile."""
+    quantizes dY and X itself and computes one row of dW in every 128-row tile
+    (power-of-two scales: the native block-scaled MMA path)."""
     N, K = wl.LLAMA8B_SHAPES[name]
     M = wl.PREFILL_TOKENS
     dy = wl.activations(M, N, seed=51, device="cuda")
     x = wl.activations(M, K, seed=52, device="cuda")
-    qa, sa = fq.quant_act_t(dy)
-    qb, sb = fq.quant_act_t(x)
-    y = fq.gemm_wgrad(qa, sa, qb, sb, M)
+    qa, sa = fq.quant_act_t(dy, mode)
+    qb, sb = fq.quant_act_t(x, mode)
+    y = fq.gemm_wgrad(qa, sa, qb, sb, M, mode)
     torch.cuda.synchronize()
     rng = np.random.default_rng(N)
     rows = np.array(sorted({0, N - 1} | {int(rng.integers(t, min(t + 128, N))) for t in range(0, N, 128)}))
-    oa, osa = oracle.quant_act_t(bf16_bits(dy[:, torch.from_numpy(rows).cuda()]), fq.SCALE_FP32)
-    ob, osb = oracle.quant_act_t(bf16_bits(x), fq.SCALE_FP32)
+    oa, osa = oracle.quant_act_t(bf16_bits(dy[:, torch.from_numpy(rows).cuda()]), mode)
+    ob, osb = oracle.quant_act_t(bf16_bits(x), mode)
     ref = oracle.gemm_wgrad(oa, osa, ob, osb)
     assert_gemm_close(bf16_to_f64(y[torch.from_numpy(rows).cuda()]), ref, "wgrad " + name)
 
