@@ -21,24 +21,26 @@
 //                   O~[n%2] = P' . V        P' (below) as A; V straight from the
 //                                           cache layout [token][d], i.e. read
 //                                           MN-major as the B operand
-//   softmax warps   thread = query row r (TMEM lane r):
+//   row warps       two threads per query row r (TMEM lane r), each with
+//                   half of every key block and half of the output columns:
 //                   s_j  = S_rj * ks_j      (the key's scale)
 //                   m    = running max of c s_j, c = scale * log2(e) * qs_r
 //                   p_j  = 2^(c s_j - m)    (0 for masked keys)
 //                   l    = 2^(m_old - m) l + sum_j p_j
 //                   P'_rj = E4M3(p_j * 256 vs_j / vmax)   with vmax the block's
 //                          largest value scale: P' lies in [0, 256]
-//   correction warps
-//                   O_r = 2^(m_old - m) O_r + (vmax / 256) O~_r    (FP32 registers)
-//                   and after the last block bf16(O_r / l).
+//   and, one block later, O_r = 2^(m_old - m) O_r + (vmax / 256) O~_r
+//                   (FP32 registers), after the last block bf16(O_r / l).
 // The weights p_j enter the value product rounded to E4M3 (relative error at
 // most 2^-4 each, as for any FP8 operand); the row sum l uses the unrounded
 // p_j.  Everything else is FP32.
 //
 // Roles (384 threads): warp 0 issues the TMA loads of Q, K and V; warp 1 owns
 // TMEM and issues the MMAs; warps 2 and 3 load the key and value scales of
-// alternate blocks and form 256 vs_j / vmax; warps 4-7 run the softmax,
-// warps 8-11 the correction and output.
+// alternate blocks and form 256 vs_j / vmax; warps 4-11 (two per scheduler,
+// so one's latency hides behind the other's work) run the softmax, the
+// output correction and the output, the two halves of a row exchanging their
+// maxima per block and their sums per unit through shared memory.
 // Waits are bounded (a second); on expiry the kernel records the site in the
 // device error word and every role stops.
 #include <cuda_bf16.h>
@@ -66,10 +68,12 @@ constexpr int kLowRegs = 56;
 constexpr int kHighRegs = 224;
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int kTmemCols = 512;           // S[2] at 0, 128; O~[2] at 256, 384
-constexpr int kNumBars = 2 * kStages + 5 * 2 * 2 + 1;  // kv ring, five full/empty pairs of two, drain
+// kv ring, four full/empty pairs of two (q, s, p, o), the row maxima's
+// exchange (two), the row sums' exchange, drain
+constexpr int kNumBars = 2 * kStages + 4 * 2 * 2 + 2 + 1 + 1;
 constexpr int kSmemBytes = 1024 + 2 * kTile /* Q */ + 2 * kStages * kTile /* K, V */ + 2 * kTile /* P' */ +
-                           kStages * kScaleSlot + 2 * kBQ * 8 /* (alpha, l) */ + 16 /* block factors */ +
-                           kNumBars * 8 + 16;
+                           kStages * kScaleSlot + 2 * 2 * kBQ * 4 /* half-row maxima */ +
+                           2 * kBQ * 4 /* half-row sums */ + kNumBars * 8 + 16;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 enum AttnWaitSite : unsigned {
@@ -174,46 +178,14 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x for x <= 0 on the FMA and integer pipes instead of the special-function
-// unit (which is the softmax's bottleneck when it computes every
-// exponential): x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the
-// low bits of the sum) and f in [-1/2, 1/2]; 2^f by a cubic fitted to it
-// (maximum relative error 1.0e-4, evaluated by Horner's rule in FP32); 2^n
-// enters by adding n to the exponent field.  x is clamped to -125, below
-// which the weight is far under the E4M3 weights' smallest step anyway.
-__device__ __forceinline__ float ex2_poly(float x) {
-  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
-  x = fmaxf(x, -125.f);
-  const float j = __fadd_rn(x, kShift);
-  const float f = __fsub_rn(x, __fsub_rn(j, kShift));
-  float p = __fmaf_rn(0.05500892922282219f, f, 0.24221095442771912f);
-  p = __fmaf_rn(p, f, 0.6932829022407532f);
-  p = __fmaf_rn(p, f, 1.f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(j) << 23));
-}
-
-// E4M3 code (round to nearest even) of w in [0, 448] on the integer and FMA
-// pipes instead of the conversion unit.  Normal range (w >= 2^-6): round the
-// binary32 pattern to 3 fraction bits (add 0x7FFFF plus the lowest kept bit),
-// then rebias the exponent from 127 to 7.  Below 2^-6 (E4M3 subnormals, steps
-// of 2^-9): adding 1.5 * 2^14 rounds w to a multiple of 2^-9 whose count is
-// left in the low bits of the sum (count 8 is 2^-6, the smallest normal code).
-// Checked against the conversion's definition on every binary32 value in
-// [0, 448].
-__device__ __forceinline__ uint32_t e4m3_nonneg(float w) {
-  const uint32_t u = __float_as_uint(w);
-  const uint32_t normal = ((u + 0x7FFFFu + ((u >> 20) & 1u)) >> 20) - (120u << 3);
-  const uint32_t sub = __float_as_uint(__fadd_rn(w, 24576.f)) - 0x46C00000u;
-  return w < 0.015625f ? sub : normal;
-}
-
 struct Bars {
   uint64_t *kv_full, *kv_empty;   // [kStages]
   uint64_t *q_full, *q_empty;     // [2]
   uint64_t *s_full, *s_empty;     // [2]
   uint64_t *p_full, *p_empty;     // [2]
   uint64_t *o_full, *o_empty;     // [2]
-  uint64_t *st_full, *st_empty;   // [2]
+  uint64_t *xbar;                 // [2] the row warps' half-row maxima of block n are in sMx[n % 2]
+  uint64_t *lbar;                 // the row warps' half-row sums of the unit are in sL
   uint64_t *drain;
 };
 
@@ -227,9 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sV = sK + kStages * kTile;       // [kStages]
   uint8_t *sP = sV + kStages * kTile;       // [2]
   uint8_t *sScale = sP + 2 * kTile;         // [kStages][kScaleSlot]
-  float2 *sStat = reinterpret_cast<float2 *>(sScale + kStages * kScaleSlot);  // [2][128] (alpha, l)
-  float *sFac = reinterpret_cast<float *>(sStat + 2 * kBQ);                  // [2] vmax / 256
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sFac + 4);
+  float *sMx = reinterpret_cast<float *>(sScale + kStages * kScaleSlot);  // [2 blocks][2 halves][128 rows]
+  float *sL = sMx + 2 * 2 * kBQ;                                          // [2 halves][128 rows]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sL + 2 * kBQ);
   Bars B;
   B.kv_full = bar;
   B.kv_empty = bar + kStages;
@@ -241,9 +213,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   B.p_empty = B.p_full + 2;
   B.o_full = B.p_empty + 2;
   B.o_empty = B.o_full + 2;
-  B.st_full = B.o_empty + 2;
-  B.st_empty = B.st_full + 2;
-  B.drain = B.st_empty + 2;
+  B.xbar = B.o_empty + 2;
+  B.lbar = B.xbar + 2;
+  B.drain = B.lbar + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(B.drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -253,20 +225,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&B.kv_full[s], 2);      // the TMA arm (with its bytes) + the scale writers
-      mbar_init(&B.kv_empty[s], 1 + 4); // the value MMA's commit + the four softmax warps
+      mbar_init(&B.kv_empty[s], 1 + 8); // the value MMA's commit + the eight row warps
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&B.q_full[i], 1);
       mbar_init(&B.q_empty[i], 1);
       mbar_init(&B.s_full[i], 1);
-      mbar_init(&B.s_empty[i], 4);
-      mbar_init(&B.p_full[i], 4);
+      mbar_init(&B.s_empty[i], 8);
+      mbar_init(&B.p_full[i], 8);
       mbar_init(&B.p_empty[i], 1);
       mbar_init(&B.o_full[i], 1);
-      mbar_init(&B.o_empty[i], 4);
-      mbar_init(&B.st_full[i], 4);
-      mbar_init(&B.st_empty[i], 4);
+      mbar_init(&B.o_empty[i], 8);
+      mbar_init(&B.xbar[i], 8);
     }
+    mbar_init(B.lbar, 8);
     mbar_init(B.drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -439,20 +411,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(B.drain, 0, nullptr, kSiteDrain);
       }
     }
-  } else if (warp < 8) {
+  } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
-    // -------------------------------------------------------------------- softmax
+    // -------------------------------------------------------------------- rows: softmax, correction, output
+    // Query row r (TMEM lane r) is shared by two threads of the same lane
+    // quarter: hf = 0 (warps 4-7) takes keys 0-63 of every block and output
+    // columns 0-63, hf = 1 (warps 8-11) keys 64-127 and columns 64-127.  They
+    // exchange their partial row maxima once per block and their partial row
+    // sums once per unit through shared memory.  The value product of block n
+    // is folded into the output while block n + 1's softmax is done.
     const int quarter = warp & 3;
+    const int hf = (warp - 4) >> 2;
     const int r = quarter * 32 + lane;  // query row within the unit = TMEM lane
-    uint32_t n = 0;
+    const int jo = 64 * hf;             // this thread's first key of a block and first output column
+    const uint32_t lane_base = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    uint32_t n = 0, lph = 0;
     bool ok = true;
+    // the eight row warps meet at `bar` (bounded wait)
+    auto meet = [&](uint64_t *bar, uint32_t parity) -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kSiteAttnStat));
+    };
+    float2 acc[32];  // output columns jo .. jo + 63, in pairs
+    // O = al O + fa O~[nn % 2] (the value product of the CTA's block nn)
+    auto correct = [&](uint32_t nn, float al, float fa) -> bool {
+      const int ob = nn & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&B.o_full[ob], (nn >> 1) & 1, abort_flag, kSiteAttnO))) return false;
+      tc_fence_after();
+      uint32_t pr[64];
+      const uint32_t taddr = lane_base + 256u + 128u * (uint32_t)ob + (uint32_t)jo;
+      tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
+      tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_relaxed(&B.o_empty[ob]);
+      const float2 al2 = make_float2(al, al), f2 = make_float2(fa, fa);
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        acc[k] = __ffma2_rn(make_float2(__uint_as_float(pr[2 * k]), __uint_as_float(pr[2 * k + 1])), f2,
+                            __fmul2_rn(acc[k], al2));
+      return true;
+    };
     for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
       const Unit x = unit_at(u, args);
-      if (x.nblk == 0) continue;
       const int i = kBQ * x.t + r;
+      uint4 *dst = reinterpret_cast<uint4 *>(args.o + (((int64_t)x.b * args.S + i) * args.Hq + x.h) * kD + jo);
+      if (x.nblk == 0) {  // the whole tile is at or past the sequence's length: zeros
+        if (i < args.S)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) dst[k] = make_uint4(0, 0, 0, 0);
+        continue;
+      }
       const float qsc = i < args.S ? __ldg(args.qs + ((int64_t)x.b * args.S + i) * args.Hq + x.h) : 0.f;
       const float c = args.c0 * qsc;
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f, al_prev = 0.f, fa_prev = 0.f;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) acc[k] = make_float2(0.f, 0.f);
       for (int kb = 0; kb < x.nblk; ++kb, ++n) {
         const int st = n % kStages;
         const int sb = n & 1;
@@ -463,12 +479,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        uint32_t sr[128];
-        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + 128u * (uint32_t)sb;
+        uint32_t sr[64];
+        const uint32_t taddr = lane_base + 128u * (uint32_t)sb + (uint32_t)jo;
         tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_ld_32x32b_x32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-        tmem_ld_32x32b_x32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
@@ -479,16 +493,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const float *slot = reinterpret_cast<const float *>(sScale + st * kScaleSlot);
-        const float4 *ks4 = reinterpret_cast<const float4 *>(slot);
-        const float4 *rv4 = reinterpret_cast<const float4 *>(slot + kBK);
-        // s_j = S_rj * ks_j and the block's row max over the visible keys.
-        // Masking is by selects (no branches); four partial maxima and four
-        // partial sums keep the dependency chains short, since one warp per
-        // scheduler runs this loop.
-        const int vis = kb == x.t ? r : kBK - 1;  // last visible key of the block
+        const float4 *ks4 = reinterpret_cast<const float4 *>(slot + jo);
+        const float4 *rv4 = reinterpret_cast<const float4 *>(slot + kBK + jo);
+        const float fa = slot[2 * kBK];
+        // s_j = S_rj * ks_j and this half's row max over the visible keys
+        // (masking by selects; four partial maxima and sums keep the
+        // dependency chains short)
+        const int vis = kb == x.t ? r - jo : 63;  // last visible key of this half (< 0: none)
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int j4 = 0; j4 < kBK / 4; ++j4) {
+        for (int j4 = 0; j4 < 16; ++j4) {
           const float4 k4 = ks4[j4];
           float sv[4] = {__uint_as_float(sr[4 * j4 + 0]) * k4.x, __uint_as_float(sr[4 * j4 + 1]) * k4.y,
                          __uint_as_float(sr[4 * j4 + 2]) * k4.z, __uint_as_float(sr[4 * j4 + 3]) * k4.w};
@@ -499,14 +513,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             mx4[e] = fmaxf(mx4[e], sv[e]);
           }
         }
-        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        sMx[(sb * 2 + hf) * kBQ + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        if (!meet(&B.xbar[sb], sph)) {
+          ok = false;
+          break;
+        }
+        const float mx = fmaxf(sMx[(sb * 2) * kBQ + r], sMx[(sb * 2 + 1) * kBQ + r]);
         // c > 0, so the max of c s is c times the max of s
         const float m_new = fmaxf(m, c * mx);
         const float alpha = ex2(m - m_new);  // 0 on the first block (m = -inf)
         float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[32];  // 128 E4M3 codes, 4 per word
+        uint32_t pk[16];  // 64 E4M3 codes, 4 per word
 #pragma unroll
-        for (int j4 = 0; j4 < kBK / 4; ++j4) {
+        for (int j4 = 0; j4 < 16; ++j4) {
           const float4 w4 = rv4[j4];
           float p[4];
 #pragma unroll
@@ -518,10 +537,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t hi = qdev::e4m3x2(p[2] * w4.z, p[3] * w4.w);
           pk[j4] = lo | (hi << 16);
         }
-        const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-        l = alpha * l + sum;
+        l = alpha * l + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
         m = m_new;
-        // P' row r into the 128-byte-swizzled K-major tile (the A operand)
+        // this half of P' row r into the 128-byte-swizzled K-major tile
         got = mbar_wait(&B.p_empty[sb], sph ^ 1, abort_flag, kSiteAttnP);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
@@ -529,87 +547,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t *prow = sP + sb * kTile + r * 128;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
+        for (int cc = 0; cc < 4; ++cc) {
+          const int ch = 4 * hf + cc;
           *reinterpret_cast<uint4 *>(prow + ((ch ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+              make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+        }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B.p_full[sb]);
-        // the row's rescale factor and running sum, and the block's value factor
-        got = mbar_wait(&B.st_empty[sb], sph ^ 1, abort_flag, kSiteAttnStat);
-        if (!__all_sync(0xffffffffu, got)) {
-          ok = false;
-          break;
-        }
-        sStat[sb * kBQ + r] = make_float2(alpha, l);
-        if (r == 0) sFac[sb] = slot[2 * kBK];
-        __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&B.st_full[sb]);
+          mbar_arrive(&B.p_full[sb]);
           mbar_arrive(&B.kv_empty[st]);  // this warp has read the stage's scales
         }
-      }
-    }
-  } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
-    // -------------------------------------------------------------------- correction + output
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    uint32_t n = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
-      const Unit x = unit_at(u, args);
-      const int i = kBQ * x.t + r;
-      float2 acc[kD / 2];
-#pragma unroll
-      for (int k = 0; k < kD / 2; ++k) acc[k] = make_float2(0.f, 0.f);
-      float l = 0.f;
-      for (int kb = 0; kb < x.nblk; ++kb, ++n) {
-        const int sb = n & 1;
-        const uint32_t sph = (n >> 1) & 1;
-        bool got = mbar_wait(&B.st_full[sb], sph, abort_flag, kSiteAttnStat);
-        if (!__all_sync(0xffffffffu, got)) {
+        // the previous block's value product, while the MMA runs this one's
+        if (kb > 0 && !correct(n - 1, al_prev, fa_prev)) {
           ok = false;
           break;
         }
-        const float2 st2 = sStat[sb * kBQ + r];
-        const float fac = sFac[sb];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B.st_empty[sb]);
-        l = st2.y;
-        const float2 al2 = make_float2(st2.x, st2.x), f2 = make_float2(fac, fac);
-        got = mbar_wait(&B.o_full[sb], sph, abort_flag, kSiteAttnO);
-        if (!__all_sync(0xffffffffu, got)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + 256u + 128u * (uint32_t)sb;
-#pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
-          uint32_t pr[64];
-          tmem_ld_32x32b_x32(taddr + 64 * hc, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
-          tmem_ld_32x32b_x32(taddr + 64 * hc + 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
-          tmem_ld_wait();
-          if (hc == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_relaxed(&B.o_empty[sb]);
-          }
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            acc[32 * hc + k] = __ffma2_rn(make_float2(__uint_as_float(pr[2 * k]), __uint_as_float(pr[2 * k + 1])), f2,
-                                          __fmul2_rn(acc[32 * hc + k], al2));
-        }
+        al_prev = alpha;
+        fa_prev = fa;
       }
-      if (!ok) break;
+      if (!ok || !correct(n - 1, al_prev, fa_prev)) break;  // the unit's last block
+      // the row sum: this half's plus the other's (in half order)
+      sL[hf * kBQ + r] = l;
+      if (!meet(B.lbar, lph)) break;
+      lph ^= 1;
+      const float lt = sL[r] + sL[kBQ + r];
       if (i < args.S) {
         // rows at or past the sequence's length are 0
-        const bool live = i < x.L && x.nblk > 0;
-        const float inv = live ? __fdiv_rn(1.f, l) : 0.f;
-        uint4 *dst = reinterpret_cast<uint4 *>(args.o + (((int64_t)x.b * args.S + i) * args.Hq + x.h) * kD);
+        const bool live = i < x.L;
+        const float inv = live ? __fdiv_rn(1.f, lt) : 0.f;
 #pragma unroll
-        for (int k = 0; k < kD / 8; ++k) {
+        for (int k = 0; k < 8; ++k) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
