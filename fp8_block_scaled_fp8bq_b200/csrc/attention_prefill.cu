@@ -48,6 +48,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "device.cuh"
 #include "internal.h"
@@ -499,20 +500,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         // s_j = S_rj * ks_j and this half's row max over the visible keys
         // (masking by selects; four partial maxima and sums keep the
         // dependency chains short)
-        const int vis = kb == x.t ? r - jo : 63;  // last visible key of this half (< 0: none)
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        auto scale_max = [&](auto masked, int vis) {  // vis: last visible key of this half (< 0: none)
 #pragma unroll
-        for (int j4 = 0; j4 < 16; ++j4) {
-          const float4 k4 = ks4[j4];
-          float sv[4] = {__uint_as_float(sr[4 * j4 + 0]) * k4.x, __uint_as_float(sr[4 * j4 + 1]) * k4.y,
-                         __uint_as_float(sr[4 * j4 + 2]) * k4.z, __uint_as_float(sr[4 * j4 + 3]) * k4.w};
+          for (int j4 = 0; j4 < 16; ++j4) {
+            const float4 k4 = ks4[j4];
+            float sv[4] = {__uint_as_float(sr[4 * j4 + 0]) * k4.x, __uint_as_float(sr[4 * j4 + 1]) * k4.y,
+                           __uint_as_float(sr[4 * j4 + 2]) * k4.z, __uint_as_float(sr[4 * j4 + 3]) * k4.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            sv[e] = 4 * j4 + e <= vis ? sv[e] : -INFINITY;
-            sr[4 * j4 + e] = __float_as_uint(sv[e]);
-            mx4[e] = fmaxf(mx4[e], sv[e]);
+            for (int e = 0; e < 4; ++e) {
+              if constexpr (decltype(masked)::value) sv[e] = 4 * j4 + e <= vis ? sv[e] : -INFINITY;
+              sr[4 * j4 + e] = __float_as_uint(sv[e]);
+              mx4[e] = fmaxf(mx4[e], sv[e]);
+            }
           }
-        }
+        };
+        // only the diagonal block (the unit's last) has keys after the row
+        if (kb == x.t) scale_max(std::true_type(), r - jo);
+        else scale_max(std::false_type(), 63);
         sMx[(sb * 2 + hf) * kBQ + r] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
         if (!meet(&B.xbar[sb], sph)) {
           ok = false;
