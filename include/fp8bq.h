@@ -383,9 +383,12 @@ FP8BQ_API fp8bq_status fp8bq_transpose_weight(const uint8_t *q, int64_t N, int64
                                               uint8_t *qt, int64_t ldqt, float *swt, void *stream);
 
 /*
- * Weight-gradient GEMM: y[n][k] = sum_m deq(qa)[n][m] deq(qb)[k][m], bf16 out,
- * FP32 promotion per 128-token block with the scale product sa * sb formed
- * per output element.
+ * Weight-gradient GEMM: y[n][k] = sum_m deq(qa)[n][m] deq(qb)[k][m], bf16 out.
+ * FP8BQ_SCALE_FP32: FP32 promotion per 128-token block with the scale product
+ * sa * sb formed per output element.  FP8BQ_SCALE_POW2 (every scale a power of
+ * two, as fp8bq_quant_act_t writes them in that mode): the tensor cores'
+ * block-scaled MMA applies both scales exactly (UE8M0 scale factors per row
+ * of each operand), with no promotion step.
  *   qa, sa  codes of dY^T [N][lda] and scales [M/128][ldsa] (fp8bq_quant_act_t of dY)
  *   qb, sb  codes of X^T [K][ldb] and scales [M/128][ldsb] (fp8bq_quant_act_t of X)
  *   y       bf16 dW [N][ldy]
