@@ -55,7 +55,14 @@ constexpr int kDHighRegs = 224;
 static_assert(128 * kDLowRegs + 256 * kDHighRegs <= kDThreads * kDLaunchRegs, "register split");
 constexpr int kMaxDecodeM = 256;
 constexpr int kSwapMaxM = 64;
+// The prefill GEMM (128-token x 256-weight-row tiles) instead of this kernel:
+// for M > 32 when N fills at least kGemmMinNTiles of its 256-row tiles, and
+// for any M when it fills kGemmAnyMNTiles.  Measured: this kernel's small
+// MMAs (128 weight rows x NT tokens x 32) cost about as much as the GEMM's
+// 128 x 256 x 32 ones, so per weight byte the GEMM issues half the MMA work
+// and streams the weight faster wherever it has enough tiles to fill the SMs.
 constexpr int kGemmMinNTiles = 24;
+constexpr int kGemmAnyMNTiles = 64;
 constexpr int kResMaxM = 16;        // activation quantized inside the GEMM kernel up to this M ...
 constexpr int kResMaxTiles = 256;   // ... when a CTA's K range holds at most this many 1x128 tiles of X
 constexpr int kMaxSplit = 8;        // CTAs of a cluster (split of K)
@@ -743,10 +750,9 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, bool vec, const DecodeDevice &dd
   p.S = p.C = 1;
   p.res = false;
   p.nres = p.nst = p.smem = 0;
-  // 0: the prefill GEMM, for M > 64, and for M > 32 when N fills at least
-  // kGemmMinNTiles of its 256-column tiles (measured faster there: its
-  // promotion runs once per 128 x 256 tile rather than per token column)
-  p.NT = M <= kSwapMaxM && (M <= 32 || (N + 255) / 256 < kGemmMinNTiles) ? pick_nt(M) : 0;
+  // 0: the prefill GEMM (M > 64, or enough 256-row tiles of N: see above)
+  const int64_t ntiles = (N + 255) / 256;
+  p.NT = M <= kSwapMaxM && ntiles < kGemmAnyMNTiles && (M <= 32 || ntiles < kGemmMinNTiles) ? pick_nt(M) : 0;
   p.NB = (int)((N + 127) / 128);
   p.KB = (int)(K / 128);
   workspace_layout(M, K, &p);
