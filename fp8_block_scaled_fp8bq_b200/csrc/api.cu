@@ -236,7 +236,7 @@ fp8bq_status fp8bq_get_device_error(uint64_t *code) {
   cudaError_t (*takers[])(unsigned long long *) = {take_device_error_gemm, take_device_error_decode,
                                                     take_device_error_native, take_device_error_pair,
                                                     take_device_error_swiglu, take_device_error_wgrad,
-                                                    take_device_error_prefill_attn};
+                                                    take_device_error_prefill_attn, take_device_error_decode_wide};
   for (auto take : takers) {
     e = take(&w);
     if (e != cudaSuccess) return cuda_fail(e, "read device error word");

@@ -1,6 +1,9 @@
 // Decode-shaped (small M, memory-bound) block-scaled FP8 linear for sm_100a:
 // Y[M,N] = q(X)[M,K] . W[N,K]^T with the activation quantized on the fly
-// (1x128 tiles) and W pre-quantized (128x128 tiles).
+// (1x128 tiles) and W pre-quantized (128x128 tiles).  This file holds the
+// call's routing (the wide form of decode_wide.cu up to M = 64 by default,
+// the prefill GEMM above), the prologue quantization kernel and the narrow
+// form below, which FP8BQ_DECODE_KERNEL=narrow selects.
 //
 // Method: "NVIDIA NeMo RL Achieves 48% Speedup With End-to-End FP8 Precision
 // Training", section "Technical breakthrough": FP8 is applied in generation as
@@ -8,8 +11,8 @@
 // 128x128).  In generation the linear layers see a handful of tokens, so the
 // time goes into streaming the weight from HBM.
 //
-// The GEMM runs with the operands swapped so that the tensor cores do useful
-// work at small M: the weight is the 128-row MMA operand and the tokens are
+// The narrow form runs with the operands swapped so that the tensor cores do
+// useful work at small M: the weight is the 128-row MMA operand and the tokens are
 // the MMA's N dimension (NT = M rounded up to 16, 32 or 64).  A work item is a
 // (128-row weight block nb, 128-deep K-block kb) pair: the weight tile (16 KB)
 // comes through a TMA stage ring; 4 x tcgen05.mma 128xNTx32 go into one of
@@ -36,6 +39,7 @@
 //     or the prologue is followed by the prefill GEMM (M > 64, where the
 //     per-token promotion costs more than the weight stream).
 #include <cuda_bf16.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -55,14 +59,10 @@ constexpr int kDHighRegs = 224;
 static_assert(128 * kDLowRegs + 256 * kDHighRegs <= kDThreads * kDLaunchRegs, "register split");
 constexpr int kMaxDecodeM = 256;
 constexpr int kSwapMaxM = 64;
-// The prefill GEMM (128-token x 256-weight-row tiles) instead of this kernel:
-// for M > 32 when N fills at least kGemmMinNTiles of its 256-row tiles, and
-// for any M when it fills kGemmAnyMNTiles.  Measured: this kernel's small
-// MMAs (128 weight rows x NT tokens x 32) cost about as much as the GEMM's
-// 128 x 256 x 32 ones, so per weight byte the GEMM issues half the MMA work
-// and streams the weight faster wherever it has enough tiles to fill the SMs.
-constexpr int kGemmMinNTiles = 24;
-constexpr int kGemmAnyMNTiles = 64;
+// The prefill GEMM (128-token x 256-weight-row tiles) instead of the wide
+// form for M > 32 when the weight has at least this many 256-row tiles: it
+// fills the SMs without a split and its promotion runs on 128 token lanes.
+constexpr int kGemmMinNTiles = 64;
 constexpr int kResMaxM = 16;        // activation quantized inside the GEMM kernel up to this M ...
 constexpr int kResMaxTiles = 256;   // ... when a CTA's K range holds at most this many 1x128 tiles of X
 constexpr int kMaxSplit = 8;        // CTAs of a cluster (split of K)
@@ -164,33 +164,6 @@ __device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t *r) {
   } else {
     tmem_ld_32x32b_x16(taddr, r);
   }
-}
-
-// One 1x128 tile of the activation (row m, K-block kb) quantized by a group of
-// four lanes into a resident shared-memory tile of NT = 16 rows x 128 bytes in
-// the MMA operand's 128-byte-swizzled layout (16-byte chunk c of row m at
-// chunk position c ^ (m & 7)); lane qd of the group owns chunks qd, qd + 4,
-// qd + 8, qd + 12 of the row, as fp8bq_quant_act's vector kernel does.
-// Every lane of the warp calls it (the amax shuffles span the warp); lanes
-// with have == false store nothing.  v: the lane's four 16-byte pieces of the
-// row (pieces qd, qd + 4, qd + 8, qd + 12), loaded by the caller.
-template <int MODE>
-__device__ __forceinline__ void quant_row_tile_to_smem(bool have, const uint4 (&v)[4], int qd, uint8_t *tile, int m,
-                                                       float *scale) {
-  uint32_t am = max(max(qdev::absmax_bits8(v[0]), qdev::absmax_bits8(v[1])),
-                    max(qdev::absmax_bits8(v[2]), qdev::absmax_bits8(v[3])));
-  am = max(am, __shfl_xor_sync(0xffffffffu, am, 1));
-  am = max(am, __shfl_xor_sync(0xffffffffu, am, 2));
-  if (!have) return;
-  const qdev::TileScale ts = qdev::tile_scale<MODE>(qdev::bits_to_amax(am));
-  uint8_t *row = tile + m * 128;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int e8 = j * 4 + qd;  // 8-element piece of the row
-    const uint2 c = qdev::fast_tile<MODE>(ts) ? qdev::encode8<MODE, true>(v[j], ts) : qdev::encode8<MODE>(v[j], ts);
-    *reinterpret_cast<uint2 *>(row + (((e8 >> 1) ^ (m & 7)) << 4) + (e8 & 1) * 8) = c;
-  }
-  if (qd == 0) *scale = ts.s;
 }
 
 template <int NT, int QM>
@@ -437,7 +410,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
           const int t = c0 + 64 * u + grp;
           const bool have = t < ntile;
           const int i = have ? t / args.M : 0, m = have ? t - (t / args.M) * args.M : 0;
-          quant_row_tile_to_smem<QM < 0 ? 0 : QM>(have, v[u], qd, sXr + i * (NT * DBK), m, sXs + i * NT + m);
+          qdev::quant_row_tile_to_smem<QM < 0 ? 0 : QM>(have, v[u], qd, sXr + i * (NT * DBK), m, sXs + i * NT + m);
         }
       }
       __syncwarp();
@@ -739,20 +712,33 @@ bool fit_split(Plan *p, int S, int64_t M, bool vec) {
   }
 }
 
+// The kernel a decode call runs.  FP8BQ_DECODE_KERNEL = narrow | wide | gemm
+// in the environment forces one where the shape allows it (narrow and wide
+// take M <= 64); unset or anything else is the default routing.
+enum Route { kAuto = 0, kNarrow, kWide, kGemm };
+
+Route route_override() {
+  const char *v = getenv("FP8BQ_DECODE_KERNEL");
+  if (v == nullptr) return kAuto;
+  if (strcmp(v, "narrow") == 0) return kNarrow;
+  if (strcmp(v, "wide") == 0) return kWide;
+  if (strcmp(v, "gemm") == 0) return kGemm;
+  return kAuto;
+}
+
 // vec: the activations allow 16-byte loads (x 16-byte aligned, ldx % 8 == 0).
 // The split S (CTAs per cluster, each a contiguous K range of every block of
 // its cluster) and the cluster count C (at most the resident clusters of that
 // size) minimise the modelled time: the busiest CTA's items,
 // ceil(NB / C) * ceil(KB / S), plus kRedItems per block when S > 1; ties go
-// to the smaller S.  Only splits whose shared memory fits count.
-Plan make_plan(int64_t M, int64_t N, int64_t K, bool vec, const DecodeDevice &dd) {
+// to the smaller S.  Only splits whose shared memory fits count.  narrow:
+// this kernel for any M <= 64; otherwise p.NT = 0 (the prefill GEMM).
+Plan make_plan(int64_t M, int64_t N, int64_t K, bool vec, const DecodeDevice &dd, bool narrow) {
   Plan p;
   p.S = p.C = 1;
   p.res = false;
   p.nres = p.nst = p.smem = 0;
-  // 0: the prefill GEMM (M > 64, or enough 256-row tiles of N: see above)
-  const int64_t ntiles = (N + 255) / 256;
-  p.NT = M <= kSwapMaxM && ntiles < kGemmAnyMNTiles && (M <= 32 || ntiles < kGemmMinNTiles) ? pick_nt(M) : 0;
+  p.NT = narrow && M <= kSwapMaxM ? pick_nt(M) : 0;
   p.NB = (int)((N + 127) / 128);
   p.KB = (int)(K / 128);
   workspace_layout(M, K, &p);
@@ -816,7 +802,19 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
   const fp8bq_status ready = decode_device(&dd);
   if (ready != FP8BQ_OK) return ready;
   const bool vec = aligned(x, 16) && ldx % 8 == 0;  // K % 128 == 0 already
-  const Plan p = make_plan(M, N, K, vec, *dd);
+  // the kernel: the wide form up to M = 64, except for M > 32 with at least
+  // kGemmMinNTiles 256-row weight tiles; the prefill GEMM above that
+  const int64_t ntiles = (N + 255) / 256;
+  Route route = route_override();
+  if (route == kAuto) route = M <= kSwapMaxM && (M <= 32 || ntiles < kGemmMinNTiles) ? kWide : kGemm;
+  DecodeWidePlan wp;
+  bool wide = false;
+  if (route == kWide) {
+    const fp8bq_status ws_st = plan_decode_wide(M, N, K, vec, &wp);
+    if (ws_st != FP8BQ_OK && ws_st != FP8BQ_ERR_UNSUPPORTED) return ws_st;
+    wide = ws_st == FP8BQ_OK;  // else the prefill GEMM (M > 64)
+  }
+  const Plan p = make_plan(M, N, K, vec, *dd, route == kNarrow);
   // the documented size (the path with a prologue), whichever path this call takes
   const size_t need = decode_workspace_size(M, N, K);
   if (ws_bytes < need || (need > 0 && (ws == nullptr || !aligned(ws, 256)))) return FP8BQ_ERR_WORKSPACE;
@@ -826,7 +824,7 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
   const uint16_t *xs = static_cast<const uint16_t *>(x);
 
   // 1. quantize X into the workspace, unless the GEMM kernel does it
-  if (!p.res) {
+  if (!(wide ? wp.res : p.res)) {
     if (vec) {
       dim3 grid((unsigned)((M + 63) / 64), (unsigned)p.KB);
       if (mode == FP8BQ_SCALE_FP32)
@@ -842,9 +840,10 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
     }
     fp8bq_status st = check_launch("gemm_decode prologue");
     if (st != FP8BQ_OK) return st;
-    if (p.NT == 0)  // M > 64: the prefill GEMM on the quantized activation
+    if (!wide && p.NT == 0)  // the prefill GEMM on the quantized activation
       return launch_gemm(q, K, sa, p.ldsa, qw, ldw, sw, y, ldy, M, N, K, mode, FP8BQ_GEMM_AUTO, stream);
   }
+  if (wide) return launch_decode_wide(wp, xs, ldx, qw, ldw, sw, q, sa, p.ldsa, y, ldy, M, N, K, mode, stream);
 
   // 2. the GEMM, K split over the CTAs of each cluster
   CUtensorMap tW, tX, tS;

@@ -140,6 +140,7 @@ cudaError_t take_device_error_pair(unsigned long long *v);
 cudaError_t take_device_error_swiglu(unsigned long long *v);
 cudaError_t take_device_error_wgrad(unsigned long long *v);
 cudaError_t take_device_error_prefill_attn(unsigned long long *v);
+cudaError_t take_device_error_decode_wide(unsigned long long *v);
 
 // Launchers (arguments already validated).
 fp8bq_status launch_encode(const float *x, int64_t n, uint8_t *q, cudaStream_t stream);
@@ -163,6 +164,22 @@ fp8bq_status check_decode_args(const void *x, int64_t ldx, const uint8_t *qw, in
                                const void *y, int64_t ldy, int64_t M, int64_t N, int64_t K, int mode, bool *work);
 fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, int64_t ldw, const float *sw, void *y,
                                 int64_t ldy, int64_t M, int64_t N, int64_t K, int mode, void *ws, size_t ws_bytes,
+                                cudaStream_t stream);
+// The decode GEMM's wide form (tokens as the 128-row MMA operand, 256 weight
+// rows per MMA, K split over clusters of up to 16 CTAs): its launch plan.
+struct DecodeWidePlan {
+  int NT;              // token rows held: M rounded up to 16, 32 or 64
+  int S, C;            // CTAs per cluster, clusters
+  int nst, nres, smem; // weight stages, resident K-blocks of codes, dynamic shared memory
+  bool res;            // activation quantized inside the kernel (no prologue)
+};
+// FP8BQ_ERR_UNSUPPORTED when the shape is outside the wide form (M > 64).
+// vec: the activations allow 16-byte loads.
+fp8bq_status plan_decode_wide(int64_t M, int64_t N, int64_t K, bool vec, DecodeWidePlan *p);
+// q/sa/ldsa: the prologue's codes and scales (unused when p.res).
+fp8bq_status launch_decode_wide(const DecodeWidePlan &p, const uint16_t *x, int64_t ldx, const uint8_t *qw,
+                                int64_t ldw, const float *sw, const uint8_t *q, const float *sa, int64_t ldsa,
+                                void *y, int64_t ldy, int64_t M, int64_t N, int64_t K, int mode,
                                 cudaStream_t stream);
 fp8bq_status launch_grouped_gemm(const uint8_t *qa, int64_t lda, const float *sa, int64_t ldsa, const uint8_t *qw,
                                  const float *sw, const int32_t *offsets, int E, int64_t rows, int64_t N, int64_t K,

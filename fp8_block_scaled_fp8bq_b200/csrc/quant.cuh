@@ -164,6 +164,32 @@ __device__ __forceinline__ uint32_t absmax_bits8(uint4 v) {
 
 __device__ __forceinline__ float bits_to_amax(uint32_t b16) { return __uint_as_float(b16 << 16); }
 
+// One 1x128 tile of the activation (row m, K-block kb) quantized by a group of
+// four lanes into a shared-memory tile of 128-byte rows in the MMA operand's
+// 128-byte-swizzled layout (16-byte chunk c of row m at chunk position
+// c ^ (m & 7)); lane qd of the group owns chunks qd, qd + 4,
+// qd + 8, qd + 12 of the row, as fp8bq_quant_act's vector kernel does.
+// Every lane of the warp calls it (the amax shuffles span the warp); lanes
+// with have == false store nothing.  v: the lane's four 16-byte pieces of the
+// row (pieces qd, qd + 4, qd + 8, qd + 12), loaded by the caller.
+template <int MODE>
+__device__ __forceinline__ void quant_row_tile_to_smem(bool have, const uint4 (&v)[4], int qd, uint8_t *tile, int m,
+                                                       float *scale) {
+  uint32_t am = max(max(absmax_bits8(v[0]), absmax_bits8(v[1])), max(absmax_bits8(v[2]), absmax_bits8(v[3])));
+  am = max(am, __shfl_xor_sync(0xffffffffu, am, 1));
+  am = max(am, __shfl_xor_sync(0xffffffffu, am, 2));
+  if (!have) return;
+  const TileScale ts = tile_scale<MODE>(bits_to_amax(am));
+  uint8_t *row = tile + m * 128;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e8 = j * 4 + qd;  // 8-element piece of the row
+    const uint2 c = fast_tile<MODE>(ts) ? encode8<MODE, true>(v[j], ts) : encode8<MODE>(v[j], ts);
+    *reinterpret_cast<uint2 *>(row + (((e8 >> 1) ^ (m & 7)) << 4) + (e8 & 1) * 8) = c;
+  }
+  if (qd == 0) *scale = ts.s;
+}
+
 // ---------------------------------------------------------------------------
 // Activation quantization, 1x128 tiles
 // ---------------------------------------------------------------------------
