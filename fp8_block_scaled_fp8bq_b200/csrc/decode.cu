@@ -59,10 +59,6 @@ constexpr int kDHighRegs = 224;
 static_assert(128 * kDLowRegs + 256 * kDHighRegs <= kDThreads * kDLaunchRegs, "register split");
 constexpr int kMaxDecodeM = 256;
 constexpr int kSwapMaxM = 64;
-// The prefill GEMM (128-token x 256-weight-row tiles) instead of the wide
-// form for M > 32 when the weight has at least this many 256-row tiles: it
-// fills the SMs without a split and its promotion runs on 128 token lanes.
-constexpr int kGemmMinNTiles = 64;
 constexpr int kResMaxM = 16;        // activation quantized inside the GEMM kernel up to this M ...
 constexpr int kResMaxTiles = 256;   // ... when a CTA's K range holds at most this many 1x128 tiles of X
 constexpr int kMaxSplit = 8;        // CTAs of a cluster (split of K)
@@ -590,11 +586,15 @@ __global__ void __launch_bounds__(kDThreads, 1)
   if (S > 1) cluster_sync();  // no CTA leaves while another may still address its shared memory
 }
 
-// Prologue: 1x128 quantization of X into the workspace.
+// Prologue: 1x128 quantization of X into the workspace.  Launched as a
+// programmatic dependent (it waits for the previous kernel before touching
+// memory) and lets the GEMM kernel that follows start its set-up at once.
 template <int MODE, bool VEC>
 __global__ void __launch_bounds__(256) decode_prologue_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
                                                               int64_t ldx, uint8_t *__restrict__ q,
                                                               float *__restrict__ sa, int64_t ldsa) {
+  pdl_launch_dependents();
+  pdl_wait();
   if constexpr (VEC) qdev::quant_act_vec_block<MODE>(blockIdx.x, blockIdx.y, x, M, K, ldx, q, K, sa, ldsa);
   else qdev::quant_act_scalar_block<MODE>(blockIdx.x, blockIdx.y, x, M, K, ldx, q, K, sa, ldsa);
 }
@@ -802,11 +802,11 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
   const fp8bq_status ready = decode_device(&dd);
   if (ready != FP8BQ_OK) return ready;
   const bool vec = aligned(x, 16) && ldx % 8 == 0;  // K % 128 == 0 already
-  // the kernel: the wide form up to M = 64, except for M > 32 with at least
-  // kGemmMinNTiles 256-row weight tiles; the prefill GEMM above that
-  const int64_t ntiles = (N + 255) / 256;
+  // the kernel: the wide form up to M = 64 (measured faster than the narrow
+  // form and the prefill GEMM on every Llama-8B projection at M = 1, 16, 64),
+  // the prefill GEMM above
   Route route = route_override();
-  if (route == kAuto) route = M <= kSwapMaxM && (M <= 32 || ntiles < kGemmMinNTiles) ? kWide : kGemm;
+  if (route == kAuto) route = M <= kSwapMaxM ? kWide : kGemm;
   DecodeWidePlan wp;
   bool wide = false;
   if (route == kWide) {
@@ -825,19 +825,21 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
 
   // 1. quantize X into the workspace, unless the GEMM kernel does it
   if (!(wide ? wp.res : p.res)) {
-    if (vec) {
-      dim3 grid((unsigned)((M + 63) / 64), (unsigned)p.KB);
-      if (mode == FP8BQ_SCALE_FP32)
-        decode_prologue_kernel<FP8BQ_SCALE_FP32, true><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, sa, p.ldsa);
-      else
-        decode_prologue_kernel<FP8BQ_SCALE_POW2, true><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, sa, p.ldsa);
-    } else {
-      dim3 grid((unsigned)((M + 15) / 16), (unsigned)p.KB);
-      if (mode == FP8BQ_SCALE_FP32)
-        decode_prologue_kernel<FP8BQ_SCALE_FP32, false><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, sa, p.ldsa);
-      else
-        decode_prologue_kernel<FP8BQ_SCALE_POW2, false><<<grid, 256, 0, stream>>>(xs, M, K, ldx, q, sa, p.ldsa);
-    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(256);
+    cfg.gridDim = dim3((unsigned)(vec ? (M + 63) / 64 : (M + 15) / 16), (unsigned)p.KB);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    auto kern = vec ? (mode == FP8BQ_SCALE_FP32 ? decode_prologue_kernel<FP8BQ_SCALE_FP32, true>
+                                                : decode_prologue_kernel<FP8BQ_SCALE_POW2, true>)
+                    : (mode == FP8BQ_SCALE_FP32 ? decode_prologue_kernel<FP8BQ_SCALE_FP32, false>
+                                                : decode_prologue_kernel<FP8BQ_SCALE_POW2, false>);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, xs, M, K, ldx, q, sa, p.ldsa);
+    if (e != cudaSuccess) return cuda_fail(e, "gemm_decode prologue launch");
     fp8bq_status st = check_launch("gemm_decode prologue");
     if (st != FP8BQ_OK) return st;
     if (!wide && p.NT == 0)  // the prefill GEMM on the quantized activation

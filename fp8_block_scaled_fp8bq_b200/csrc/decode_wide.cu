@@ -24,10 +24,17 @@
 //
 // Split over K in thread-block clusters of S CTAs (S up to 16): cluster c
 // owns tiles c, c + C, ...; rank r takes K-blocks r, r + S, ... of each.  At
-// the end of a tile every rank leaves its FP32 partial (NT x 256) in its own
-// shared memory, and rank r adds up column slice r of all S partials in rank
-// order (distributed shared memory, deterministic) and writes those columns
-// of Y: the cross-CTA sum is spread over the cluster.
+// the end of a tile every rank sends each 4-column piece of its FP32 partial
+// (NT x 256) to the rank that owns those columns (rank r owns slice r of the
+// 256 columns), with st.async stores into the owner's shared memory that
+// complete on the owner's mbarrier; the owner adds the S partials of its
+// slice in rank order (deterministic) and writes those columns of Y.  No
+// fence and no remote load is on that path, and the sum is spread over the
+// cluster.
+//
+// The kernel is launched as a programmatic dependent of the previous kernel
+// of the stream: its set-up (barriers, TMEM, cluster) overlaps that kernel's
+// tail, and every global access comes after griddepcontrol.wait.
 //
 // The activation's codes either come from a quantization inside this kernel
 // (M <= 16 and at most 256 1x128 tiles per CTA: the epilogue warps write them
@@ -69,6 +76,10 @@ constexpr int kWResMaxTiles = 256;   // 1x128 activation tiles per CTA quantized
 // CTA's items plus, for a split tile, about kWRedItems for the cross-CTA sum.
 constexpr int kWRedItems = 1;
 
+// Columns of a tile owned by each rank in the cross-CTA sum of a split of S:
+// whole 8-column pieces (rank r: [r c, min(256, (r + 1) c)), c = this).
+__host__ __device__ constexpr int slice_cols(int S) { return ((WBN + S - 1) / S + 7) / 8 * 8; }
+
 // QM < 0: activation codes and scales from the workspace (TMA, in the weight
 // stages); QM = FP8BQ_SCALE_FP32 / POW2: quantized in the kernel (NT = 16).
 template <int NT, int QM>
@@ -81,7 +92,6 @@ struct WCfg {
   static constexpr int kTx = kWBytes + (kRes ? 0 : kXBytes + kSBytes);
   static constexpr int kQuarters = (NT + 31) / 32;   // TMEM lane quarters holding tokens
   static constexpr int kActWarps = 4 * kQuarters;    // token warps (four column quarters each)
-  static constexpr int kPartFloats = NT * WBN;
   static constexpr int kTmemCols = 2 * WBN;          // two accumulator buffers
   static_assert(!kRes || NT == 16, "activation quantized in the kernel only for NT = 16");
   static_assert(kXBytes % 1024 == 0, "A tiles start on the 1024-byte swizzle atom");
@@ -89,14 +99,16 @@ struct WCfg {
   // Shared memory (after up to 1024 bytes of alignment): the codes (nres
   // resident K-blocks, or one slot per stage) first, so that the 16 KB an A
   // descriptor spans from any code tile stays inside the weight stages that
-  // follow; the weight stages; the activation scales; the partial (S > 1);
-  // the staged weight scales; the barriers.
+  // follow; the weight stages; the activation scales; the receive buffer of
+  // the cross-CTA sum (S > 1); the staged weight scales; the barriers.
   static __host__ __device__ int x_bytes(int nst, int nres) {
     return kRes ? (nres * kXBytes + 1023) / 1024 * 1024 : nst * kXBytes;
   }
   static __host__ __device__ int s_bytes(int nst, int nres) { return kRes ? nres * NT * 4 : nst * kSSlot; }
+  // [S][NT][slice_cols(S)]: every rank's partial of this CTA's column slice
+  static __host__ __device__ int recv_floats(int S) { return S > 1 ? S * NT * slice_cols(S) : 0; }
   static int smem_bytes(int nst, int nres, int S) {
-    return 1024 + x_bytes(nst, nres) + nst * kWBytes + s_bytes(nst, nres) + (S > 1 ? kPartFloats * 4 : 0) +
+    return 1024 + x_bytes(nst, nres) + nst * kWBytes + s_bytes(nst, nres) + recv_floats(S) * 4 +
            kWSwItems * 2 * 4 + 512;
   }
   static int stages_for(int nres, int S) {
@@ -179,8 +191,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
   uint8_t *sX = base;                                 // codes: nres resident tiles, or nst stage slots
   uint8_t *sW = sX + C::x_bytes(nst, args.nres);      // nst weight tiles
   float *sSx = reinterpret_cast<float *>(sW + nst * C::kWBytes);  // [nres][NT], or nst slots of kSSlot bytes
-  float *sP = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(sSx) + C::s_bytes(nst, args.nres));
-  float *sSw = sP + (S > 1 ? C::kPartFloats : 0);     // [kWSwItems][2]
+  float *sR = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(sSx) + C::s_bytes(nst, args.nres));
+  float *sSw = sR + C::recv_floats(S);                // [kWSwItems][2]
   uint64_t *bars = reinterpret_cast<uint64_t *>(sSw + 2 * kWSwItems);
   uint64_t *full = bars;
   uint64_t *empty = bars + kWMaxStages;
@@ -188,9 +200,9 @@ __global__ void __launch_bounds__(kWThreads, 1)
   uint64_t *tempty = tfull + 2;
   uint64_t *drain = tempty + 2;
   uint64_t *xready = drain + 1;   // resident activation codes written
-  uint64_t *pready = xready + 1;  // every rank's partial of the current tile is in its shared memory
-  uint64_t *pdone = pready + 1;   // every rank has read this CTA's partial
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pdone + 1);
+  uint64_t *rbar = xready + 1;    // every rank's partial of this CTA's slice has arrived (st.async bytes)
+  uint64_t *pfree = rbar + 1;     // every rank has read its slice: this CTA may send the next tile's pieces
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pfree + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -200,9 +212,6 @@ __global__ void __launch_bounds__(kWThreads, 1)
   const bool worker = warp >= kWWorkWarp0 && warp < kWWorkWarp0 + kWWorkWarps;
   const bool tokw = (warp & 3) < C::kQuarters && warp != kWProducerWarp && warp != kWMmaWarp;
 
-  // The workers issue the first pass of the activation's loads (when it is
-  // quantized here) and the weight scales' loads before the set-up, so that
-  // they overlap it.
   constexpr int kChunk = 2;  // passes of 64 1x128 tiles whose loads are issued together
   const int et = threadIdx.x - 32 * kWWorkWarp0;  // worker thread 0..255
   const int grp = et >> 2, qd = et & 3;
@@ -224,15 +233,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
     const int nb = 2 * sh.tile(q) + hh;
     return nb < args.NB ? __ldg(args.sw + (int64_t)nb * args.KB + sh.kb(q)) : 0.f;
   };
-  if (worker) {
-    if constexpr (kRes) load_pass(0, xv);
-#pragma unroll
-    for (int i = 0; i < 2 * kWSwItems / 256; ++i) {
-      const int z = et + 256 * i;
-      swv[i] = (z >> 1) < sh.items ? sw_global(z >> 1, z & 1) : 0.f;
-    }
-  }
-
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < nst; ++s) {
       mbar_init(&full[s], 1);
@@ -245,8 +246,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
     }
     mbar_init(drain, 1);
     mbar_init(xready, 1);
-    mbar_init(pready, S * C::kActWarps);  // the token warps of every rank
-    mbar_init(pdone, S * kWWorkWarps);    // the workers of every rank
+    mbar_init(rbar, 1);                   // this CTA's expect_tx; the bytes come from every rank
+    mbar_init(pfree, S * kWWorkWarps);    // the workers of every rank
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -266,6 +267,18 @@ __global__ void __launch_bounds__(kWThreads, 1)
   if (S > 1) cluster_sync();  // every CTA's barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the previous kernel of the stream has completed: global memory from here
+  // on.  The workers issue the first pass of the activation's loads (when it
+  // is quantized here) and the weight scales' loads first.
+  pdl_wait();
+  if (worker) {
+    if constexpr (kRes) load_pass(0, xv);
+#pragma unroll
+    for (int i = 0; i < 2 * kWSwItems / 256; ++i) {
+      const int z = et + 256 * i;
+      swv[i] = (z >> 1) < sh.items ? sw_global(z >> 1, z & 1) : 0.f;
+    }
+  }
 
   if (warp == kWProducerWarp) {
     if (lane == 0) {
@@ -384,8 +397,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
     for (int j = 0; j < 64; ++j) acc[j] = 0.f;
     bool alive = tokw || worker;
     auto sw_of = [&](int q) -> float { return q < kWSwItems ? sSw[2 * q + (g >> 1)] : sw_global(q, g >> 1); };
-    // this rank's column slice of the cross-CTA sum: whole 8-column pieces
-    const int cw = ((WBN + S - 1) / S + 7) / 8 * 8;
+    // this rank's column slice of the cross-CTA sum
+    const int cw = slice_cols(S);
     const int s0 = min(WBN, rank * cw), s1 = min(WBN, s0 + cw);
     const int nch = (s1 - s0) / 8;
     for (int jb = 0; jb < sh.nblk && alive; ++jb) {
@@ -452,27 +465,30 @@ __global__ void __launch_bounds__(kWThreads, 1)
         }
       } else {
         if (tokw) {
-          // the partial of tile jb, once every rank has read this CTA's partial of tile jb - 1;
-          // row m of sP holds 64 16-byte pieces, piece c at position c ^ (m & 7)
-          const bool fine = jb == 0 || mbar_wait_cluster(pdone, (uint32_t)((jb - 1) & 1), abort_flag, kSiteEpiTmemFull);
+          // tile jb's pieces, once every rank has read its slice of tile jb - 1:
+          // each 4-column piece to the rank that owns those columns
+          const bool fine = jb == 0 || mbar_wait_cluster(pfree, (uint32_t)((jb - 1) & 1), abort_flag, kSiteEpiTmemFull);
           if (!__all_sync(0xffffffffu, fine)) {
             alive = false;
             break;
           }
           if (m < args.M) {
-            float4 *prow = reinterpret_cast<float4 *>(sP + m * WBN);
+            const uint32_t row = smem_addr(sR + (rank * NT + m) * cw);
+            const uint32_t rb = smem_addr(rbar);
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-              prow[(16 * g + c) ^ (m & 7)] = make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+            for (int c = 0; c < 16; ++c) {
+              const int col = 64 * g + 4 * c;
+              const int owner = col / cw;
+              st_async_v4(mapa_shared(row + (uint32_t)(col - owner * cw) * 4u, (uint32_t)owner),
+                          make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]),
+                          mapa_shared(rb, (uint32_t)owner));
+            }
           }
-          asm volatile("fence.acq_rel.cluster;" ::: "memory");
-          __syncwarp();
-          if (lane == 0)
-            for (int pr = 0; pr < S; ++pr) mbar_arrive_cluster(mapa_shared(smem_addr(pready), (uint32_t)pr));
         }
         if (worker) {
           // columns [s0, s1) of tile jb: the S partials added in rank order
-          const bool got = mbar_wait_cluster(pready, (uint32_t)(jb & 1), abort_flag, kSiteEpiTmemFull);
+          if (warp == kWWorkWarp0 && lane == 0) mbar_arrive_expect_tx(rbar, (uint32_t)(S * args.M * (s1 - s0) * 4));
+          const bool got = mbar_wait_cluster(rbar, (uint32_t)(jb & 1), abort_flag, kSiteEpiTmemFull);
           if (!__all_sync(0xffffffffu, got)) {
             alive = false;
             break;
@@ -483,42 +499,29 @@ __global__ void __launch_bounds__(kWThreads, 1)
           for (int u = et; u < units; u += 256) {
             const int mm = u / nch, col = s0 + 8 * (u - mm * nch);
             if (nbase + col >= args.N) continue;
-            const uint32_t row = smem_addr(sP + mm * WBN);
-            const uint32_t o0 = row + ((uint32_t)((col >> 2) ^ (mm & 7)) << 4);
-            const uint32_t o1 = row + ((uint32_t)(((col >> 2) + 1) ^ (mm & 7)) << 4);
+            const float *src = sR + mm * cw + (col - s0);
             float sum[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) sum[j] = 0.f;
 #pragma unroll 1
-            for (int p0 = 0; p0 < S; p0 += 2) {
-              float4 a[2], b[2];
-#pragma unroll
-              for (int k = 0; k < 2; ++k) {
-                if (p0 + k < S) {
-                  a[k] = ld_shared_cluster_v4(mapa_shared(o0, (uint32_t)(p0 + k)));
-                  b[k] = ld_shared_cluster_v4(mapa_shared(o1, (uint32_t)(p0 + k)));
-                }
-              }
-#pragma unroll
-              for (int k = 0; k < 2; ++k) {
-                if (p0 + k < S) {
-                  sum[0] += a[k].x;
-                  sum[1] += a[k].y;
-                  sum[2] += a[k].z;
-                  sum[3] += a[k].w;
-                  sum[4] += b[k].x;
-                  sum[5] += b[k].y;
-                  sum[6] += b[k].z;
-                  sum[7] += b[k].w;
-                }
-              }
+            for (int p = 0; p < S; ++p) {
+              const float4 a = *reinterpret_cast<const float4 *>(src + p * (NT * cw));
+              const float4 b = *reinterpret_cast<const float4 *>(src + p * (NT * cw) + 4);
+              sum[0] += a.x;
+              sum[1] += a.y;
+              sum[2] += a.z;
+              sum[3] += a.w;
+              sum[4] += b.x;
+              sum[5] += b.y;
+              sum[6] += b.z;
+              sum[7] += b.w;
             }
             store8(args.y + (int64_t)mm * args.ldy, nbase + col, args.N, sum);
           }
-          // the partials have been read (their sums are stored): the ranks may overwrite them
+          // the slice has been read (its sums are stored): the ranks may send the next tile
           __syncwarp();
           if (lane == 0)
-            for (int pr = 0; pr < S; ++pr) mbar_arrive_cluster_relaxed(mapa_shared(smem_addr(pdone), (uint32_t)pr));
+            for (int pr = 0; pr < S; ++pr) mbar_arrive_cluster_relaxed(mapa_shared(smem_addr(pfree), (uint32_t)pr));
         }
       }
 #pragma unroll
@@ -532,7 +535,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
-  if (S > 1) cluster_sync();  // no CTA leaves while another may still read its shared memory
+  if (S > 1) cluster_sync();  // no CTA leaves while another may still write its shared memory
 }
 
 // Per-device set-up of the five instantiations (shared-memory and cluster-size
@@ -634,13 +637,15 @@ fp8bq_status launch_wide_nt(const CUtensorMap &tW, const CUtensorMap &tX, const 
   cfg.gridDim = dim3((unsigned)(p.C * p.S));
   cfg.dynamicSmemBytes = (size_t)p.smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)p.S;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)p.S;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = p.S > 1 ? 1 : 0;
+  cfg.numAttrs = p.S > 1 ? 2 : 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, decode_wide_kernel<NT, QM>, tW, tX, tS, a);
   if (e != cudaSuccess) return cuda_fail(e, "gemm_decode (wide) launch");
   return check_launch("gemm_decode (wide)");

@@ -410,6 +410,25 @@ __device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t cluster_addr) {
   return v;
 }
 
+// 16-byte asynchronous store into the shared memory of a CTA of the cluster
+// (16-byte aligned shared::cluster address); its completion counts 16 bytes
+// on that CTA's mbarrier `cluster_bar` (complete_tx), so the receiver learns
+// of it by waiting on its own barrier and the sender needs no fence.
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, float4 v, uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+               ::"r"(cluster_addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(cluster_bar)
+               : "memory");
+}
+
+// Programmatic dependent launch: let the next kernel of the stream (if it was
+// launched as a programmatic dependent) start its set-up, and wait until the
+// previous kernel of the stream has completed and its writes are visible
+// (returns at once for a kernel not launched as a dependent).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Relaxed remote arrive (see mbar_arrive_relaxed).
 __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
