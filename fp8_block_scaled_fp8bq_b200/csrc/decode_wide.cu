@@ -37,9 +37,9 @@
 // tail, and every global access comes after griddepcontrol.wait.
 //
 // The activation's codes either come from a quantization inside this kernel
-// (M <= 16 and at most 256 1x128 tiles per CTA: the epilogue warps write them
-// in the operand layout while the weight ring fills) or from the workspace,
-// written by a prologue kernel and loaded by TMA beside the weight tiles.
+// (M <= 16 and at most 64 1x128 tiles per CTA: worker warps write them in the
+// operand layout while the weight ring fills) or from the workspace, written
+// by a prologue kernel and loaded by TMA beside the weight tiles.
 #include <cuda_bf16.h>
 #include <string.h>
 
@@ -58,20 +58,22 @@ constexpr int WBN = 256, WBK = 128;
 // warps 2 and 3 (quarters that never hold a token) are the TMA producer and
 // the MMA issuer, and warp w of a token quarter takes weight columns
 // 64 (w / 4) .. 64 (w / 4) + 63 of the tile: 64 FP32 accumulators per thread
-// within the 128 registers a 512-thread CTA allows.  Warps 4..11 also
-// quantize the activation, stage the weight scales and do the cross-CTA sum.
+// within the 128 registers a 512-thread CTA allows.  Warps 4..11 (the
+// "workers") also quantize the activation, stage the weight scales and do the
+// cross-CTA sum.
 constexpr int kWThreads = 512;
 constexpr int kWProducerWarp = 2;
 constexpr int kWMmaWarp = 3;
-constexpr int kWWorkWarp0 = 4;        // warps 4..11: the 256 worker threads
 constexpr int kWMaxM = 64;
 constexpr int kWMaxSplit = 16;       // CTAs per cluster (above 8: the non-portable cluster sizes)
 constexpr int kWSmemCap = 232448;    // dynamic shared memory per CTA (227 KB)
 constexpr int kWMaxStages = 8;
 constexpr int kWMinStages = 3;
-constexpr int kWWorkWarps = 8;
 constexpr int kWSwItems = 256;       // work items whose two weight scales are staged in shared memory
-constexpr int kWResMaxTiles = 256;   // 1x128 activation tiles per CTA quantized in the kernel (M <= 16)
+// 1x128 activation tiles per CTA quantized inside the kernel (one pass of the
+// 256 worker threads, four per tile).  Measured: beyond one pass the prologue
+// kernel is faster (the extra passes' loads wait behind the weight stream).
+constexpr int kWResMaxTiles = 64;
 // Split choice, in units of one work item (a 32 KB weight tile): the busiest
 // CTA's items plus, for a split tile, about kWRedItems for the cross-CTA sum.
 constexpr int kWRedItems = 1;
@@ -86,12 +88,18 @@ template <int NT, int QM>
 struct WCfg {
   static constexpr bool kRes = QM >= 0;
   static constexpr int kWBytes = WBN * WBK;   // weight tile
-  static constexpr int kXBytes = NT * WBK;    // the token rows of one K-block's A tile
+  static constexpr int kXBytes = NT * WBK;    // the token rows of one K-block's A tile (a stage slot)
   static constexpr int kSBytes = NT * 4;      // the K-block's activation scales
   static constexpr int kSSlot = (kSBytes + 127) / 128 * 128;
   static constexpr int kTx = kWBytes + (kRes ? 0 : kXBytes + kSBytes);
   static constexpr int kQuarters = (NT + 31) / 32;   // TMEM lane quarters holding tokens
   static constexpr int kActWarps = 4 * kQuarters;    // token warps (four column quarters each)
+  // workers: warps 4..11 (some of them token warps as well).  Measured: the
+  // same role on the eight warps whose quarters hold no token was 0.3 to
+  // 1.6 us slower per call at M = 1 and 2.
+  static constexpr int kWorkWarps = 8;
+  static constexpr int kWorkThreads = 32 * kWorkWarps;
+  static __device__ __forceinline__ int work_slot(int w) { return w >= 4 && w < 12 ? w - 4 : -1; }
   static constexpr int kTmemCols = 2 * WBN;          // two accumulator buffers
   static_assert(!kRes || NT == 16, "activation quantized in the kernel only for NT = 16");
   static_assert(kXBytes % 1024 == 0, "A tiles start on the 1024-byte swizzle atom");
@@ -101,19 +109,22 @@ struct WCfg {
   // descriptor spans from any code tile stays inside the weight stages that
   // follow; the weight stages; the activation scales; the receive buffer of
   // the cross-CTA sum (S > 1); the staged weight scales; the barriers.
-  static __host__ __device__ int x_bytes(int nst, int nres) {
-    return kRes ? (nres * kXBytes + 1023) / 1024 * 1024 : nst * kXBytes;
+  // a resident K-block's codes: the M token rows rounded up to the 8-row
+  // swizzle atom (the A window's further rows read the next K-blocks' codes)
+  static __host__ __device__ int res_tile_bytes(int M) { return (M + 7) / 8 * 1024; }
+  static __host__ __device__ int x_bytes(int nst, int nres, int M) {
+    return kRes ? nres * res_tile_bytes(M) : nst * kXBytes;
   }
   static __host__ __device__ int s_bytes(int nst, int nres) { return kRes ? nres * NT * 4 : nst * kSSlot; }
-  // [S][NT][slice_cols(S)]: every rank's partial of this CTA's column slice
-  static __host__ __device__ int recv_floats(int S) { return S > 1 ? S * NT * slice_cols(S) : 0; }
-  static int smem_bytes(int nst, int nres, int S) {
-    return 1024 + x_bytes(nst, nres) + nst * kWBytes + s_bytes(nst, nres) + recv_floats(S) * 4 +
+  // [S][M][slice_cols(S)]: every rank's partial of this CTA's column slice
+  static __host__ __device__ int recv_floats(int S, int M) { return S > 1 ? S * M * slice_cols(S) : 0; }
+  static int smem_bytes(int nst, int nres, int S, int M) {
+    return 1024 + x_bytes(nst, nres, M) + nst * kWBytes + s_bytes(nst, nres) + recv_floats(S, M) * 4 +
            kWSwItems * 2 * 4 + 512;
   }
-  static int stages_for(int nres, int S) {
+  static int stages_for(int nres, int S, int M) {
     const int per = kWBytes + (kRes ? 0 : kXBytes + kSSlot);
-    const int n = (kWSmemCap - smem_bytes(0, nres, S)) / per;
+    const int n = (kWSmemCap - smem_bytes(0, nres, S, M)) / per;
     return n < kWMinStages ? 0 : (n > kWMaxStages ? kWMaxStages : n);
   }
 };
@@ -189,17 +200,18 @@ __global__ void __launch_bounds__(kWThreads, 1)
   const int nst = args.nst;
   const int S = args.split;
   uint8_t *sX = base;                                 // codes: nres resident tiles, or nst stage slots
-  uint8_t *sW = sX + C::x_bytes(nst, args.nres);      // nst weight tiles
+  uint8_t *sW = sX + C::x_bytes(nst, args.nres, args.M);  // nst weight tiles
+  const int xtile = C::res_tile_bytes(args.M);        // resident codes: bytes per K-block
   float *sSx = reinterpret_cast<float *>(sW + nst * C::kWBytes);  // [nres][NT], or nst slots of kSSlot bytes
   float *sR = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(sSx) + C::s_bytes(nst, args.nres));
-  float *sSw = sR + C::recv_floats(S);                // [kWSwItems][2]
+  float *sSw = sR + C::recv_floats(S, args.M);        // [kWSwItems][2]
   uint64_t *bars = reinterpret_cast<uint64_t *>(sSw + 2 * kWSwItems);
   uint64_t *full = bars;
   uint64_t *empty = bars + kWMaxStages;
   uint64_t *tfull = empty + kWMaxStages;
   uint64_t *tempty = tfull + 2;
   uint64_t *drain = tempty + 2;
-  uint64_t *xready = drain + 1;   // resident activation codes written
+  uint64_t *xready = drain + 1;   // the codes (if quantized here) and the staged weight scales are written
   uint64_t *rbar = xready + 1;    // every rank's partial of this CTA's slice has arrived (st.async bytes)
   uint64_t *pfree = rbar + 1;     // every rank has read its slice: this CTA may send the next tile's pieces
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pfree + 1);
@@ -209,24 +221,24 @@ __global__ void __launch_bounds__(kWThreads, 1)
   const int rank = S > 1 ? (int)cluster_ctarank() : 0;
   const WShare sh(args, S > 1 ? (int)cluster_id_x() : (int)blockIdx.x, S > 1 ? (int)nclusters_x() : (int)gridDim.x,
                   rank);
-  const bool worker = warp >= kWWorkWarp0 && warp < kWWorkWarp0 + kWWorkWarps;
+  const int wslot = C::work_slot(warp);
+  const bool worker = wslot >= 0;
   const bool tokw = (warp & 3) < C::kQuarters && warp != kWProducerWarp && warp != kWMmaWarp;
 
-  constexpr int kChunk = 2;  // passes of 64 1x128 tiles whose loads are issued together
-  const int et = threadIdx.x - 32 * kWWorkWarp0;  // worker thread 0..255
+  const int et = 32 * wslot + lane;  // worker thread 0 .. kWorkThreads - 1
   const int grp = et >> 2, qd = et & 3;
-  uint4 xv[kChunk][4];
-  float swv[2 * kWSwItems / 256];
-  auto load_pass = [&](int c0, uint4 (&v)[kChunk][4]) {
-    const int ntile = sh.nk * args.M;
+  // The activation's loads (when it is quantized here): tile t of the CTA's
+  // nk * M <= 64 (K-block t / M, row t % M) by the four lanes of group t.
+  uint4 xv[4];
+  constexpr int kSwPer = (2 * kWSwItems + C::kWorkThreads - 1) / C::kWorkThreads;
+  float swv[kSwPer];
+  auto load_x = [&]() {
+    const int t = grp;
+    const int i = t / args.M, m = t - (t / args.M) * args.M;
+    const uint16_t *xrow = args.x + (int64_t)m * args.ldx + (int64_t)(sh.kb0 + i * sh.ks) * WBK;
+    const bool have = t < sh.nk * args.M;
 #pragma unroll
-    for (int u = 0; u < kChunk; ++u) {
-      const int t = c0 + 64 * u + grp;
-      const int i = t / args.M, m = t - (t / args.M) * args.M;
-      const uint16_t *xrow = args.x + (int64_t)m * args.ldx + (int64_t)(sh.kb0 + i * sh.ks) * WBK;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) v[u][j] = t < ntile ? ld_nc_v4(xrow + (j * 4 + qd) * 8) : make_uint4(0, 0, 0, 0);
-    }
+    for (int j = 0; j < 4; ++j) xv[j] = have ? ld_nc_v4(xrow + (j * 4 + qd) * 8) : make_uint4(0, 0, 0, 0);
   };
   // weight scale of item q's half hh (0 for a half beyond the last weight row)
   auto sw_global = [&](int q, int hh) -> float {
@@ -245,9 +257,9 @@ __global__ void __launch_bounds__(kWThreads, 1)
       mbar_init(&tempty[b], C::kActWarps);
     }
     mbar_init(drain, 1);
-    mbar_init(xready, 1);
+    mbar_init(xready, C::kWorkWarps);
     mbar_init(rbar, 1);                   // this CTA's expect_tx; the bytes come from every rank
-    mbar_init(pfree, S * kWWorkWarps);    // the workers of every rank
+    mbar_init(pfree, S * C::kWorkWarps);  // the workers of every rank
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -267,16 +279,16 @@ __global__ void __launch_bounds__(kWThreads, 1)
   if (S > 1) cluster_sync();  // every CTA's barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // the previous kernel of the stream has completed: global memory from here
-  // on.  The workers issue the first pass of the activation's loads (when it
-  // is quantized here) and the weight scales' loads first.
+  // After the wait (the previous kernel of the stream has completed) global
+  // memory is read and written; the workers issue the activation's loads and
+  // the weight scales' loads first.
   pdl_wait();
   if (worker) {
-    if constexpr (kRes) load_pass(0, xv);
+    if constexpr (kRes) load_x();
 #pragma unroll
-    for (int i = 0; i < 2 * kWSwItems / 256; ++i) {
-      const int z = et + 256 * i;
-      swv[i] = (z >> 1) < sh.items ? sw_global(z >> 1, z & 1) : 0.f;
+    for (int i = 0; i < kSwPer; ++i) {
+      const int z = et + C::kWorkThreads * i;
+      swv[i] = z < 2 * kWSwItems && (z >> 1) < sh.items ? sw_global(z >> 1, z & 1) : 0.f;
     }
   }
 
@@ -317,7 +329,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
       int stage = 0, buf = 0;
       uint32_t phase = 0, bphase = 0;
       bool ok = true, issued = false;
-      if constexpr (kRes) ok = mbar_wait(xready, 0, abort_flag, kSiteMmaFull);  // the resident codes are written
+      if constexpr (kRes) ok = mbar_wait(xready, 0, abort_flag, kSiteMmaFull);  // the codes are written
       for (int q = 0; q < sh.items && ok; ++q) {
         if (!mbar_wait(&tempty[buf], bphase ^ 1, abort_flag, kSiteMmaTmemEmpty) ||
             !mbar_wait(&full[stage], phase, abort_flag, kSiteMmaFull)) {
@@ -326,7 +338,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(buf * WBN);
-        const uint32_t a0 = kRes ? smem_addr(sX + sh.pos(q) * C::kXBytes) : smem_addr(sX + stage * C::kXBytes);
+        const uint32_t a0 = kRes ? smem_addr(sX + sh.pos(q) * xtile) : smem_addr(sX + stage * C::kXBytes);
         const uint32_t b0 = smem_addr(sW + stage * C::kWBytes);
 #pragma unroll
         for (int k = 0; k < WBK / 32; ++k)
@@ -351,46 +363,33 @@ __global__ void __launch_bounds__(kWThreads, 1)
   } else {
     if (worker) {
 #pragma unroll
-      for (int i = 0; i < 2 * kWSwItems / 256; ++i)
-        if (((et + 256 * i) >> 1) < sh.items) sSw[et + 256 * i] = swv[i];
+      for (int i = 0; i < kSwPer; ++i) {
+        const int z = et + C::kWorkThreads * i;
+        if (z < 2 * kWSwItems && (z >> 1) < sh.items) sSw[z] = swv[i];
+      }
       if constexpr (kRes) {
         // ---------------------------------------------------------- activation quantization
         // tile (i, m) for i < nk, m < M, four lanes each (groups never
-        // straddle a warp); rows M..15 of a code tile are left as they are:
-        // they only feed accumulator rows that are never read
-        const int ntile = sh.nk * args.M;
-#pragma unroll 1
-        for (int c0 = 0; c0 < ntile; c0 += 64 * kChunk) {
-          uint4 v[kChunk][4];
-          if (c0 == 0) {
-#pragma unroll
-            for (int u = 0; u < kChunk; ++u)
-#pragma unroll
-              for (int j = 0; j < 4; ++j) v[u][j] = xv[u][j];
-          } else {
-            load_pass(c0, v);
-          }
-#pragma unroll
-          for (int u = 0; u < kChunk; ++u) {
-            const int t = c0 + 64 * u + grp;
-            const bool have = t < ntile;
-            const int i = have ? t / args.M : 0, m = have ? t - (t / args.M) * args.M : 0;
-            qdev::quant_row_tile_to_smem<QM < 0 ? 0 : QM>(have, v[u], qd, sX + i * C::kXBytes, m, sSx + i * NT + m);
-          }
-        }
+        // straddle a warp); a code tile's rows from M up to its 8-row atom
+        // are left as they are: they only feed accumulator rows never read
+        const int t = grp;
+        const bool have = t < sh.nk * args.M;
+        const int i = have ? t / args.M : 0, m = have ? t - (t / args.M) * args.M : 0;
+        qdev::quant_row_tile_to_smem<QM < 0 ? 0 : QM>(have, xv, qd, sX + i * xtile, m, sSx + i * NT + m);
         __syncwarp();
         fence_proxy_async_smem();
+      } else {
+        __syncwarp();
       }
+      if (lane == 0) mbar_arrive(xready);
     }
-    // the codes, their scales and the staged weight scales are written
-    named_barrier_sync(1, kWThreads - 64);
-    if (kRes && warp == kWWorkWarp0 && lane == 0) mbar_arrive(xready);
     // ------------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     const int g = warp >> 2;                    // weight columns 64 g .. 64 g + 63 of the tile
     const int m = quarter * 32 + lane;          // token = accumulator row (token warps)
     const int ms = m < NT ? m : NT - 1;         // its scale slot (lanes beyond NT read a valid one)
     int stage = 0, buf = 0;
+    bool xw = false;  // xready seen
     uint32_t bphase = 0;
     float acc[64];
 #pragma unroll
@@ -413,6 +412,13 @@ __global__ void __launch_bounds__(kWThreads, 1)
             break;
           }
           tc_fence_after();
+          // the activation scales and the weight scales are written
+          const bool xok = xw || mbar_wait(xready, 0, abort_flag, kSiteEpiTmemFull);
+          xw = true;
+          if (!__all_sync(0xffffffffu, xok)) {
+            alive = false;
+            break;
+          }
           float sx;
           if constexpr (kRes) sx = sSx[i * NT + ms];
           else sx = sSx[stage * (C::kSSlot / 4) + ms];
@@ -473,21 +479,28 @@ __global__ void __launch_bounds__(kWThreads, 1)
             break;
           }
           if (m < args.M) {
-            const uint32_t row = smem_addr(sR + (rank * NT + m) * cw);
+            const uint32_t row = smem_addr(sR + (rank * args.M + m) * cw);
             const uint32_t rb = smem_addr(rbar);
+            int owner = (64 * g) / cw;
+            int ob = owner * cw;
+            uint32_t dst_row = mapa_shared(row, (uint32_t)owner), dst_bar = mapa_shared(rb, (uint32_t)owner);
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
               const int col = 64 * g + 4 * c;
-              const int owner = col / cw;
-              st_async_v4(mapa_shared(row + (uint32_t)(col - owner * cw) * 4u, (uint32_t)owner),
-                          make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]),
-                          mapa_shared(rb, (uint32_t)owner));
+              if (col >= ob + cw) {
+                ++owner;
+                ob += cw;
+                dst_row = mapa_shared(row, (uint32_t)owner);
+                dst_bar = mapa_shared(rb, (uint32_t)owner);
+              }
+              st_async_v4(dst_row + (uint32_t)(col - ob) * 4u,
+                          make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]), dst_bar);
             }
           }
         }
         if (worker) {
           // columns [s0, s1) of tile jb: the S partials added in rank order
-          if (warp == kWWorkWarp0 && lane == 0) mbar_arrive_expect_tx(rbar, (uint32_t)(S * args.M * (s1 - s0) * 4));
+          if (wslot == 0 && lane == 0) mbar_arrive_expect_tx(rbar, (uint32_t)(S * args.M * (s1 - s0) * 4));
           const bool got = mbar_wait_cluster(rbar, (uint32_t)(jb & 1), abort_flag, kSiteEpiTmemFull);
           if (!__all_sync(0xffffffffu, got)) {
             alive = false;
@@ -496,17 +509,17 @@ __global__ void __launch_bounds__(kWThreads, 1)
           const int nbase = t * WBN;
           const int units = args.M * nch;
 #pragma unroll 1
-          for (int u = et; u < units; u += 256) {
+          for (int u = et; u < units; u += C::kWorkThreads) {
             const int mm = u / nch, col = s0 + 8 * (u - mm * nch);
             if (nbase + col >= args.N) continue;
             const float *src = sR + mm * cw + (col - s0);
             float sum[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) sum[j] = 0.f;
-#pragma unroll 1
+#pragma unroll 4
             for (int p = 0; p < S; ++p) {
-              const float4 a = *reinterpret_cast<const float4 *>(src + p * (NT * cw));
-              const float4 b = *reinterpret_cast<const float4 *>(src + p * (NT * cw) + 4);
+              const float4 a = *reinterpret_cast<const float4 *>(src + p * (args.M * cw));
+              const float4 b = *reinterpret_cast<const float4 *>(src + p * (args.M * cw) + 4);
               sum[0] += a.x;
               sum[1] += a.y;
               sum[2] += a.z;
@@ -520,8 +533,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
           }
           // the slice has been read (its sums are stored): the ranks may send the next tile
           __syncwarp();
-          if (lane == 0)
-            for (int pr = 0; pr < S; ++pr) mbar_arrive_cluster_relaxed(mapa_shared(smem_addr(pfree), (uint32_t)pr));
+          if (lane < S) mbar_arrive_cluster_relaxed(mapa_shared(smem_addr(pfree), (uint32_t)lane));
         }
       }
 #pragma unroll
@@ -606,24 +618,24 @@ bool fit_wide(DecodeWidePlan *p, int S, int64_t M, int KB, bool vec) {
   p->res = false;
   if (p->NT == 16 && vec && nk * M <= kWResMaxTiles) {
     p->nres = nk;
-    p->nst = WCfg<16, FP8BQ_SCALE_FP32>::stages_for(nk, S);  // both modes lay shared memory out alike
-    p->smem = WCfg<16, FP8BQ_SCALE_FP32>::smem_bytes(p->nst, nk, S);
+    p->nst = WCfg<16, FP8BQ_SCALE_FP32>::stages_for(nk, S, (int)M);  // both modes lay shared memory out alike
+    p->smem = WCfg<16, FP8BQ_SCALE_FP32>::smem_bytes(p->nst, nk, S, (int)M);
     p->res = p->nst > 0;
     if (p->res) return true;
   }
   p->nres = 0;
   switch (p->NT) {
     case 16:
-      p->nst = WCfg<16, -1>::stages_for(0, S);
-      p->smem = WCfg<16, -1>::smem_bytes(p->nst, 0, S);
+      p->nst = WCfg<16, -1>::stages_for(0, S, (int)M);
+      p->smem = WCfg<16, -1>::smem_bytes(p->nst, 0, S, (int)M);
       break;
     case 32:
-      p->nst = WCfg<32, -1>::stages_for(0, S);
-      p->smem = WCfg<32, -1>::smem_bytes(p->nst, 0, S);
+      p->nst = WCfg<32, -1>::stages_for(0, S, (int)M);
+      p->smem = WCfg<32, -1>::smem_bytes(p->nst, 0, S, (int)M);
       break;
     default:
-      p->nst = WCfg<64, -1>::stages_for(0, S);
-      p->smem = WCfg<64, -1>::smem_bytes(p->nst, 0, S);
+      p->nst = WCfg<64, -1>::stages_for(0, S, (int)M);
+      p->smem = WCfg<64, -1>::smem_bytes(p->nst, 0, S, (int)M);
       break;
   }
   return p->nst > 0;

@@ -231,13 +231,14 @@ FP8BQ_API fp8bq_status fp8bq_gemm_ex(const uint8_t *qa, int64_t lda, const float
  * weight rows its N dimension, with K split over the CTAs of thread-block
  * clusters (up to 16) whose partial sums are added over distributed shared
  * memory in a fixed rank order (results are deterministic); for M > 64 the
- * prefill GEMM runs on the quantized activation.  One launch when M <= 16, x is 16-byte
- * aligned with ldx % 8 == 0 and each CTA's share of K holds at most 256 of
- * X's 1x128 tiles (the activation is then quantized inside the GEMM kernel);
- * two launches otherwise.  The environment variable FP8BQ_DECODE_KERNEL =
- * wide | narrow | gemm forces a kernel where the shape allows it (narrow: the
- * weight as the 128-row operand and the tokens as N, M <= 64), for
- * comparisons; it is read at every call.
+ * prefill GEMM runs on the quantized activation.  One launch when M <= 16, x
+ * is 16-byte aligned with ldx % 8 == 0 and each CTA's share of K holds at
+ * most 64 of X's 1x128 tiles (the activation is then quantized inside the
+ * GEMM kernel; 256 for the narrow form); two launches otherwise.  The
+ * environment variable FP8BQ_DECODE_KERNEL = wide | narrow | gemm forces a
+ * kernel where the shape allows it (narrow: the weight as the 128-row
+ * operand and the tokens as N, M <= 64), for comparisons; it is read at
+ * every call.
  * Requirements: as fp8bq_gemm, and M <= 256.  Output equals fp8bq_quant_act
  * followed by fp8bq_gemm up to FP32 summation order.
  */
