@@ -64,7 +64,7 @@ constexpr int WBN = 256, WBK = 128;
 constexpr int kWThreads = 512;
 constexpr int kWProducerWarp = 2;
 constexpr int kWMmaWarp = 3;
-constexpr int kWMaxM = 64;
+constexpr int kWMaxM = 256;          // tokens; above 64 in groups of 64 (one block per weight tile and group)
 constexpr int kWMaxSplit = 16;       // CTAs per cluster (above 8: the non-portable cluster sizes)
 constexpr int kWSmemCap = 232448;    // dynamic shared memory per CTA (227 KB)
 constexpr int kWMaxStages = 8;
@@ -133,6 +133,7 @@ struct WideArgs {
   const float *sw;
   int32_t M, N, KB, NB;  // NB: 128-row weight blocks (rows of sw)
   int32_t NW;            // 256-row weight tiles
+  int32_t MG;            // token groups of 64 rows (1 when M <= 64)
   int32_t split;         // CTAs per cluster (S)
   int32_t nst;           // weight stages
   int32_t nres;          // resident K-blocks of activation codes (0 unless quantized in the kernel)
@@ -142,22 +143,30 @@ struct WideArgs {
   int64_t ldx;
 };
 
-// The work of CTA `rank` of cluster `cid` (of `ncl`): tiles cid, cid + ncl,
-// ... and of each the K-blocks rank, rank + S, ... (interleaved, so that the
-// cluster's CTAs stream neighbouring pieces of the same weight rows at the
-// same time); item q is tile t0 + (q / nk) * ncl, K-block kb0 + (q % nk) * S.
+// A block is a (256-row weight tile, group of 64 tokens) pair, block b =
+// tile * MG + group (the groups of a tile are neighbours, so the clusters
+// streaming one weight tile for different tokens run at the same time and
+// share it in L2).  The work of CTA `rank` of cluster `cid` (of `ncl`):
+// blocks cid, cid + ncl, ... and of each the K-blocks rank, rank + S, ...
+// (interleaved, so that the cluster's CTAs stream neighbouring pieces of the
+// same weight rows at the same time); item q is block t0 + (q / nk) * ncl,
+// K-block kb0 + (q % nk) * S.
 struct WShare {
-  int t0, ncl, kb0, ks, nk, nblk, items;
+  int t0, ncl, kb0, ks, nk, nblk, items, mg;
   __device__ WShare(const WideArgs &a, int cid, int ncls, int rank) {
     t0 = cid;
     ncl = ncls;
     kb0 = rank;
     ks = a.split;
     nk = (a.KB - rank + a.split - 1) / a.split;
-    nblk = cid < a.NW ? (a.NW - cid + ncls - 1) / ncls : 0;
+    mg = a.MG;
+    const int nbt = a.NW * a.MG;
+    nblk = cid < nbt ? (nbt - cid + ncls - 1) / ncls : 0;
     items = nblk * nk;
   }
-  __device__ int tile(int q) const { return t0 + (q / nk) * ncl; }
+  __device__ int blk(int q) const { return t0 + (q / nk) * ncl; }
+  __device__ int tile(int q) const { return blk(q) / mg; }
+  __device__ int tgroup(int q) const { return blk(q) % mg; }
   __device__ int pos(int q) const { return q % nk; }
   __device__ int kb(int q) const { return kb0 + (q % nk) * ks; }
 };
@@ -204,7 +213,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
   const int xtile = C::res_tile_bytes(args.M);        // resident codes: bytes per K-block
   float *sSx = reinterpret_cast<float *>(sW + nst * C::kWBytes);  // [nres][NT], or nst slots of kSSlot bytes
   float *sR = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(sSx) + C::s_bytes(nst, args.nres));
-  float *sSw = sR + C::recv_floats(S, args.M);        // [kWSwItems][2]
+  float *sSw = sR + C::recv_floats(S, min(args.M, NT));  // [kWSwItems][2]
   uint64_t *bars = reinterpret_cast<uint64_t *>(sSw + 2 * kWSwItems);
   uint64_t *full = bars;
   uint64_t *empty = bars + kWMaxStages;
@@ -299,7 +308,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
       uint32_t phase = 0, armed = 0, armed_parity = 0;
       bool ok = true;
       for (int q = 0; q < sh.items; ++q) {
-        const int t = sh.tile(q), kb = sh.kb(q);
+        const int t = sh.tile(q), kb = sh.kb(q), r0 = 64 * sh.tgroup(q);
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, kSiteProducerEmpty)) {
           ok = false;
           break;
@@ -307,8 +316,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
         mbar_arrive_expect_tx(&full[stage], C::kTx);
         tma_load_2d(sW + stage * C::kWBytes, &tmW, &full[stage], kb * WBK, t * WBN);
         if constexpr (!kRes) {
-          tma_load_2d(sX + stage * C::kXBytes, &tmX, &full[stage], kb * WBK, 0);
-          tma_load_2d(reinterpret_cast<uint8_t *>(sSx) + stage * C::kSSlot, &tmS, &full[stage], 0, kb);
+          tma_load_2d(sX + stage * C::kXBytes, &tmX, &full[stage], kb * WBK, r0);
+          tma_load_2d(reinterpret_cast<uint8_t *>(sSx) + stage * C::kSSlot, &tmS, &full[stage], r0, kb);
         }
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -401,7 +410,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
     const int s0 = min(WBN, rank * cw), s1 = min(WBN, s0 + cw);
     const int nch = (s1 - s0) / 8;
     for (int jb = 0; jb < sh.nblk && alive; ++jb) {
-      const int t = sh.tile(jb * sh.nk);
+      const int t = sh.tile(jb * sh.nk), r0 = 64 * sh.tgroup(jb * sh.nk);
+      const int Mb = min(args.M - r0, 64);  // this block's tokens: rows r0 .. r0 + Mb - 1
       if (tokw) {
 #pragma unroll 1
         for (int i = 0; i < sh.nk; ++i) {
@@ -450,8 +460,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
       }
       if (!alive) break;
       if (S == 1) {
-        if (tokw && m < args.M) {
-          uint16_t *yr = args.y + (int64_t)m * args.ldy;
+        if (tokw && m < Mb) {
+          uint16_t *yr = args.y + (int64_t)(r0 + m) * args.ldy;
           const int n0 = t * WBN + g * 64;
           if (n0 + 64 <= args.N) {
 #pragma unroll
@@ -478,8 +488,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
             alive = false;
             break;
           }
-          if (m < args.M) {
-            const uint32_t row = smem_addr(sR + (rank * args.M + m) * cw);
+          if (m < Mb) {
+            const uint32_t row = smem_addr(sR + (rank * Mb + m) * cw);
             const uint32_t rb = smem_addr(rbar);
             int owner = (64 * g) / cw;
             int ob = owner * cw;
@@ -500,14 +510,14 @@ __global__ void __launch_bounds__(kWThreads, 1)
         }
         if (worker) {
           // columns [s0, s1) of tile jb: the S partials added in rank order
-          if (wslot == 0 && lane == 0) mbar_arrive_expect_tx(rbar, (uint32_t)(S * args.M * (s1 - s0) * 4));
+          if (wslot == 0 && lane == 0) mbar_arrive_expect_tx(rbar, (uint32_t)(S * Mb * (s1 - s0) * 4));
           const bool got = mbar_wait_cluster(rbar, (uint32_t)(jb & 1), abort_flag, kSiteEpiTmemFull);
           if (!__all_sync(0xffffffffu, got)) {
             alive = false;
             break;
           }
           const int nbase = t * WBN;
-          const int units = args.M * nch;
+          const int units = Mb * nch;
 #pragma unroll 1
           for (int u = et; u < units; u += C::kWorkThreads) {
             const int mm = u / nch, col = s0 + 8 * (u - mm * nch);
@@ -518,8 +528,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
             for (int j = 0; j < 8; ++j) sum[j] = 0.f;
 #pragma unroll 4
             for (int p = 0; p < S; ++p) {
-              const float4 a = *reinterpret_cast<const float4 *>(src + p * (args.M * cw));
-              const float4 b = *reinterpret_cast<const float4 *>(src + p * (args.M * cw) + 4);
+              const float4 a = *reinterpret_cast<const float4 *>(src + p * (Mb * cw));
+              const float4 b = *reinterpret_cast<const float4 *>(src + p * (Mb * cw) + 4);
               sum[0] += a.x;
               sum[1] += a.y;
               sum[2] += a.z;
@@ -529,7 +539,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
               sum[6] += b.z;
               sum[7] += b.w;
             }
-            store8(args.y + (int64_t)mm * args.ldy, nbase + col, args.N, sum);
+            store8(args.y + (int64_t)(r0 + mm) * args.ldy, nbase + col, args.N, sum);
           }
           // the slice has been read (its sums are stored): the ranks may send the next tile
           __syncwarp();
@@ -624,18 +634,19 @@ bool fit_wide(DecodeWidePlan *p, int S, int64_t M, int KB, bool vec) {
     if (p->res) return true;
   }
   p->nres = 0;
+  const int mrows = (int)std::min<int64_t>(M, 64);  // a block's tokens at most
   switch (p->NT) {
     case 16:
-      p->nst = WCfg<16, -1>::stages_for(0, S, (int)M);
-      p->smem = WCfg<16, -1>::smem_bytes(p->nst, 0, S, (int)M);
+      p->nst = WCfg<16, -1>::stages_for(0, S, mrows);
+      p->smem = WCfg<16, -1>::smem_bytes(p->nst, 0, S, mrows);
       break;
     case 32:
-      p->nst = WCfg<32, -1>::stages_for(0, S, (int)M);
-      p->smem = WCfg<32, -1>::smem_bytes(p->nst, 0, S, (int)M);
+      p->nst = WCfg<32, -1>::stages_for(0, S, mrows);
+      p->smem = WCfg<32, -1>::smem_bytes(p->nst, 0, S, mrows);
       break;
     default:
-      p->nst = WCfg<64, -1>::stages_for(0, S, (int)M);
-      p->smem = WCfg<64, -1>::smem_bytes(p->nst, 0, S, (int)M);
+      p->nst = WCfg<64, -1>::stages_for(0, S, mrows);
+      p->smem = WCfg<64, -1>::smem_bytes(p->nst, 0, S, mrows);
       break;
   }
   return p->nst > 0;
@@ -677,13 +688,14 @@ fp8bq_status plan_decode_wide(int64_t M, int64_t N, int64_t K, bool vec, DecodeW
   const fp8bq_status ready = wide_device(&wd);
   if (ready != FP8BQ_OK) return ready;
   p->NT = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
-  const int NW = (int)((N + WBN - 1) / WBN);
+  p->MG = (int)((M + 63) / 64);
+  const int NBT = (int)((N + WBN - 1) / WBN) * p->MG;  // blocks: weight tiles x token groups
   const int KB = (int)(K / WBK);
   int best = 0x7fffffff, bestS = 0;
   for (int s = 1; s <= kWMaxSplit && s <= KB; ++s) {
-    const int c = std::min(NW, std::min(wd->max_clusters[1] / s, wd->max_clusters[s]));
+    const int c = std::min(NBT, std::min(wd->max_clusters[1] / s, wd->max_clusters[s]));
     if (c < 1 || !fit_wide(p, s, M, KB, vec)) continue;
-    const int blocks = (NW + c - 1) / c;
+    const int blocks = (NBT + c - 1) / c;
     const int cost = blocks * ((KB + s - 1) / s) + (s > 1 ? blocks * kWRedItems : 0);
     if (cost < best) {
       best = cost;
@@ -692,7 +704,7 @@ fp8bq_status plan_decode_wide(int64_t M, int64_t N, int64_t K, bool vec, DecodeW
   }
   if (bestS == 0) return FP8BQ_ERR_UNSUPPORTED;
   p->S = bestS;
-  p->C = std::min(NW, std::min(wd->max_clusters[1] / bestS, wd->max_clusters[bestS]));
+  p->C = std::min(NBT, std::min(wd->max_clusters[1] / bestS, wd->max_clusters[bestS]));
   fit_wide(p, bestS, M, KB, vec);
   return FP8BQ_OK;
 }
@@ -721,6 +733,7 @@ fp8bq_status launch_decode_wide(const DecodeWidePlan &p, const uint16_t *x, int6
   a.KB = (int32_t)(K / WBK);
   a.NB = (int32_t)((N + 127) / 128);
   a.NW = (int32_t)((N + WBN - 1) / WBN);
+  a.MG = p.MG;
   a.split = p.S;
   a.nst = p.nst;
   a.nres = p.nres;

@@ -168,12 +168,13 @@ fp8bq_status launch_gemm_decode(const void *x, int64_t ldx, const uint8_t *qw, i
 // The decode GEMM's wide form (tokens as the 128-row MMA operand, 256 weight
 // rows per MMA, K split over clusters of up to 16 CTAs): its launch plan.
 struct DecodeWidePlan {
-  int NT;              // token rows held: M rounded up to 16, 32 or 64
+  int NT;              // token rows held per block: M rounded up to 16, 32 or 64
+  int MG;              // groups of 64 tokens (M > 64: each weight tile is streamed once per group)
   int S, C;            // CTAs per cluster, clusters
   int nst, nres, smem; // weight stages, resident K-blocks of codes, dynamic shared memory
   bool res;            // activation quantized inside the kernel (no prologue)
 };
-// FP8BQ_ERR_UNSUPPORTED when the shape is outside the wide form (M > 64).
+// FP8BQ_ERR_UNSUPPORTED when the shape is outside the wide form (M > 256).
 // vec: the activations allow 16-byte loads.
 fp8bq_status plan_decode_wide(int64_t M, int64_t N, int64_t K, bool vec, DecodeWidePlan *p);
 // q/sa/ldsa: the prologue's codes and scales (unused when p.res).

@@ -231,8 +231,9 @@ FP8BQ_API fp8bq_status fp8bq_gemm_ex(const uint8_t *qa, int64_t lda, const float
  * Kernels: up to M = 64 the tokens are the MMA's 128-row operand and 256
  * weight rows its N dimension, with K split over the CTAs of thread-block
  * clusters (up to 16) whose partial sums are added over distributed shared
- * memory in a fixed rank order (results are deterministic); for M > 64 the
- * prefill GEMM runs on the quantized activation.  One launch when M <= 16, x
+ * memory in a fixed rank order (results are deterministic); for 64 < M <= 256
+ * the same kernel in groups of 64 tokens when N <= 4096, else the prefill
+ * GEMM on the quantized activation.  One launch when M <= 16, x
  * is 16-byte aligned with ldx % 8 == 0 and each CTA's share of K holds at
  * most 64 of X's 1x128 tiles (the activation is then quantized inside the
  * GEMM kernel; 256 for the narrow form); two launches otherwise.  The

@@ -107,3 +107,13 @@ def test_wide_many_tiles_per_cluster(monkeypatch):
     # several tiles each, so the partial buffer is reused across tiles
     check("wide", monkeypatch, 5, 28672, 4096, fq.SCALE_FP32)
     check("wide", monkeypatch, 40, 28672, 1024, fq.SCALE_POW2)
+
+
+@pytest.mark.parametrize("M", [65, 100, 129, 200, 256])
+@pytest.mark.parametrize("N,K", [(6144, 4096), (4096, 14336), (1000, 2048)])
+def test_wide_token_groups(M, N, K, monkeypatch):
+    # M > 64 in the wide form: one block per (weight tile, group of 64
+    # tokens), the last group ragged
+    check("wide", monkeypatch, M, N, K, fq.SCALE_FP32)
+    if N == 1000:
+        check("wide", monkeypatch, M, N, K, fq.SCALE_POW2)
