@@ -171,42 +171,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The CTA's (tile, K-block) steps in order; each step's scales are
       // loaded PD - 1 steps ahead (a ring of register sets), so their latency
       // (about a microsecond under the GEMM's memory load) hides behind the
-      // steps before it.  Measured on gate+up at M = 8192: one step ahead
-      // 1.16-1.22 ms, three steps ahead 1.02-1.07 ms.  Lane l writes A rows l + 32 c and B rows l + 32 c of both
-      // 128-row halves; an absent row's scale loads as 0 (UE8M0 byte 0).
+      // steps before it.  Lane l writes A rows l + 32 c and B rows l + 32 c of
+      // both 128-row halves; an absent row's scale loads as 0 (UE8M0 byte 0).
       constexpr int NBV = ROWB ? 8 : 2;
       const int my_tiles = (int)blockIdx.x < total ? (total - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
       const int steps = my_tiles * KB;
-      auto load = [&](int s, float (&av)[4], float (&bv)[NBV]) {
-        const int t = (int)blockIdx.x + (s / KB) * (int)gridDim.x, kb = s % KB;
-        int mb, nb;
-        tile_mn(t, args, mb, nb);
-        const float *sap = args.sa + (int64_t)kb * args.ldsa + mb * BM + lane;
-        const int m = mb * BM + lane;
+      // the load cursor: tile lt (its position lmb, lnb) and K-block lkb of
+      // the next step to load; the tile's position is worked out once per
+      // tile, not per step (the raster's divisions would pace this warp)
+      int lt = (int)blockIdx.x, lkb = 0, lmb = 0, lnb = 0;
+      if (lt < total) tile_mn(lt, args, lmb, lnb);
+      auto load = [&](float (&av)[4], float (&bv)[NBV]) {
+        const float *sap = args.sa + (int64_t)lkb * args.ldsa + lmb * BM + lane;
+        const int m = lmb * BM + lane;
 #pragma unroll
         for (int c = 0; c < 4; ++c) av[c] = m + 32 * c < args.M ? __ldg(sap + 32 * c) : 0.f;
         if constexpr (ROWB) {
-          const float *sbp = args.sw + (int64_t)kb * args.ldsw;
-          const int n0 = nb * BN + lane;
+          const float *sbp = args.sw + (int64_t)lkb * args.ldsw;
+          const int n0 = lnb * BN + lane;
 #pragma unroll
           for (int c = 0; c < 8; ++c) bv[c] = n0 + 32 * c < args.N ? __ldg(sbp + n0 + 32 * c) : 0.f;
         } else {
-          const int wb0 = nb * 2, wb1 = nb * 2 + 1;
-          bv[0] = wb0 < args.NB ? __ldg(args.sw + (int64_t)wb0 * KB + kb) : 0.f;
-          bv[1] = wb1 < args.NB ? __ldg(args.sw + (int64_t)wb1 * KB + kb) : 0.f;
+          const int wb0 = lnb * 2, wb1 = lnb * 2 + 1;
+          bv[0] = wb0 < args.NB ? __ldg(args.sw + (int64_t)wb0 * KB + lkb) : 0.f;
+          bv[1] = wb1 < args.NB ? __ldg(args.sw + (int64_t)wb1 * KB + lkb) : 0.f;
+        }
+        if (++lkb == KB) {
+          lkb = 0;
+          lt += (int)gridDim.x;
+          if (lt < total) tile_mn(lt, args, lmb, lnb);
         }
       };
       constexpr int PD = ROWB ? 2 : 4;  // eight B scales per step with ROWB: fewer steps ahead
       float av[PD][4], bv[PD][NBV];
 #pragma unroll
       for (int p = 0; p < PD - 1; ++p)
-        if (p < steps) load(p, av[p], bv[p]);
+        if (p < steps) load(av[p], bv[p]);
       float (&a0)[4] = av[0];
       float (&b0)[NBV] = bv[0];
       int stage = 0;
       uint32_t phase = 0;
       for (int s = 0; s < steps; ++s) {
-        if (s + PD - 1 < steps) load(s + PD - 1, av[PD - 1], bv[PD - 1]);
+        if (s + PD - 1 < steps) load(av[PD - 1], bv[PD - 1]);
         const bool got = mbar_wait(&empty[stage], phase ^ 1, abort_flag, kSiteProducerEmpty);
         if (!__all_sync(0xffffffffu, got)) break;
         uint8_t *sf = sSF + stage * kSFBytes;

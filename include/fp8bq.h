@@ -181,11 +181,10 @@ FP8BQ_API size_t fp8bq_recalibrate_workspace_size(int n);
  *   y     bf16 [M][ldy]      output
  * Each 128-deep K-block's FP32 partial product is multiplied by
  * sa[kb][m] * sw[n/128][kb] and added into an FP32 accumulator; the result is
- * rounded to bf16.  `mode` states how the scales were made (with
- * FP8BQ_SCALE_POW2 they must be powers of two); both modes run the promotion
- * kernel.  fp8bq_gemm_ex's FP8BQ_GEMM_NATIVE_POW2 instead applies power-of-2
- * scales inside the tensor cores' native block-scaled MMA (exact products,
- * so only the FP32 summation order differs), measured slower here.
+ * rounded to bf16.  `mode` states how the scales were made; with
+ * FP8BQ_SCALE_POW2 the library uses the tensor cores' native block-scaled MMA
+ * (scales are exact powers of two, so only the FP32 summation order differs);
+ * the scales must then be powers of two.
  * Requirements: K % 128 == 0; M, N, K < 2^31; qa, qw 16-byte aligned with
  * lda, ldw >= K and multiples of 16; y 16-byte aligned with ldy >= N a
  * multiple of 8; sa 16-byte aligned with ldsa >= M a multiple of 4; sw
@@ -199,8 +198,8 @@ FP8BQ_API fp8bq_status fp8bq_gemm(const uint8_t *qa, int64_t lda, const float *s
 
 /* Variant selector for fp8bq_gemm_ex (testing and benchmarking). */
 typedef enum {
-    FP8BQ_GEMM_AUTO = 0,          /* what fp8bq_gemm does: FP8BQ_GEMM_PROMOTE for both
-                                     scale modes */
+    FP8BQ_GEMM_AUTO = 0,          /* what fp8bq_gemm does: FP8BQ_GEMM_PROMOTE for FP32 scales,
+                                     FP8BQ_GEMM_NATIVE_POW2 for POW2 scales */
     FP8BQ_GEMM_PROMOTE = 1,       /* FP32 promotion of every K-block partial, one SM per
                                      128x256 tile */
     FP8BQ_GEMM_NATIVE_POW2 = 2,   /* native block-scaled MMA (POW2 scales only) */
