@@ -478,6 +478,25 @@ def config_rows(fq, dev, peaks, gemm_ms_step):
             del qws
         del wq, wsc, oqw, osw
 
+    # --- the prefill GEMMs with power-of-2 scales (the native block-scaled
+    # MMA, what fp8bq_gemm runs for them), M = 8192, inputs quantized once
+    for name, (N, K) in wl.LLAMA8B_SHAPES.items():
+        xa = wl.activations(M_TOKENS, K, seed=3, device=dev)
+        wq_ = wl.weights(N, K, seed=4, device=dev)
+        qa2, sa2 = fq.quant_act(xa, fq.SCALE_POW2)
+        qw2, sw2 = fq.quant_weight(wq_, fq.SCALE_POW2)
+        del xa, wq_
+        y2 = torch.empty((M_TOKENS, N), dtype=torch.bfloat16, device=dev)
+        # operand copies cycled so that no call finds its inputs in L2
+        nr = rotations(M_TOKENS * K + N * K)
+        ops = [(qa2, qw2)] + [(qa2.clone(), qw2.clone()) for _ in range(nr - 1)]
+        ms = graph_ms([(lambda a=a, b=b: fq.gemm(a, sa2, b, sw2, fq.SCALE_POW2, out=y2)) for a, b in ops] *
+                      max(1, 8 // nr))
+        tf = 2.0 * M_TOKENS * N * K / (ms / 1e3) / 1e12
+        rows["gemm_pow2:" + name] = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac_fp8_peak": round(tf / fp8, 3),
+                                     "kernel": "gemm_native_kernel (block-scaled MMA, UE8M0 scale factors)"}
+        del qa2, sa2, qw2, sw2, y2, ops
+
     # --- MoE expert GEMMs (Qwen3-30B-A3B-shaped, Zipf top-8 routing)
     moe = wl.moe_layer(seed=0, device=dev)
     off = moe["offsets"].to(torch.int32).to(dev)
