@@ -11,7 +11,7 @@
 // training, block-wise E4M3 with 1x128 activation and 128x128 weight tiles.
 //
 // Both kernels are HBM-bound: 2 bytes read and 1 written per element for the
-// quantizer, 1 and 1 for the transpose.  Each block stages its tile in shared
+// quantizer, 1 and 1 for the transpose.  Both stage their tiles in shared
 // memory so that the global reads and writes are both row-contiguous.
 #include <algorithm>
 
@@ -123,43 +123,191 @@ __global__ void __launch_bounds__(256) quant_act_t_kernel(const uint16_t *__rest
 // ---------------------------------------------------------------------------
 // Transpose of a weight's codes and tile scales
 // ---------------------------------------------------------------------------
-// Block (bx, by): rows [64 by, +64) x columns [64 bx, +64) of q.  Staged as
-// 64 x 64 bytes (16-byte loads, 4 lanes per row), read back column-wise as
-// 4-byte words gathered from 4 rows, written as 16-byte rows of q^T.
-constexpr int kTB = 64;
+// Weight-code transpose: q [R][C] bytes -> q^T [C][R], 128 x 128-byte tiles.
+// Persistent CTAs (two per SM); per CTA a producer thread streams tiles in by
+// TMA through a four-stage ring (row-major, no swizzle), eight warps each take
+// one 8 x 8-byte block per thread (thread t: rows 8 (t / 16) .., columns
+// 8 (t % 16) ..), transpose it in registers with byte permutes and write it
+// into one of two output tiles in the TMA's 128-byte-swizzled layout, from
+// which a TMA store writes whole 128-byte rows of q^T.  Reads: each half-warp
+// reads one 128-byte row per instruction (conflict-free).  Writes: thread t
+// writes its eight output rows in the order rotated by (t % 16) & 7, so that
+// with the swizzle the 16 lanes of a half-warp hit 8 different 16-byte
+// chunks (two wavefronts per warp instruction, the minimum for 256 bytes).
+constexpr int kTT = 128;                 // tile edge, bytes = elements
+constexpr int kTTileBytes = kTT * kTT;   // 16 KB
+constexpr int kTStages = 4;
+constexpr int kTOut = 2;
+constexpr int kTWarps = 8;               // transposing warps; warp 8 is the producer
+constexpr int kTThreads = 32 * (kTWarps + 1);
+constexpr int kTSmemBytes = (kTStages + kTOut) * kTTileBytes + 256 + 1024;
 
-__global__ void __launch_bounds__(256) transpose_codes_kernel(const uint8_t *__restrict__ q, int64_t R, int64_t C,
-                                                              int64_t ldq, uint8_t *__restrict__ qt, int64_t ldqt) {
-  __shared__ __align__(16) uint8_t tile[kTB][kTB + 4];
-  const int64_t r0 = (int64_t)blockIdx.y * kTB, c0 = (int64_t)blockIdx.x * kTB;
-  {
-    const int r = threadIdx.x >> 2, c = (threadIdx.x & 3) * 16;  // 64 rows x 4 chunks
-    const int64_t gr = r0 + r, gc = c0 + c;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (gr < R && gc < C) v = *reinterpret_cast<const uint4 *>(q + gr * ldq + gc);
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+// 8 x 8 bytes: row i of the block is lo[i] (bytes 0-3) and hi[i] (bytes 4-7);
+// on return row i holds column i.  Three exchange stages: 4 x 4-byte blocks,
+// 2 x 2 blocks of 2 bytes, single bytes.
+__device__ __forceinline__ void transpose8x8(uint32_t (&lo)[8], uint32_t (&hi)[8]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) *reinterpret_cast<uint32_t *>(&tile[r][c + 4 * i]) = u[i];
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t t = hi[i];
+    hi[i] = lo[i + 4];
+    lo[i + 4] = t;
   }
-  __syncthreads();
-  {
-    const int oc = threadIdx.x >> 2, orr = (threadIdx.x & 3) * 16;  // output row = input column oc
-    uint32_t u[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int rr = orr + 4 * i;
-      u[i] = (uint32_t)tile[rr][oc] | ((uint32_t)tile[rr + 1][oc] << 8) | ((uint32_t)tile[rr + 2][oc] << 16) |
-             ((uint32_t)tile[rr + 3][oc] << 24);
-    }
-    const int64_t gr = c0 + oc, gc = r0 + orr;
-    if (gr < C && gc < R) *reinterpret_cast<uint4 *>(qt + gr * ldqt + gc) = make_uint4(u[0], u[1], u[2], u[3]);
+  for (int i = 0; i < 8; ++i) {
+    if ((i & 2) != 0) continue;  // rows i and i + 2 for i in {0, 1, 4, 5}
+    uint32_t a = lo[i], b = lo[i + 2];
+    lo[i] = __byte_perm(a, b, 0x5410);
+    lo[i + 2] = __byte_perm(a, b, 0x7632);
+    a = hi[i];
+    b = hi[i + 2];
+    hi[i] = __byte_perm(a, b, 0x5410);
+    hi[i + 2] = __byte_perm(a, b, 0x7632);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {  // rows i and i + 1
+    uint32_t a = lo[i], b = lo[i + 1];
+    lo[i] = __byte_perm(a, b, 0x6240);
+    lo[i + 1] = __byte_perm(a, b, 0x7351);
+    a = hi[i];
+    b = hi[i + 1];
+    hi[i] = __byte_perm(a, b, 0x6240);
+    hi[i + 1] = __byte_perm(a, b, 0x7351);
   }
 }
 
-__global__ void transpose_scales_kernel(const float *__restrict__ s, int64_t NB, int64_t KB, float *__restrict__ st) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < NB * KB; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t nb = i / KB, kb = i - nb * KB;
-    st[kb * NB + nb] = s[i];
+// rows v[s] <- v[(s + r) & 7] for r in 0..7 (three conditional rotations)
+__device__ __forceinline__ void rotate8(uint32_t (&lo)[8], uint32_t (&hi)[8], int r) {
+#pragma unroll
+  for (int bit = 0; bit < 3; ++bit) {
+    const int d = 1 << bit;
+    const bool on = (r >> bit) & 1;
+    uint32_t l2[8], h2[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      l2[s] = on ? lo[(s + d) & 7] : lo[s];
+      h2[s] = on ? hi[(s + d) & 7] : hi[s];
+    }
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      lo[s] = l2[s];
+      hi[s] = h2[s];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kTThreads, 1)
+    transpose_codes_kernel(const __grid_constant__ CUtensorMap tmIn, const __grid_constant__ CUtensorMap tmOut,
+                           int32_t nrb, int32_t ncb, const float *__restrict__ sw, float *__restrict__ swt) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sIn = base;                                 // [kTStages][128][128]
+  uint8_t *sOut = base + kTStages * kTTileBytes;       // [kTOut][128][128], 128-byte swizzle
+  uint64_t *full = reinterpret_cast<uint64_t *>(sOut + kTOut * kTTileBytes);
+  uint64_t *empty = full + kTStages;
+  uint64_t *ofree = empty + kTStages;  // [kTOut] the output buffer's previous store has read it
+  uint64_t *ofull = ofree + kTOut;     // every transposing thread has written the current output tile
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ofull + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total = nrb * ncb;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kTWarps);
+    }
+    for (int b = 0; b < kTOut; ++b) mbar_init(&ofree[b], 1);
+    mbar_init(ofull, 32 * kTWarps);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == kTWarps && lane == 0) {
+    prefetch_tensormap(&tmIn);
+    prefetch_tensormap(&tmOut);
+  }
+  __syncthreads();
+
+  if (warp == kTWarps) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- producer
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_parity = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, kSiteProducerEmpty)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[stage], kTTileBytes);
+        tma_load_2d(sIn + stage * kTTileBytes, &tmIn, &full[stage], (t % ncb) * kTT, (t / ncb) * kTT);
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == kTStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) {  // every load issued must land before the CTA may exit
+        for (int s = 0; s < kTStages; ++s)
+          if (armed >> s & 1u) mbar_wait(&full[s], (armed_parity >> s) & 1u, nullptr, kSiteDrain);
+      }
+    } else {
+      // the tiles' scales: a 128 x 128 tile is one scale block, so sw[rb][cb]
+      // goes to swt[cb][rb] (lanes 1..31, one tile each per pass)
+      for (int t = blockIdx.x + (lane - 1) * (int)gridDim.x; t < total; t += 31 * (int)gridDim.x)
+        swt[(int64_t)(t % ncb) * nrb + t / ncb] = __ldg(sw + (int64_t)(t / ncb) * ncb + t % ncb);
+    }
+  } else {
+    // ------------------------------------------------------------------ transposers
+    const int tid = threadIdx.x;
+    const int br = tid >> 4, bc = tid & 15;  // the thread's 8 x 8 block: input rows 8 br, columns 8 bc
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x, k = 0; t < total; t += gridDim.x, ++k) {
+      const bool got = mbar_wait(&full[stage], phase, abort_flag, kSiteMmaFull);
+      if (!__all_sync(0xffffffffu, got)) break;
+      uint32_t lo[8], hi[8];
+      const uint8_t *src = sIn + stage * kTTileBytes + (8 * br) * kTT + 8 * bc;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(src + i * kTT);
+        lo[i] = v.x;
+        hi[i] = v.y;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);  // the stage has been read
+      if (++stage == kTStages) {
+        stage = 0;
+        phase ^= 1;
+      }
+      transpose8x8(lo, hi);     // row j: output row 8 bc + j, bytes 8 br .. 8 br + 7
+      rotate8(lo, hi, bc & 7);  // row s: output row 8 bc + ((s + bc) & 7)
+      // output buffer b's use u = k / 2, once its store of use u - 1 has read it
+      const int b = k & 1;
+      const bool free_ok = mbar_wait(&ofree[b], (uint32_t)(((k >> 1) & 1) ^ 1), abort_flag, kSiteEpiTmemFull);
+      if (!__all_sync(0xffffffffu, free_ok)) break;
+      uint8_t *dst = sOut + b * kTTileBytes;
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const int r = 8 * bc + ((s + bc) & 7);
+        const int off = r * kTT + ((((br >> 1) ^ (r & 7)) << 4) | ((br & 1) << 3));
+        *reinterpret_cast<uint2 *>(dst + off) = make_uint2(lo[s], hi[s]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(ofull);
+      bool stored = true;
+      if (tid == 0) {
+        // every thread's part is written: store the tile, then hand the other
+        // buffer back once its store (the previous tile's) has read it
+        stored = mbar_wait(ofull, (uint32_t)(k & 1), abort_flag, kSiteEpiTmemFull);
+        if (stored) {
+          tma_store_2d(&tmOut, dst, (t / ncb) * kTT, (t % ncb) * kTT);
+          bulk_commit_group();
+          bulk_wait_group_read1();
+          if (k > 0) mbar_arrive(&ofree[b ^ 1]);  // the previous tile's store (buffer b ^ 1) is done reading
+        }
+      }
+      if (!__all_sync(0xffffffffu, stored)) break;  // warp 0 leaves as a whole
+    }
+    if (tid == 0) bulk_wait_group_read0();  // the stores have read shared memory before the CTA exits
   }
 }
 
@@ -180,15 +328,25 @@ fp8bq_status launch_quant_act_t(const void *x, int64_t M, int64_t K, int64_t ldx
 
 fp8bq_status launch_transpose_weight(const uint8_t *q, int64_t N, int64_t K, int64_t ldq, const float *sw,
                                      uint8_t *qt, int64_t ldqt, float *swt, cudaStream_t stream) {
-  const int64_t gx = (K + kTB - 1) / kTB, gy = (N + kTB - 1) / kTB;
-  if (gx > 0x7fffffff || gy > 65535) return FP8BQ_ERR_UNSUPPORTED;
-  transpose_codes_kernel<<<dim3((unsigned)gx, (unsigned)gy), 256, 0, stream>>>(q, N, K, ldq, qt, ldqt);
-  fp8bq_status st = check_launch("transpose_weight(codes)");
-  if (st != FP8BQ_OK) return st;
-  const int64_t NB = (N + 127) / 128, KB = (K + 127) / 128;
-  const int blocks = (int)std::min<int64_t>((NB * KB + 255) / 256, 1024);
-  transpose_scales_kernel<<<blocks, 256, 0, stream>>>(sw, NB, KB, swt);
-  return check_launch("transpose_weight(scales)");
+  // q [N][K] in 128 x 128-byte boxes; q^T [K][N] stored through the 128-byte swizzle
+  CUtensorMap tIn, tOut;
+  if (!make_tmap_2d(&tIn, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, (uint64_t)K, (uint64_t)N, (uint64_t)ldq, kTT, kTT,
+                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&tOut, CU_TENSOR_MAP_DATA_TYPE_UINT8, qt, (uint64_t)N, (uint64_t)K, (uint64_t)ldqt, kTT, kTT,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return FP8BQ_ERR_INVALID_ARG;
+  const int64_t nrb = (N + kTT - 1) / kTT, ncb = (K + kTT - 1) / kTT;
+  if (nrb * ncb > 0x7fffffff) return FP8BQ_ERR_UNSUPPORTED;
+  static DeviceOnce once;
+  const fp8bq_status ready = once.get([](int) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(transpose_codes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTSmemBytes);
+    return e == cudaSuccess ? FP8BQ_OK : cuda_fail(e, "cudaFuncSetAttribute(transpose_codes)");
+  });
+  if (ready != FP8BQ_OK) return ready;
+  const int grid = (int)std::min<int64_t>(nrb * ncb, 2 * (int64_t)num_sms());
+  transpose_codes_kernel<<<grid, kTThreads, kTSmemBytes, stream>>>(tIn, tOut, (int32_t)nrb, (int32_t)ncb, sw, swt);
+  return check_launch("transpose_weight");
 }
 
 }  // namespace fp8bq
