@@ -142,6 +142,11 @@ constexpr int kTWarps = 8;               // transposing warps; warp 8 is the pro
 constexpr int kTThreads = 32 * (kTWarps + 1);
 constexpr int kTSmemBytes = (kTStages + kTOut) * kTTileBytes + 256 + 1024;
 
+// At most one bulk group of this thread still reading its shared-memory source.
+__device__ __forceinline__ void bulk_wait_group_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 // 8 x 8 bytes: row i of the block is lo[i] (bytes 0-3) and hi[i] (bytes 4-7);
 // on return row i holds column i.  Three exchange stages: 4 x 4-byte blocks,
 // 2 x 2 blocks of 2 bytes, single bytes.
