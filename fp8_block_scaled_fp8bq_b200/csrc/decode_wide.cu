@@ -1,6 +1,7 @@
 // Decode-shaped block-scaled FP8 linear, wide form, for sm_100a:
-// Y[M,N] = q(X)[M,K] . W[N,K]^T for M <= 64 tokens, with the activation
-// quantized in 1x128 tiles and W pre-quantized in 128x128 tiles.
+// Y[M,N] = q(X)[M,K] . W[N,K]^T for M <= 256 tokens (in groups of 64), with
+// the activation quantized in 1x128 tiles and W pre-quantized in 128x128
+// tiles.
 //
 // Method: "NVIDIA NeMo RL Achieves 48% Speedup With End-to-End FP8 Precision
 // Training", section "Technical breakthrough": FP8 is applied in generation as
@@ -11,19 +12,21 @@
 // The tokens are the MMA's 128-row operand (A) and 256 weight rows its N
 // dimension: one tcgen05.mma 128x256x32 covers twice the weight bytes of a
 // 128-weight-row MMA at the same issue cost, so the MMA no longer paces the
-// weight stream.  Only A's first NT rows (NT = M rounded up to 16, 32 or 64)
-// hold tokens; the MMA reads the rest of its 128 rows from whatever follows
-// in shared memory (the layout keeps that window inside the allocation) and
-// the matching accumulator rows (TMEM lanes NT..127) are never read back.
+// weight stream.  Only A's first NT rows (NT = M, or a group's 64 tokens,
+// rounded up to 16, 32 or 64) hold tokens; the MMA reads the rest of its 128
+// rows from whatever follows in shared memory (the layout keeps that window
+// inside the allocation) and the matching accumulator rows (TMEM lanes
+// NT..127) are never read back.
 //
 // A work item is (256-row weight tile t, 128-deep K-block kb): its 32 KB
 // weight tile arrives by TMA, 4 MMAs accumulate into one of two 256-column
 // TMEM buffers, and the epilogue warps of the token lanes (thread = token,
-// 128 weight rows each) add P * (sa[kb][token] * sw[nb][kb]) into FP32
-// registers, nb being the 128-row weight block of that half of the tile.
+// 64 weight rows each) add P * (sa[kb][token] * sw[nb][kb]) into FP32
+// registers, nb being the 128-row weight block of those rows.
 //
 // Split over K in thread-block clusters of S CTAs (S up to 16): cluster c
-// owns tiles c, c + C, ...; rank r takes K-blocks r, r + S, ... of each.  At
+// owns blocks c, c + C, ... (a block is a weight tile and a group of up to 64
+// tokens); rank r takes K-blocks r, r + S, ... of each.  At
 // the end of a tile every rank sends each 4-column piece of its FP32 partial
 // (NT x 256) to the rank that owns those columns (rank r owns slice r of the
 // 256 columns), with st.async stores into the owner's shared memory that
@@ -109,8 +112,9 @@ struct WCfg {
   // descriptor spans from any code tile stays inside the weight stages that
   // follow; the weight stages; the activation scales; the receive buffer of
   // the cross-CTA sum (S > 1); the staged weight scales; the barriers.
-  // a resident K-block's codes: the M token rows rounded up to the 8-row
-  // swizzle atom (the A window's further rows read the next K-blocks' codes)
+  //
+  // A resident K-block's codes: the M token rows rounded up to the 8-row
+  // swizzle atom (the A window's further rows read the next K-blocks' codes).
   static __host__ __device__ int res_tile_bytes(int M) { return (M + 7) / 8 * 1024; }
   static __host__ __device__ int x_bytes(int nst, int nres, int M) {
     return kRes ? nres * res_tile_bytes(M) : nst * kXBytes;
